@@ -1,0 +1,239 @@
+/*
+ * rm_attn.h -- C ABI of librm_attn.so: the single-GPU (B200, sm_100a) hot path
+ * of ring / striped / Ulysses context-parallel attention.
+ *
+ * Sources of the operations (web pages; section in brackets):
+ *  - exact attention softmax(Q K^T / sqrt(d)) V
+ *      [Mosaic: Sharding Attention Across GPUs..., "The Problem"]
+ *  - computing it one KV chunk at a time and normalising at the end, with the
+ *    softmax rescaling trick
+ *      [Mosaic, "How Ring Attention Works"; Ring Attention & Friends,
+ *       "Flash Attention - Tiling with the Softmax Rescaling Trick"]
+ *  - LSE merge of partial results, contiguous / head_tail (zigzag) layouts,
+ *    the reverse-ring backward, the Ulysses head all-to-all
+ *      [ringmaster (axolotl-ringmaster 0.2.0), "Why", "Status", "Layout"]
+ *  - striped layout (token t on rank t mod P)
+ *      [Ring Attention & Friends, "Striped Attention"]
+ *
+ * Conventions shared by every entry point
+ *  - Tokens-major layout [B, N, H, d] ("bshd"): the d axis is contiguous
+ *    (stride 1); batch, token and head strides are given in ELEMENTS through
+ *    rm_tensor.  LSE / delta vectors are dense fp32 [B, H, N] (N fastest).
+ *  - "Rank-major order": a sequence of P*L tokens stored as rank 0's L local
+ *    tokens, then rank 1's, ...  Local token j of rank r sits at global
+ *    position pos(r, j):
+ *        contiguous  pos = r*L + j
+ *        zigzag      C = N/(2P); j < C: r*C + j;  else (2P-1-r)*C + (j-C)
+ *        striped     pos = j*P + r
+ *  - Causal masking: key u is visible to query t iff pos(u) <= pos(t).
+ *  - Grouped-query attention: query head h reads KV head h / (Hq/Hkv).
+ *  - scale <= 0 selects 1/sqrt(d) with d the true head dimension.
+ *  - LSE is the natural log of the softmax normaliser; a row with no visible
+ *    key has O = 0 and LSE = -inf.
+ *  - Ownership: the caller owns every buffer, the workspace included; the
+ *    library never allocates device memory and keeps no per-call state.
+ *  - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t,
+ *    NULL = legacy default stream).  Argument errors are detected on the host
+ *    before anything is launched and return RM_ERR_INVALID_ARG /
+ *    RM_ERR_UNSUPPORTED / RM_ERR_WORKSPACE; launch failures return
+ *    RM_ERR_CUDA.  Device-side bounded waits that expire record
+ *    RM_ERR_TIMEOUT in a device status word read by rm_get_device_status.
+ *    rm_last_error() gives a thread-local one-line reason for the last
+ *    non-OK status.
+ *  - Alignment: device pointers 16-byte aligned; every stride times the
+ *    element size a multiple of 16 bytes (bf16 attention calls); other calls
+ *    state their own rule.
+ *  - Aliasing: outputs never alias inputs, except where an entry point says so.
+ */
+#ifndef RM_ATTN_H
+#define RM_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Everything declared here is exported from librm_attn.so; the library is
+ * built with hidden visibility otherwise. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef enum {
+  RM_OK = 0,
+  RM_ERR_INVALID_ARG = 1,  /* bad pointer / shape / stride / enum            */
+  RM_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement    */
+  RM_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
+  RM_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed            */
+  RM_ERR_TIMEOUT = 5       /* a device-side bounded wait expired             */
+} rm_status;
+
+typedef enum { RM_F32 = 0, RM_BF16 = 1 } rm_dtype;
+
+typedef enum {
+  RM_LAYOUT_CONTIGUOUS = 0,
+  RM_LAYOUT_ZIGZAG = 1,
+  RM_LAYOUT_STRIPED = 2
+} rm_layout;
+
+/* Forward ring execution mode. */
+typedef enum {
+  RM_RING_FUSED = 0,    /* one persistent launch; running softmax state carried
+                           across KV shards (the merge happens in registers) */
+  RM_RING_STEPWISE = 1  /* per ring step one block launch per rank writing fp32
+                           partials to the workspace, then rm_lse_merge */
+} rm_ring_mode;
+
+/* A strided [B, N, H, d] view; strides in elements, d stride is 1. */
+typedef struct {
+  void* ptr;
+  int64_t stride_b;
+  int64_t stride_n;
+  int64_t stride_h;
+} rm_tensor;
+
+/* One attention problem: B sequences of N tokens split over P virtual ranks
+ * (L = N / P tokens each) laid out by `layout`.  d is the true head
+ * dimension.  bf16 supports d in {24, 32, 64, 128} (24 is zero-padded to 32
+ * on chip); fp32 supports d % 4 == 0, d <= 128. */
+typedef struct {
+  rm_dtype dtype;
+  int B;
+  int Hq;
+  int Hkv;
+  int d;
+  int64_t N;
+  int P;
+  rm_layout layout;
+  int causal;
+  float scale;        /* <= 0: 1/sqrt(d) */
+  rm_ring_mode mode;  /* rm_ring_attn_fwd only */
+} rm_attn_desc;
+
+/* ---- block level: one Q shard against one KV shard ---------------------- */
+
+/* Attention of rank q_rank's query shard against rank kv_rank's KV shard
+ * [Mosaic, "How Ring Attention Works": one step's partial result].
+ *   q  [B, L, Hq, d] (desc->dtype), the L tokens of q_rank in local order
+ *   k, v [B, L, Hkv, d], the L tokens of kv_rank in local order
+ *   o  [B, L, Hq, d] written: fp32 if o_f32 != 0, else desc->dtype
+ *   lse dense fp32 [B, Hq, L] written
+ * Keys with pos > pos(query) are masked when desc->causal.  A shard pair with
+ * no visible key writes O = 0, LSE = -inf.  L may have a ragged tail (any
+ * L >= 1).  desc->mode is ignored. */
+rm_status rm_attn_block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank,
+                            rm_tensor q, rm_tensor k, rm_tensor v,
+                            rm_tensor o, int o_f32, float* lse, void* stream);
+
+/* Backward contribution of one (q_rank, kv_rank) pair [ringmaster, "Status":
+ * flash-style reverse-ring backward; the derivative of the definition]:
+ *   P_tu = exp(s_tu - lse_final_t);  dP = dO V^T;  dS = P o (dP - delta)
+ *   dq_acc += scale dS K;  dk_acc += scale dS^T Q;  dv_acc += P^T dO
+ * lse_final / delta: dense fp32 [B, Hq, L] of the query shard (the FINAL LSE
+ * of the whole ring, and delta_t = dO_t . O_t of the final O).
+ * dq_acc [B, L, Hq, d], dk_acc / dv_acc [B, L, Hkv, d]: fp32 accumulators,
+ * read-modify-written (+=).  dK/dV of a KV head sum over its query heads. */
+rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank,
+                            rm_tensor q, rm_tensor k, rm_tensor v, rm_tensor dout,
+                            const float* lse_final, const float* delta,
+                            rm_tensor dq_acc, rm_tensor dk_acc, rm_tensor dv_acc,
+                            void* stream);
+
+/* delta[b, h, t] = sum_c dout[b, t, h, c] * o[b, t, h, c] (fp32 accumulate),
+ * the row term of the softmax derivative computed from the FINAL output.
+ * o / dout in `dtype`, [B, N, H, d]; delta dense fp32 [B, H, N]. */
+rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
+                                 rm_tensor o, rm_tensor dout, float* delta,
+                                 void* stream);
+
+/* ---- LSE merge ---------------------------------------------------------- */
+
+/* Merge n_parts partial results [ringmaster, "Layout": ring/merge.py, the
+ * online-softmax LSE merge; formula is the exact identity of the LSE]:
+ *   m = max_i lse_i;  LSE = m + ln sum_i exp(lse_i - m);
+ *   O = sum_i exp(lse_i - LSE) O_i
+ * Parts with lse = -inf get weight 0; if all are -inf, O = 0, LSE = -inf.
+ *   o_parts[i]  fp32 [B, Nq, H, d] (strided)     lse_parts[i] fp32 [B, H, Nq]
+ *   o_out       out_dtype [B, Nq, H, d]          lse_out      fp32 [B, H, Nq]
+ * 1 <= n_parts <= 16; d % 4 == 0, d <= 128; strides multiples of 4 elements.
+ * o_out may alias o_parts[0] exactly (in-place merge) when out_dtype is fp32;
+ * lse_out may alias lse_parts[0]. */
+rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d,
+                       int n_parts, const rm_tensor* o_parts,
+                       const float* const* lse_parts, rm_tensor o_out,
+                       float* lse_out, void* stream);
+
+/* ---- ring driver over P virtual ranks ----------------------------------- */
+
+/* Workspace bytes rm_ring_attn_fwd (backward = 0) or rm_ring_attn_bwd
+ * (backward = 1) needs for *desc; 0 is a valid answer. */
+rm_status rm_ring_workspace_size(const rm_attn_desc* desc, int backward,
+                                 size_t* bytes);
+
+/* Ring forward [Mosaic, "How Ring Attention Works"]: for every rank r and
+ * step k = 0..P-1, rank r attends to KV shard (r - k) mod P; the partials are
+ * merged by the LSE merge.  q [B, N, Hq, d], k/v [B, N, Hkv, d] in rank-major
+ * order; o [B, N, Hq, d] (desc->dtype) and lse fp32 [B, Hq, N] in rank-major
+ * order.  Shard pairs (and tiles) that the causal mask empties are skipped.
+ * ws: 256-byte aligned device buffer of rm_ring_workspace_size(desc, 0). */
+rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
+                           rm_tensor v, rm_tensor o, float* lse, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Ring backward: delta from the final (o, dout), then every (query shard,
+ * KV shard) pair's contribution accumulated in fp32, KV shards visiting the
+ * ranks in reverse ring order; dq/dk/dv written in desc->dtype, rank-major.
+ * o, lse: the outputs of rm_ring_attn_fwd.  ws: rm_ring_workspace_size(desc, 1)
+ * bytes, 256-byte aligned. */
+rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
+                           rm_tensor v, rm_tensor o, const float* lse,
+                           rm_tensor dout, rm_tensor dq, rm_tensor dk,
+                           rm_tensor dv, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- bit-exact layout transforms ---------------------------------------- */
+
+/* Global token order <-> rank-major order (see pos(r, j) above) of a dense
+ * [B, N, H, d] tensor of `dtype`.  inverse = 0: out[b, r*L + j] = in[b, pos];
+ * inverse = 1: out[b, pos] = in[b, r*L + j].  Bit copy.  N % P == 0 (and
+ * N % 2P == 0 for zigzag).  in and out must not overlap. */
+rm_status rm_layout_permute(rm_dtype dtype, int B, int64_t N, int H, int d,
+                            rm_layout layout, int P, int inverse,
+                            const void* in, void* out, void* stream);
+
+/* Ulysses sequence <-> head repack as a local pack [ringmaster, "Why": the
+ * all-to-all on the head dim, capped by the head count].
+ * head_to_seq = 0 (seq -> head):
+ *   in  [P][N_local][H][d]      (rank s's sequence shard of all heads)
+ *   out [P][P*N_local][H/P][d]  out[r][s*N_local + t][h] = in[s][t][r*H/P + h]
+ * head_to_seq = 1 is the inverse (in and out swap roles).  Bit copy; dense
+ * tensors; H % P == 0.  in and out must not overlap. */
+rm_status rm_seq_head_repack(rm_dtype dtype, int P, int64_t N_local, int H,
+                             int d, int head_to_seq, const void* in, void* out,
+                             void* stream);
+
+/* ---- status ------------------------------------------------------------- */
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: RM_ERR_TIMEOUT if a bounded wait expired in any kernel
+ * since the last call, RM_ERR_CUDA if the synchronisation failed, else RM_OK. */
+rm_status rm_get_device_status(void* stream);
+
+const char* rm_status_string(rm_status s);
+const char* rm_last_error(void);
+
+/* Test hook for the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing arrives at, giving up after `spin_limit` polls, and records
+ * RM_ERR_TIMEOUT in the device status word.  Faults and hangs nothing. */
+rm_status rm_debug_expire_wait(uint32_t spin_limit, void* stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RM_ATTN_H */

@@ -1,0 +1,92 @@
+// Shared device/host helpers of librm_attn.so (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/rm_attn.h"
+
+namespace rm {
+
+// ---- token layouts --------------------------------------------------------
+// Global position of local token j of rank r (ringmaster "Layout":
+// contiguous shard / head_tail balancer; Ring Attention & Friends, "Striped
+// Attention").  L = N / P tokens per rank; C = N / (2P) zigzag chunk.
+struct LayoutMap {
+  int layout;   // rm_layout
+  int P;
+  int64_t L;
+  int64_t C;
+
+  __host__ __device__ __forceinline__ int64_t pos(int r, int64_t j) const {
+    if (layout == RM_LAYOUT_CONTIGUOUS) return (int64_t)r * L + j;
+    if (layout == RM_LAYOUT_STRIPED) return j * P + r;
+    return j < C ? (int64_t)r * C + j : (int64_t)(2 * P - 1 - r) * C + (j - C);
+  }
+
+  // pos(r, j) is strictly increasing in j for every layout (the second
+  // zigzag chunk, from (2P-1-r)*C, lies above the first, which ends at
+  // (r+1)*C - 1), so under the causal rule the keys of shard s visible to a
+  // query at global position t are a prefix of the shard: local keys
+  // [0, visible_count(s, t)).
+  __host__ __device__ __forceinline__ int64_t visible_count(int s, int64_t t) const {
+    if (layout == RM_LAYOUT_CONTIGUOUS) return clamp64(t - (int64_t)s * L + 1, 0, L);
+    if (layout == RM_LAYOUT_STRIPED) return t < s ? 0 : min64((t - s) / P + 1, L);
+    int64_t n1 = clamp64(t - (int64_t)s * C + 1, 0, C);
+    int64_t n2 = clamp64(t - (int64_t)(2 * P - 1 - s) * C + 1, 0, C);
+    return n1 + n2;
+  }
+
+  __host__ __device__ __forceinline__ static int64_t min64(int64_t a, int64_t b) {
+    return a < b ? a : b;
+  }
+  __host__ __device__ __forceinline__ static int64_t clamp64(int64_t x, int64_t lo, int64_t hi) {
+    return x < lo ? lo : (x > hi ? hi : x);
+  }
+};
+
+__host__ __device__ inline LayoutMap make_layout(int layout, int64_t N, int P) {
+  LayoutMap m;
+  m.layout = layout;
+  m.P = P;
+  m.L = N / P;
+  m.C = N / (2 * P);
+  return m;
+}
+
+// ---- device status word (bounded-wait expiry) ------------------------------
+enum : uint32_t { kStatusTimeout = 1u };
+
+// Host: address of the status word on the current device.
+unsigned int* status_word();
+
+__device__ __forceinline__ void report_timeout(unsigned int* status) {
+  if (status) atomicOr(status, kStatusTimeout);
+}
+
+// ---- small math helpers -----------------------------------------------------
+__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+}  // namespace rm

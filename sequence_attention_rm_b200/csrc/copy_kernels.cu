@@ -1,0 +1,132 @@
+// Bit-exact layout transforms: global <-> rank-major token permutation and
+// the Ulysses sequence <-> head repack.  Both are row gathers of contiguous
+// byte runs, done with 16-byte vector loads/stores where the run length and
+// the pointers allow it.  HBM-bound: algorithmic traffic is one read and one
+// write of the tensor.
+#include "common.cuh"
+#include "internal.h"
+
+namespace rm {
+
+namespace {
+
+// Copies `rows` runs of `run_vecs` vectors.  Run i goes from src + so(i) to
+// dst + dof(i) (byte offsets from the map).  One warp owns one run at a time
+// (the map is evaluated once per run, not per vector); each lane keeps UNROLL
+// independent 16/4/2-byte loads in flight before storing them.
+template <typename VEC, int UNROLL, typename Map>
+__global__ void __launch_bounds__(256) gather_runs_kernel(const char* __restrict__ src,
+                                                          char* __restrict__ dst, int64_t rows,
+                                                          int run_vecs, Map map) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    int64_t so, dof;
+    map(row, so, dof);
+    const VEC* s = reinterpret_cast<const VEC*>(src + so);
+    VEC* d = reinterpret_cast<VEC*>(dst + dof);
+    for (int v0 = 0; v0 < run_vecs; v0 += 32 * UNROLL) {
+      VEC buf[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        int v = v0 + u * 32 + lane;
+        if (v < run_vecs) buf[u] = __ldcs(s + v);
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        int v = v0 + u * 32 + lane;
+        if (v < run_vecs) __stcs(d + v, buf[u]);
+      }
+    }
+  }
+}
+
+// Row map of the token permutation: output row (b, r*L + j) <- input row
+// (b, pos(r, j)) (forward) or the reverse.
+struct PermuteMap {
+  LayoutMap lay;
+  int64_t N;
+  int64_t row_bytes;
+  int inverse;
+  __device__ __forceinline__ void operator()(int64_t row, int64_t& so, int64_t& dof) const {
+    int64_t b = row / N;
+    int64_t n = row - b * N;           // rank-major index
+    int r = (int)(n / lay.L);
+    int64_t j = n - (int64_t)r * lay.L;
+    int64_t g = lay.pos(r, j);         // global index
+    int64_t rm_off = (b * N + n) * row_bytes;
+    int64_t gl_off = (b * N + g) * row_bytes;
+    if (inverse) { so = rm_off; dof = gl_off; }
+    else { so = gl_off; dof = rm_off; }
+  }
+};
+
+// Run map of the repack, seen as [Ntot][P][run] <-> [P][Ntot][run] with
+// Ntot = P * N_local and run = (H/P) * d elements:
+//   seq -> head: out[r][n] <- in[n][r];   head -> seq: out[n][r] <- in[r][n].
+struct RepackMap {
+  int64_t ntot;
+  int P;
+  int64_t run_bytes;
+  int head_to_seq;
+  __device__ __forceinline__ void operator()(int64_t row, int64_t& so, int64_t& dof) const {
+    // row enumerates the destination runs in destination order
+    if (!head_to_seq) {
+      int64_t r = row / ntot, n = row - r * ntot;
+      so = (n * P + r) * run_bytes;
+      dof = row * run_bytes;
+    } else {
+      int64_t n = row / P, r = row - n * P;
+      so = (r * ntot + n) * run_bytes;
+      dof = row * run_bytes;
+    }
+  }
+};
+
+template <typename Map>
+cudaError_t launch_gather(const void* src, void* dst, int64_t rows, int64_t run_bytes, Map map,
+                          cudaStream_t stream) {
+  if (rows == 0 || run_bytes == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t warps_cap = (int64_t)num_sms() * 16 * (threads / 32);
+  const int64_t warps = rows < warps_cap ? rows : warps_cap;
+  const int blocks = (int)((warps + (threads / 32) - 1) / (threads / 32));
+  uintptr_t a = (uintptr_t)src | (uintptr_t)dst;
+  if (run_bytes % 16 == 0 && a % 16 == 0) {
+    gather_runs_kernel<uint4, 4, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)(run_bytes / 16), map);
+  } else if (run_bytes % 4 == 0 && a % 4 == 0) {
+    gather_runs_kernel<uint32_t, 8, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)(run_bytes / 4), map);
+  } else {
+    gather_runs_kernel<uint16_t, 8, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)(run_bytes / 2), map);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_layout_permute(int esize, int B, int64_t N, int H, int d, int layout, int P,
+                                  int inverse, const void* in, void* out, cudaStream_t stream) {
+  PermuteMap m;
+  m.lay = make_layout(layout, N, P);
+  m.N = N;
+  m.row_bytes = (int64_t)H * d * esize;
+  m.inverse = inverse;
+  return launch_gather(in, out, (int64_t)B * N, m.row_bytes, m, stream);
+}
+
+cudaError_t launch_seq_head_repack(int esize, int P, int64_t n_local, int H, int d,
+                                   int head_to_seq, const void* in, void* out,
+                                   cudaStream_t stream) {
+  RepackMap m;
+  m.ntot = (int64_t)P * n_local;
+  m.P = P;
+  m.run_bytes = (int64_t)(H / P) * d * esize;
+  m.head_to_seq = head_to_seq;
+  return launch_gather(in, out, m.ntot * P, m.run_bytes, m, stream);
+}
+
+}  // namespace rm

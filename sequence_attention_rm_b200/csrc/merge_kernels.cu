@@ -1,0 +1,238 @@
+// Row-wise HBM-bound kernels: the LSE merge of partial (O, LSE) results, the
+// backward preprocess (delta = rowsum(dO * O)) and the fp32 -> output-dtype
+// finalize.  A "row" is one (b, t, h) vector of d values; a group of
+// d/4 lanes (rounded up to a power of two) owns a row and moves it with
+// 16-byte fp32 vectors.  Rows are enumerated (b, h, t) with t fastest so that
+// the per-row LSE / delta scalars of neighbouring warps share sectors.
+#include "common.cuh"
+#include "internal.h"
+
+namespace rm {
+
+namespace {
+
+struct RowGroup {
+  int lanes;      // lanes per row (power of two, <= 32)
+  int rows_per_warp;
+};
+
+inline RowGroup row_group(int d) {
+  int need = (d + 3) / 4;
+  int lanes = 1;
+  while (lanes < need) lanes <<= 1;
+  return RowGroup{lanes, 32 / lanes};
+}
+
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// ---- LSE merge --------------------------------------------------------------
+template <typename OutT, int NPARTS>
+__global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, int rows_per_warp) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes;      // row slot within the warp
+  const int col = (lane % lanes) * 4;
+  const int64_t rows = (int64_t)a.B * a.H * a.Nq;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int nparts = NPARTS > 0 ? NPARTS : a.n_parts;
+  for (int64_t base = warp0 * rows_per_warp; base < rows; base += nwarps * rows_per_warp) {
+    const int64_t row = base + sub;
+    if (row >= rows) continue;
+    const int64_t t = row % a.Nq;
+    const int64_t bh = row / a.Nq;
+    const int h = (int)(bh % a.H);
+    const int b = (int)(bh / a.H);
+    const int64_t lidx = bh * a.lse_ld + t;
+    float l[kMaxMergeParts];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxMergeParts; ++i) {
+      if (i < nparts) {
+        l[i] = a.lse_ptr[i][lidx];
+        m = fmaxf(m, l[i]);
+      }
+    }
+    const bool active = col < a.d;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lse;
+    if (m == -INFINITY) {
+      lse = -INFINITY;
+    } else {
+      float w[kMaxMergeParts];
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxMergeParts; ++i) {
+        if (i < nparts) {
+          w[i] = expf(l[i] - m);  // exp(-inf) = 0 for empty partials
+          sum += w[i];
+        }
+      }
+      const float inv = 1.0f / sum;
+      lse = m + logf(sum);
+      if (active) {
+        float4 x[kMaxMergeParts];
+#pragma unroll
+        for (int i = 0; i < kMaxMergeParts; ++i)
+          if (i < nparts)
+            x[i] = load4(a.o_ptr[i] + b * a.o_sb[i] + t * a.o_sn[i] + h * a.o_sh[i] + col);
+#pragma unroll
+        for (int i = 0; i < kMaxMergeParts; ++i) {
+          if (i < nparts && w[i] != 0.f) {
+            const float c = w[i] * inv;
+            acc.x = fmaf(c, x[i].x, acc.x);
+            acc.y = fmaf(c, x[i].y, acc.y);
+            acc.z = fmaf(c, x[i].z, acc.z);
+            acc.w = fmaf(c, x[i].w, acc.w);
+          }
+        }
+      }
+    }
+    if (active) {
+      OutT* out = reinterpret_cast<OutT*>(a.out) + b * a.out_sb + t * a.out_sn + h * a.out_sh + col;
+      store4(out, acc);
+    }
+    if ((lane % lanes) == 0) a.lse_out[lidx] = lse;
+  }
+}
+
+// ---- backward preprocess ----------------------------------------------------
+template <typename InT>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(int B, int64_t N, int H, int d,
+                                                             rm_tensor o, rm_tensor dout,
+                                                             float* __restrict__ delta,
+                                                             float* __restrict__ zero_fill,
+                                                             int lanes, int rows_per_warp) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes;
+  const int col = (lane % lanes) * 4;
+  const int64_t rows = (int64_t)B * H * N;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t base = warp0 * rows_per_warp; base < rows; base += nwarps * rows_per_warp) {
+    const int64_t row = base + sub;
+    const bool valid = row < rows;
+    float s = 0.f;
+    int64_t t = 0, bh = 0;
+    if (valid) {
+      t = row % N;
+      bh = row / N;
+      const int h = (int)(bh % H);
+      const int b = (int)(bh / H);
+      if (col < d) {
+        float4 x = load4(reinterpret_cast<const InT*>(o.ptr) + b * o.stride_b + t * o.stride_n +
+                         h * o.stride_h + col);
+        float4 y = load4(reinterpret_cast<const InT*>(dout.ptr) + b * dout.stride_b +
+                         t * dout.stride_n + h * dout.stride_h + col);
+        s = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+        if (zero_fill) store4(zero_fill + row * d + col, make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+    }
+    for (int off = lanes >> 1; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (valid && (lane % lanes) == 0) delta[row] = s;
+  }
+}
+
+// ---- fp32 -> output dtype ---------------------------------------------------
+template <typename OutT>
+__global__ void __launch_bounds__(256) convert_f32_kernel(int B, int64_t N, int H, int d,
+                                                          rm_tensor in, rm_tensor out, int lanes,
+                                                          int rows_per_warp) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes;
+  const int col = (lane % lanes) * 4;
+  const int64_t rows = (int64_t)B * N * H;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t base = warp0 * rows_per_warp; base < rows; base += nwarps * rows_per_warp) {
+    const int64_t row = base + sub;  // (b, t, h) with h fastest
+    if (row >= rows || col >= d) continue;
+    const int h = (int)(row % H);
+    const int64_t bt = row / H;
+    const int64_t t = bt % N;
+    const int b = (int)(bt / N);
+    float4 x = load4(reinterpret_cast<const float*>(in.ptr) + b * in.stride_b + t * in.stride_n +
+                     h * in.stride_h + col);
+    store4(reinterpret_cast<OutT*>(out.ptr) + b * out.stride_b + t * out.stride_n +
+               h * out.stride_h + col,
+           x);
+  }
+}
+
+int grid_for_rows(int64_t rows, int rows_per_warp) {
+  int64_t warps = (rows + rows_per_warp - 1) / rows_per_warp;
+  int64_t blocks = (warps + 7) / 8;
+  int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
+template <typename OutT>
+cudaError_t merge_dispatch(const MergeArgs& a, RowGroup g, int grid, cudaStream_t s) {
+  switch (a.n_parts) {
+    case 2: lse_merge_kernel<OutT, 2><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 4: lse_merge_kernel<OutT, 4><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 8: lse_merge_kernel<OutT, 8><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    default: lse_merge_kernel<OutT, 0><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stream) {
+  const int64_t rows = (int64_t)a.B * a.H * a.Nq;
+  if (rows == 0) return cudaSuccess;
+  RowGroup g = row_group(a.d);
+  int grid = grid_for_rows(rows, g.rows_per_warp);
+  return out_bf16 ? merge_dispatch<__nv_bfloat16>(a, g, grid, stream)
+                  : merge_dispatch<float>(a, g, grid, stream);
+}
+
+cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, rm_tensor o,
+                                  rm_tensor dout, float* delta, float* zero_fill,
+                                  cudaStream_t stream) {
+  const int64_t rows = (int64_t)B * H * N;
+  if (rows == 0) return cudaSuccess;
+  RowGroup g = row_group(d);
+  int grid = grid_for_rows(rows, g.rows_per_warp);
+  if (in_bf16)
+    bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        B, N, H, d, o, dout, delta, zero_fill, g.lanes, g.rows_per_warp);
+  else
+    bwd_preprocess_kernel<float><<<grid, 256, 0, stream>>>(B, N, H, d, o, dout, delta, zero_fill,
+                                                           g.lanes, g.rows_per_warp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_f32(int out_bf16, int B, int64_t N, int H, int d, rm_tensor in,
+                               rm_tensor out, cudaStream_t stream) {
+  const int64_t rows = (int64_t)B * N * H;
+  if (rows == 0) return cudaSuccess;
+  RowGroup g = row_group(d);
+  int grid = grid_for_rows(rows, g.rows_per_warp);
+  if (out_bf16)
+    convert_f32_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes,
+                                                                g.rows_per_warp);
+  else
+    convert_f32_kernel<float><<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes,
+                                                        g.rows_per_warp);
+  return cudaGetLastError();
+}
+
+}  // namespace rm

@@ -1,0 +1,524 @@
+// C ABI of librm_attn.so: argument validation, workspace carving and kernel
+// dispatch.  Every entry point validates on the host and returns before any
+// launch on a bad argument; no entry point allocates device memory.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_attn.h"
+
+namespace rm {
+
+__device__ unsigned int g_device_status;  // bit kStatusTimeout: a bounded wait expired
+
+namespace {
+thread_local std::string t_last_error;
+
+rm_status fail(rm_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+rm_status fail(rm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+rm_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(RM_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_sms[kMaxDevices];
+unsigned int* g_status_ptr[kMaxDevices];
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return dev < 0 || dev >= kMaxDevices ? 0 : dev;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int esize_of(rm_dtype t) { return t == RM_BF16 ? 2 : 4; }
+
+rm_status check_desc(const rm_attn_desc* d) {
+  if (!d) return fail(RM_ERR_INVALID_ARG, "desc is NULL");
+  if (d->dtype != RM_F32 && d->dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (d->B < 0 || d->N < 0 || d->P < 1 || d->Hq < 1 || d->Hkv < 1)
+    return fail(RM_ERR_INVALID_ARG, "bad sizes (B=%d N=%lld P=%d Hq=%d Hkv=%d)", d->B,
+                (long long)d->N, d->P, d->Hq, d->Hkv);
+  if (d->Hq % d->Hkv) return fail(RM_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (d->layout != RM_LAYOUT_CONTIGUOUS && d->layout != RM_LAYOUT_ZIGZAG &&
+      d->layout != RM_LAYOUT_STRIPED)
+    return fail(RM_ERR_INVALID_ARG, "bad layout");
+  if (d->N % d->P) return fail(RM_ERR_INVALID_ARG, "N %% P != 0");
+  if (d->layout == RM_LAYOUT_ZIGZAG && d->N % (2 * (int64_t)d->P))
+    return fail(RM_ERR_INVALID_ARG, "zigzag needs N %% 2P == 0");
+  if (d->mode != RM_RING_FUSED && d->mode != RM_RING_STEPWISE)
+    return fail(RM_ERR_INVALID_ARG, "bad ring mode");
+  if (!(d->scale == d->scale) || isinf(d->scale)) return fail(RM_ERR_INVALID_ARG, "bad scale");
+  if (d->dtype == RM_BF16) {
+    if (!tc_supported_head_dim(d->d))
+      return fail(RM_ERR_UNSUPPORTED, "bf16 head dim %d not in {24, 32, 64, 128}", d->d);
+  } else {
+    if (d->d < 4 || d->d > 128 || d->d % 4)
+      return fail(RM_ERR_UNSUPPORTED, "fp32 head dim %d: need d %% 4 == 0, d <= 128", d->d);
+  }
+  return RM_OK;
+}
+
+float eff_scale(const rm_attn_desc* d) {
+  return d->scale > 0.f ? d->scale : 1.0f / sqrtf((float)d->d);
+}
+
+// A strided [B, rows, H, d] operand: pointer and strides must keep every row
+// 16-byte aligned (TMA and vector access).
+rm_status check_tensor(const char* name, rm_tensor t, int esize, int64_t rows, int heads,
+                       int d) {
+  if (rows == 0) return RM_OK;
+  if (!t.ptr) return fail(RM_ERR_INVALID_ARG, "%s: NULL pointer", name);
+  if (!aligned16(t.ptr)) return fail(RM_ERR_INVALID_ARG, "%s: pointer not 16-byte aligned", name);
+  if (t.stride_b < 0 || t.stride_n <= 0 || t.stride_h < 0)
+    return fail(RM_ERR_INVALID_ARG, "%s: negative / zero stride", name);
+  if ((t.stride_b * esize) % 16 || (t.stride_n * esize) % 16 || (t.stride_h * esize) % 16)
+    return fail(RM_ERR_INVALID_ARG, "%s: strides * element size must be multiples of 16 bytes",
+                name);
+  if (heads > 1 && t.stride_h < d)
+    return fail(RM_ERR_INVALID_ARG, "%s: head stride smaller than d (overlapping heads)", name);
+  return RM_OK;
+}
+
+#define RM_TRY(x)                   \
+  do {                              \
+    rm_status _s = (x);             \
+    if (_s != RM_OK) return _s;     \
+  } while (0)
+
+#define RM_CUDA(x, where)                               \
+  do {                                                  \
+    cudaError_t _e = (x);                               \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace layout (byte offsets from ws).
+struct FwdWs {
+  size_t o_parts, lse_parts, total;
+};
+FwdWs fwd_ws(const rm_attn_desc* d) {
+  FwdWs w{0, 0, 0};
+  if (d->mode != RM_RING_STEPWISE) return w;
+  const size_t rows = (size_t)d->B * d->N * d->Hq;
+  w.o_parts = 0;
+  w.lse_parts = align_up(rows * d->d * 4 * (size_t)d->P);
+  w.total = w.lse_parts + align_up(rows * 4 * (size_t)d->P);
+  return w;
+}
+struct BwdWs {
+  size_t delta, dq, total;
+};
+BwdWs bwd_ws(const rm_attn_desc* d) {
+  BwdWs w;
+  const size_t rows_q = (size_t)d->B * d->N * d->Hq;
+  w.delta = 0;
+  w.dq = align_up(rows_q * 4);
+  // fp32 (SIMT) problems write dQ directly; the tensor-core backward
+  // accumulates dQ in fp32 [B, Hq, N, d] and writes dK / dV itself
+  w.total = d->dtype == RM_F32 ? w.dq : w.dq + align_up(rows_q * d->d * 4);
+  return w;
+}
+
+rm_tensor dense_bnhd(void* p, int64_t N, int H, int d) {
+  rm_tensor t;
+  t.ptr = p;
+  t.stride_b = N * H * d;
+  t.stride_n = (int64_t)H * d;
+  t.stride_h = d;
+  return t;
+}
+rm_tensor dense_bhnd(void* p, int64_t N, int H, int d) {
+  rm_tensor t;
+  t.ptr = p;
+  t.stride_b = (int64_t)H * N * d;
+  t.stride_n = d;
+  t.stride_h = N * d;
+  return t;
+}
+
+rm_tensor offset_rows(rm_tensor t, int64_t rows, int esize) {
+  t.ptr = (char*)t.ptr + rows * t.stride_n * esize;
+  return t;
+}
+
+}  // namespace
+
+int num_sms() {
+  int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+unsigned int* status_word() {
+  int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = (unsigned int*)p;
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace rm
+
+using namespace rm;
+
+extern "C" {
+
+const char* rm_status_string(rm_status s) {
+  switch (s) {
+    case RM_OK: return "RM_OK";
+    case RM_ERR_INVALID_ARG: return "RM_ERR_INVALID_ARG";
+    case RM_ERR_UNSUPPORTED: return "RM_ERR_UNSUPPORTED";
+    case RM_ERR_WORKSPACE: return "RM_ERR_WORKSPACE";
+    case RM_ERR_CUDA: return "RM_ERR_CUDA";
+    case RM_ERR_TIMEOUT: return "RM_ERR_TIMEOUT";
+  }
+  return "RM_ERR_UNKNOWN";
+}
+
+const char* rm_last_error(void) { return t_last_error.c_str(); }
+
+rm_status rm_get_device_status(void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  RM_CUDA(cudaStreamSynchronize(st), "rm_get_device_status: stream sync");
+  unsigned int* p = status_word();
+  if (!p) return fail(RM_ERR_CUDA, "rm_get_device_status: no status word");
+  unsigned int v = 0;
+  RM_CUDA(cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, st), "status read");
+  RM_CUDA(cudaMemsetAsync(p, 0, sizeof(v), st), "status clear");
+  RM_CUDA(cudaStreamSynchronize(st), "status sync");
+  if (v & kStatusTimeout) return fail(RM_ERR_TIMEOUT, "a device-side bounded wait expired");
+  return RM_OK;
+}
+
+rm_status rm_debug_expire_wait(uint32_t spin_limit, void* stream) {
+  unsigned int* p = status_word();
+  if (!p) return fail(RM_ERR_CUDA, "no status word");
+  RM_CUDA(launch_debug_expire_wait(spin_limit, p, (cudaStream_t)stream), "debug wait launch");
+  return RM_OK;
+}
+
+rm_status rm_layout_permute(rm_dtype dtype, int B, int64_t N, int H, int d, rm_layout layout,
+                            int P, int inverse, const void* in, void* out, void* stream) {
+  if (dtype != RM_F32 && dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || N < 0 || H < 1 || d < 1 || P < 1) return fail(RM_ERR_INVALID_ARG, "bad sizes");
+  if (layout != RM_LAYOUT_CONTIGUOUS && layout != RM_LAYOUT_ZIGZAG && layout != RM_LAYOUT_STRIPED)
+    return fail(RM_ERR_INVALID_ARG, "bad layout");
+  if (N % P) return fail(RM_ERR_INVALID_ARG, "N %% P != 0");
+  if (layout == RM_LAYOUT_ZIGZAG && N % (2 * (int64_t)P))
+    return fail(RM_ERR_INVALID_ARG, "zigzag needs N %% 2P == 0");
+  if (inverse != 0 && inverse != 1) return fail(RM_ERR_INVALID_ARG, "inverse must be 0 or 1");
+  const int64_t bytes = (int64_t)B * N * H * d * esize_of(dtype);
+  if (bytes == 0) return RM_OK;
+  if (!in || !out) return fail(RM_ERR_INVALID_ARG, "NULL pointer");
+  if ((const char*)in < (const char*)out + bytes && (const char*)out < (const char*)in + bytes)
+    return fail(RM_ERR_INVALID_ARG, "in and out overlap");
+  RM_CUDA(launch_layout_permute(esize_of(dtype), B, N, H, d, layout, P, inverse, in, out,
+                                (cudaStream_t)stream),
+          "layout_permute launch");
+  return RM_OK;
+}
+
+rm_status rm_seq_head_repack(rm_dtype dtype, int P, int64_t N_local, int H, int d,
+                             int head_to_seq, const void* in, void* out, void* stream) {
+  if (dtype != RM_F32 && dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (P < 1 || N_local < 0 || H < 1 || d < 1) return fail(RM_ERR_INVALID_ARG, "bad sizes");
+  if (H % P) return fail(RM_ERR_INVALID_ARG, "H %% P != 0 (Ulysses degree exceeds heads)");
+  if (head_to_seq != 0 && head_to_seq != 1)
+    return fail(RM_ERR_INVALID_ARG, "head_to_seq must be 0 or 1");
+  const int64_t bytes = (int64_t)P * N_local * H * d * esize_of(dtype);
+  if (bytes == 0) return RM_OK;
+  if (!in || !out) return fail(RM_ERR_INVALID_ARG, "NULL pointer");
+  if ((const char*)in < (const char*)out + bytes && (const char*)out < (const char*)in + bytes)
+    return fail(RM_ERR_INVALID_ARG, "in and out overlap");
+  RM_CUDA(launch_seq_head_repack(esize_of(dtype), P, N_local, H, d, head_to_seq, in, out,
+                                 (cudaStream_t)stream),
+          "seq_head_repack launch");
+  return RM_OK;
+}
+
+rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d, int n_parts,
+                       const rm_tensor* o_parts, const float* const* lse_parts, rm_tensor o_out,
+                       float* lse_out, void* stream) {
+  if (out_dtype != RM_F32 && out_dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || H < 1 || Nq < 0 || d < 4 || d > 128 || d % 4)
+    return fail(RM_ERR_INVALID_ARG, "bad sizes (need d %% 4 == 0, 4 <= d <= 128)");
+  if (n_parts < 1 || n_parts > kMaxMergeParts)
+    return fail(RM_ERR_INVALID_ARG, "n_parts must be in [1, %d]", kMaxMergeParts);
+  if (!o_parts || !lse_parts) return fail(RM_ERR_INVALID_ARG, "NULL part arrays");
+  const int64_t rows = (int64_t)B * Nq;
+  if (rows == 0) return RM_OK;
+  MergeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.d = d;
+  a.Nq = Nq;
+  a.n_parts = n_parts;
+  a.lse_ld = Nq;
+  for (int i = 0; i < n_parts; ++i) {
+    RM_TRY(check_tensor("o_parts[i]", o_parts[i], 4, rows, H, d));
+    if (!lse_parts[i] || ((uintptr_t)lse_parts[i] & 3))
+      return fail(RM_ERR_INVALID_ARG, "lse_parts[%d] NULL or misaligned", i);
+    a.o_ptr[i] = (const float*)o_parts[i].ptr;
+    a.o_sb[i] = o_parts[i].stride_b;
+    a.o_sn[i] = o_parts[i].stride_n;
+    a.o_sh[i] = o_parts[i].stride_h;
+    a.lse_ptr[i] = lse_parts[i];
+  }
+  RM_TRY(check_tensor("o_out", o_out, out_dtype == RM_BF16 ? 2 : 4, rows, H, d));
+  if (out_dtype == RM_BF16 && o_out.ptr == o_parts[0].ptr)
+    return fail(RM_ERR_INVALID_ARG, "in-place merge needs an fp32 output");
+  if (!lse_out || ((uintptr_t)lse_out & 3)) return fail(RM_ERR_INVALID_ARG, "lse_out NULL/misaligned");
+  a.out = o_out.ptr;
+  a.out_sb = o_out.stride_b;
+  a.out_sn = o_out.stride_n;
+  a.out_sh = o_out.stride_h;
+  a.lse_out = lse_out;
+  RM_CUDA(launch_lse_merge(a, out_dtype == RM_BF16, (cudaStream_t)stream), "lse_merge launch");
+  return RM_OK;
+}
+
+rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d, rm_tensor o,
+                                 rm_tensor dout, float* delta, void* stream) {
+  if (dtype != RM_F32 && dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || N < 0 || H < 1 || d < 4 || d > 128 || d % 4)
+    return fail(RM_ERR_INVALID_ARG, "bad sizes (need d %% 4 == 0, 4 <= d <= 128)");
+  const int64_t rows = (int64_t)B * N;
+  if (rows == 0) return RM_OK;
+  RM_TRY(check_tensor("o", o, esize_of(dtype), rows, H, d));
+  RM_TRY(check_tensor("dout", dout, esize_of(dtype), rows, H, d));
+  if (!delta || ((uintptr_t)delta & 3)) return fail(RM_ERR_INVALID_ARG, "delta NULL/misaligned");
+  RM_CUDA(launch_bwd_preprocess(dtype == RM_BF16, B, N, H, d, o, dout, delta, nullptr,
+                                (cudaStream_t)stream),
+          "bwd_preprocess launch");
+  return RM_OK;
+}
+
+static rm_status check_qkv(const rm_attn_desc* desc, int64_t rows, rm_tensor q, rm_tensor k,
+                           rm_tensor v) {
+  const int es = esize_of(desc->dtype);
+  const int64_t r = (int64_t)desc->B * rows;
+  RM_TRY(check_tensor("q", q, es, r, desc->Hq, desc->d));
+  RM_TRY(check_tensor("k", k, es, r, desc->Hkv, desc->d));
+  RM_TRY(check_tensor("v", v, es, r, desc->Hkv, desc->d));
+  return RM_OK;
+}
+
+static AttnArgs attn_args(const rm_attn_desc* desc, int64_t lse_ld) {
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = desc->B;
+  a.Hq = desc->Hq;
+  a.Hkv = desc->Hkv;
+  a.d = desc->d;
+  a.N = desc->N;
+  a.P = desc->P;
+  a.layout = desc->layout;
+  a.causal = desc->causal ? 1 : 0;
+  a.scale = eff_scale(desc);
+  a.lse_ld = lse_ld;
+  a.status = status_word();
+  return a;
+}
+
+// One (q_rank, kv_rank) forward with shard-local operands; LSE rows lse_ld apart.
+static rm_status block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm_tensor q,
+                           rm_tensor k, rm_tensor v, rm_tensor o, int o_f32, float* lse,
+                           int64_t lse_ld, cudaStream_t st) {
+  AttnArgs a = attn_args(desc, lse_ld);
+  a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = o_f32; a.lse = lse;
+  if (desc->dtype == RM_F32) {
+    RM_CUDA(launch_simt_fwd(a, q_rank, kv_rank, st), "simt fwd launch");
+    return RM_OK;
+  }
+  return tc_fwd(a, q_rank, kv_rank, st);
+}
+
+rm_status rm_attn_block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm_tensor q,
+                            rm_tensor k, rm_tensor v, rm_tensor o, int o_f32, float* lse,
+                            void* stream) {
+  RM_TRY(check_desc(desc));
+  if (q_rank < 0 || q_rank >= desc->P || kv_rank < 0 || kv_rank >= desc->P)
+    return fail(RM_ERR_INVALID_ARG, "rank out of range");
+  const int64_t L = desc->N / desc->P;
+  if (desc->B == 0 || L == 0) return RM_OK;
+  RM_TRY(check_qkv(desc, L, q, k, v));
+  const int f32_out = (o_f32 || desc->dtype == RM_F32) ? 1 : 0;
+  RM_TRY(check_tensor("o", o, f32_out ? 4 : 2, (int64_t)desc->B * L, desc->Hq, desc->d));
+  if (!lse || ((uintptr_t)lse & 3)) return fail(RM_ERR_INVALID_ARG, "lse NULL/misaligned");
+  return block_fwd(desc, q_rank, kv_rank, q, k, v, o, f32_out, lse, L, (cudaStream_t)stream);
+}
+
+rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm_tensor q,
+                            rm_tensor k, rm_tensor v, rm_tensor dout, const float* lse_final,
+                            const float* delta, rm_tensor dq_acc, rm_tensor dk_acc,
+                            rm_tensor dv_acc, void* stream) {
+  RM_TRY(check_desc(desc));
+  if (q_rank < 0 || q_rank >= desc->P || kv_rank < 0 || kv_rank >= desc->P)
+    return fail(RM_ERR_INVALID_ARG, "rank out of range");
+  const int64_t L = desc->N / desc->P;
+  if (desc->B == 0 || L == 0) return RM_OK;
+  RM_TRY(check_qkv(desc, L, q, k, v));
+  const int64_t rows = (int64_t)desc->B * L;
+  RM_TRY(check_tensor("dout", dout, esize_of(desc->dtype), rows, desc->Hq, desc->d));
+  RM_TRY(check_tensor("dq_acc", dq_acc, 4, rows, desc->Hq, desc->d));
+  RM_TRY(check_tensor("dk_acc", dk_acc, 4, rows, desc->Hkv, desc->d));
+  RM_TRY(check_tensor("dv_acc", dv_acc, 4, rows, desc->Hkv, desc->d));
+  if (!lse_final || !delta) return fail(RM_ERR_INVALID_ARG, "lse_final / delta NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  AttnArgs a = attn_args(desc, L);
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse_in = lse_final; a.delta = delta;
+  a.dq = dq_acc; a.dk = dk_acc; a.dv = dv_acc;
+  a.accumulate = 1;
+  if (desc->dtype == RM_F32) {
+    RM_CUDA(launch_simt_bwd(a, q_rank, kv_rank, st), "simt bwd launch");
+    return RM_OK;
+  }
+  return tc_bwd(a, q_rank, kv_rank, st);
+}
+
+rm_status rm_ring_workspace_size(const rm_attn_desc* desc, int backward, size_t* bytes) {
+  RM_TRY(check_desc(desc));
+  if (!bytes) return fail(RM_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = backward ? bwd_ws(desc).total : fwd_ws(desc).total;
+  return RM_OK;
+}
+
+rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, rm_tensor v,
+                           rm_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  RM_TRY(check_desc(desc));
+  if (desc->B == 0 || desc->N == 0) return RM_OK;
+  RM_TRY(check_qkv(desc, desc->N, q, k, v));
+  const int es = esize_of(desc->dtype);
+  RM_TRY(check_tensor("o", o, es, (int64_t)desc->B * desc->N, desc->Hq, desc->d));
+  if (!lse || ((uintptr_t)lse & 3)) return fail(RM_ERR_INVALID_ARG, "lse NULL/misaligned");
+  const FwdWs w = fwd_ws(desc);
+  if (w.total && (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255)))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  if (desc->mode == RM_RING_STEPWISE && desc->P > kMaxMergeParts)
+    return fail(RM_ERR_UNSUPPORTED, "stepwise mode supports P <= %d", kMaxMergeParts);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t L = desc->N / desc->P;
+  if (desc->mode == RM_RING_FUSED) {
+    AttnArgs a = attn_args(desc, desc->N);
+    a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = desc->dtype == RM_F32; a.lse = lse;
+    if (desc->dtype == RM_F32) {
+      RM_CUDA(launch_simt_fwd(a, -1, -1, st), "simt ring fwd launch");
+      return RM_OK;
+    }
+    return tc_fwd(a, -1, -1, st);
+  }
+  // Stepwise: at ring step k rank r attends to shard (r - k) mod P; the fp32
+  // partial O of step k fills slot k ([B, N, Hq, d], rank-major) and its LSE
+  // slot k ([B, Hq, N]); then every rank merges its P partials.
+  const size_t rows_q = (size_t)desc->B * desc->N * desc->Hq;
+  float* o_slots = (float*)((char*)ws + w.o_parts);
+  float* lse_slots = (float*)((char*)ws + w.lse_parts);
+  for (int step = 0; step < desc->P; ++step) {
+    rm_tensor o_k = dense_bnhd(o_slots + (size_t)step * rows_q * desc->d, desc->N, desc->Hq,
+                               desc->d);
+    float* lse_k = lse_slots + (size_t)step * rows_q;
+    for (int r = 0; r < desc->P; ++r) {
+      const int s = ((r - step) % desc->P + desc->P) % desc->P;
+      RM_TRY(block_fwd(desc, r, s, offset_rows(q, (int64_t)r * L, es),
+                       offset_rows(k, (int64_t)s * L, es), offset_rows(v, (int64_t)s * L, es),
+                       offset_rows(o_k, (int64_t)r * L, 4), 1, lse_k + (int64_t)r * L, desc->N,
+                       st));
+    }
+  }
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  m.B = desc->B;
+  m.H = desc->Hq;
+  m.d = desc->d;
+  m.Nq = desc->N;  // all ranks at once: rank-major rows, every row has P partials
+  m.n_parts = desc->P;
+  m.lse_ld = desc->N;
+  for (int step = 0; step < desc->P; ++step) {
+    m.o_ptr[step] = o_slots + (size_t)step * rows_q * desc->d;
+    m.o_sb[step] = desc->N * desc->Hq * desc->d;
+    m.o_sn[step] = (int64_t)desc->Hq * desc->d;
+    m.o_sh[step] = desc->d;
+    m.lse_ptr[step] = lse_slots + (size_t)step * rows_q;
+  }
+  m.out = o.ptr;
+  m.out_sb = o.stride_b;
+  m.out_sn = o.stride_n;
+  m.out_sh = o.stride_h;
+  m.lse_out = lse;
+  RM_CUDA(launch_lse_merge(m, desc->dtype == RM_BF16, st), "ring merge launch");
+  return RM_OK;
+}
+
+rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, rm_tensor v,
+                           rm_tensor o, const float* lse, rm_tensor dout, rm_tensor dq,
+                           rm_tensor dk, rm_tensor dv, void* ws, size_t ws_bytes, void* stream) {
+  RM_TRY(check_desc(desc));
+  if (desc->B == 0 || desc->N == 0) return RM_OK;
+  RM_TRY(check_qkv(desc, desc->N, q, k, v));
+  const int es = esize_of(desc->dtype);
+  const int64_t rows = (int64_t)desc->B * desc->N;
+  RM_TRY(check_tensor("o", o, es, rows, desc->Hq, desc->d));
+  RM_TRY(check_tensor("dout", dout, es, rows, desc->Hq, desc->d));
+  RM_TRY(check_tensor("dq", dq, es, rows, desc->Hq, desc->d));
+  RM_TRY(check_tensor("dk", dk, es, rows, desc->Hkv, desc->d));
+  RM_TRY(check_tensor("dv", dv, es, rows, desc->Hkv, desc->d));
+  if (!lse) return fail(RM_ERR_INVALID_ARG, "lse NULL");
+  const BwdWs w = bwd_ws(desc);
+  if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  float* delta = (float*)((char*)ws + w.delta);
+  float* dq_acc = (float*)((char*)ws + w.dq);
+  AttnArgs a = attn_args(desc, desc->N);
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse_in = lse; a.delta = delta;
+  a.accumulate = 0;
+  if (desc->dtype == RM_F32) {
+    // every SIMT thread owns complete sums: dq / dk / dv are written directly
+    RM_CUDA(launch_bwd_preprocess(0, desc->B, desc->N, desc->Hq, desc->d, o, dout, delta, nullptr,
+                                  st),
+            "bwd preprocess launch");
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    RM_CUDA(launch_simt_bwd(a, -1, -1, st), "simt ring bwd launch");
+    return RM_OK;
+  }
+  // delta from the final O, and the dQ accumulator ([B, Hq, N, d]) zeroed in the same pass
+  RM_CUDA(launch_bwd_preprocess(1, desc->B, desc->N, desc->Hq, desc->d, o, dout, delta, dq_acc,
+                                st),
+          "bwd preprocess launch");
+  rm_tensor dq_t = dense_bhnd(dq_acc, desc->N, desc->Hq, desc->d);
+  a.dq = dq_t; a.dk = dk; a.dv = dv;
+  RM_TRY(tc_bwd(a, -1, -1, st));
+  RM_CUDA(launch_convert_f32(1, desc->B, desc->N, desc->Hq, desc->d, dq_t, dq, st), "dq out");
+  return RM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,20 @@
+// Tensor-core (tcgen05 / TMEM / TMA) bf16 attention, sm_100a.
+#pragma once
+
+#include "internal.h"
+
+namespace rm {
+
+bool tc_supported_head_dim(int d);
+
+// Forward.  q_rank < 0: the fused ring over all P ranks (operands rank-major,
+// running softmax state carried across KV shards); else one (q_rank, kv_rank)
+// shard pair with shard-local operands.  o is bf16 unless a.o_f32.
+rm_status tc_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
+
+// Backward.  Same rank convention.  dq is an fp32 accumulator (+=, any
+// strides); dk / dv are fp32 accumulators (+=) when a.accumulate, else bf16
+// outputs written once (ring mode: every KV tile owns its complete sums).
+rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
+
+}  // namespace rm

@@ -1,0 +1,532 @@
+// Forward attention on the sm_100a tensor cores (bf16 in, fp32 accumulate).
+//
+// One CTA owns two 128-row query tiles, A and B, that read the same KV head:
+// two query heads of one GQA group on the same rows when the group size is
+// even, else two consecutive row tiles of one head.  It walks the KV tiles
+// the tiles may see -- in ring mode over every KV shard in ring order
+// (r, r-1, ...; Mosaic, "How Ring Attention Works") -- and keeps the running
+// softmax state (m, l, O) across tiles and shards, so the LSE merge of the
+// per-shard partials happens implicitly in the rescaling (Ring Attention &
+// Friends, "Tiling with the Softmax Rescaling Trick").
+//
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax for tile A (one thread per TMEM lane = query row)
+//   warps 4-7  softmax for tile B
+//   warp  8    TMA producer: Q once, then K / V tiles into a 2-stage ring
+//   warp  9    MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
+//              read from TMEM (written over S by the softmax warps)
+//   warps 10-11 idle
+// Register split: the block launches at 168 registers a thread (64512 in
+// all); the softmax warpgroups grow to 216 and the third shrinks to 64:
+// 2*128*216 + 128*64 = 63488 <= 64512.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A, O_B after them.
+// While softmax A works on S_A(j), the tensor core runs PV_B(j-1) / S_B(j),
+// and vice versa.
+//
+// Causal masking: positions are increasing in the local index for every
+// layout, so the keys of shard s visible to a query form a prefix of the
+// shard; tiles past the last row's prefix are never loaded, and only tiles
+// that cut a row's prefix apply an element mask.
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "tc_attn.h"
+#include "tc_common.cuh"
+
+namespace rm {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;  // keys per KV tile
+constexpr int kStages = 2;
+constexpr int kThreads = 384;
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 64;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr long long kDefaultWaitLimit = 4000000000LL;  // clock cycles (~2 s)
+
+template <int DP>
+struct FwdCfg {
+  static constexpr int kBoxCols = DP >= 64 ? 64 : DP;  // elements per TMA box row (<= 128 B)
+  static constexpr int kBoxes = DP / kBoxCols;         // boxes per 128-row tile
+  static constexpr int kRowBytes = kBoxCols * 2;
+  static constexpr uint32_t kSwz = kRowBytes == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr int kBoxBytes = kBM * kRowBytes;
+  static constexpr int kTileBytes = kBM * DP * 2;
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTileBytes;
+  static constexpr int kK = 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kSmem = kBar + 256 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr uint32_t kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + DP;
+  static_assert(kO1 + DP <= 512, "TMEM budget");
+};
+
+struct FwdParams {
+  int B, Hq, Hkv, d, P, layout, causal;
+  int64_t N, L;
+  float scale_log2;  // softmax scale * log2(e)
+  int ring, q_rank, kv_rank;
+  int head_pairs;
+  void* o;
+  int64_t o_sb, o_sn, o_sh;
+  int o_f32;
+  float* lse;
+  int64_t lse_ld;
+  unsigned int* status;
+  long long wait_limit;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// K-major operand tile (Q or K): descriptor for UMMA K-step k (16 elements).
+template <int DP>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int k) {
+  using C = FwdCfg<DP>;
+  const int col = k * 16;
+  const uint32_t addr = tile_addr + (col / C::kBoxCols) * C::kBoxBytes + (col % C::kBoxCols) * 2;
+  return smem_desc(addr, 16, 8 * C::kRowBytes, C::kSwz);
+}
+// V tile as the MN-major B operand of O += P V: K-step k covers kv rows
+// [16k, 16k+16); the d axis is split over boxes kBoxBytes apart.
+template <int DP>
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile_addr, int k) {
+  using C = FwdCfg<DP>;
+  return smem_desc(tile_addr + k * 16 * C::kRowBytes, C::kBoxBytes, 8 * C::kRowBytes, C::kSwz);
+}
+
+template <int DP>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<DP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* bar_q = bars + 0;
+  uint64_t* bar_k_full = bars + 1;    // [kStages]
+  uint64_t* bar_v_full = bars + 3;    // [kStages]
+  uint64_t* bar_kv_empty = bars + 5;  // [kStages]
+  uint64_t* bar_s_full = bars + 7;    // [2] per query tile
+  uint64_t* bar_p_full = bars + 9;    // [2] per query tile
+  uint64_t* bar_o_done = bars + 11;
+  uint64_t* bar_drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const LayoutMap lay = make_layout(p.layout, p.N, p.P);
+  const int64_t L = p.L;
+  const int r = p.ring ? (int)(blockIdx.z % p.P) : p.q_rank;
+  const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
+  const int unit = gridDim.x - 1 - blockIdx.x;  // later rows see more keys: start them first
+  int hA, hB;
+  int64_t rowA, rowB;
+  if (p.head_pairs) {
+    hA = 2 * blockIdx.y;
+    hB = hA + 1;
+    rowA = rowB = (int64_t)unit * kBM;
+  } else {
+    hA = hB = blockIdx.y;
+    rowA = (int64_t)unit * 2 * kBM;
+    rowB = rowA + kBM;
+  }
+  const int g = hA / (p.Hq / p.Hkv);
+  const int64_t last_row = min((p.head_pairs ? rowA : rowB) + kBM - 1, L - 1);
+  const int64_t t_last = lay.pos(r, last_row);
+  const int nsteps = p.ring ? p.P : 1;
+  const long long limit = p.wait_limit;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_v_full + s, 1);
+      mbar_init(bar_kv_empty + s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_s_full + x, 1);
+      mbar_init(bar_p_full + x, 128);
+    }
+    mbar_init(bar_o_done, 1);
+    mbar_init(bar_drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  // KV shard of ring step `step`, and how many of its keys the CTA may see.
+  auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
+  auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
+
+  if (warp >= 8) {
+    regs_dec<kRegsOther>();
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int qs = p.ring ? r : 0;
+      mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
+#pragma unroll
+      for (int x = 0; x < C::kBoxes; ++x) {
+        tma_load_5d(smem + C::kQ0 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hA, (int)rowA,
+                    qs, b);
+        tma_load_5d(smem + C::kQ1 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hB, (int)rowB,
+                    qs, b);
+      }
+      int j = 0;
+      bool ok = true;
+      for (int step = 0; step < nsteps && ok; ++step) {
+        const int s = shard_of(step);
+        const int nt = (int)((cta_keys(s) + kBN - 1) / kBN);
+        const int ks = p.ring ? s : 0;
+        for (int t = 0; t < nt; ++t, ++j) {
+          const int st = j & 1;
+          if (j >= kStages && !mbar_wait(bar_kv_empty + st, ((j >> 1) - 1) & 1, limit, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_k_full + st, C::kTileBytes);
+#pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_5d(smem + C::kK + st * C::kTileBytes + x * C::kBoxBytes, &tmK,
+                        bar_k_full + st, x * C::kBoxCols, g, t * kBN, ks, b);
+          mbar_arrive_expect_tx(bar_v_full + st, C::kTileBytes);
+#pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_5d(smem + C::kV + st * C::kTileBytes + x * C::kBoxBytes, &tmV,
+                        bar_v_full + st, x * C::kBoxCols, g, t * kBN, ks, b);
+        }
+      }
+      // drain: the last load issued into each stage has landed before exit
+      for (int st = 0; st < kStages && j > st; ++st) {
+        const int uses = (j - st + 1) / 2;  // loads issued into stage st
+        mbar_wait(bar_k_full + st, (uses - 1) & 1, limit, p.status);
+        mbar_wait(bar_v_full + st, (uses - 1) & 1, limit, p.status);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);
+      constexpr uint32_t idO = idesc_bf16(kBM, DP, 0, 1);
+      const uint32_t q0 = smem_u32(smem + C::kQ0), q1 = smem_u32(smem + C::kQ1);
+      const uint32_t kbase = smem_u32(smem + C::kK), vbase = smem_u32(smem + C::kV);
+      int n = 0;
+      for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + kBN - 1) / kBN);
+      auto issue_s = [&](uint32_t qaddr, uint32_t scol, int st) {
+        const uint32_t kaddr = kbase + st * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < DP / 16; ++k)
+          mma_ss(tmem + scol, kmajor_desc<DP>(qaddr, k), kmajor_desc<DP>(kaddr, k), idS, k > 0);
+      };
+      auto issue_pv = [&](uint32_t scol, uint32_t ocol, int st, bool first) {
+        const uint32_t vaddr = vbase + st * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          mma_ts(tmem + ocol, tmem + scol + k * 8, v_desc<DP>(vaddr, k), idO,
+                 (first && k == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(bar_q, 0, limit, p.status);
+      if (ok && n > 0) {
+        ok = mbar_wait(bar_k_full + 0, 0, limit, p.status);
+        if (ok) {
+          fence_after_sync();
+          issue_s(q0, C::kS0, 0);
+          mma_commit(bar_s_full + 0);
+          issue_s(q1, C::kS1, 0);
+          mma_commit(bar_s_full + 1);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j & 1;
+        const int nx = (j + 1) & 1;
+        if (!mbar_wait(bar_v_full + st, (j >> 1) & 1, limit, p.status)) break;
+        if (!mbar_wait(bar_p_full + 0, j & 1, limit, p.status)) break;
+        fence_after_sync();
+        issue_pv(C::kS0, C::kO0, st, j == 0);
+        if (j + 1 < n) {
+          if (!mbar_wait(bar_k_full + nx, ((j + 1) >> 1) & 1, limit, p.status)) break;
+          fence_after_sync();
+          issue_s(q0, C::kS0, nx);
+          mma_commit(bar_s_full + 0);
+        }
+        if (!mbar_wait(bar_p_full + 1, j & 1, limit, p.status)) break;
+        fence_after_sync();
+        issue_pv(C::kS1, C::kO1, st, j == 0);
+        mma_commit(bar_kv_empty + st);
+        if (j + 1 < n) {
+          issue_s(q1, C::kS1, nx);
+          mma_commit(bar_s_full + 1);
+        }
+      }
+      mma_commit(bar_o_done);
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, limit, p.status);
+    }
+  }
+  } else {
+    regs_inc<kRegsSoftmax>();
+    // ---------------- softmax warpgroups ----------------
+    const int X = warp >> 2;
+    const int lane_base = (warp & 3) * 32;
+    const int64_t row = (X ? rowB : rowA) + lane_base + lane;
+    const int h = X ? hB : hA;
+    const bool live = row < L;
+    const int64_t tq = live ? lay.pos(r, row) : -1;
+    const uint32_t tS = tmem + ((uint32_t)lane_base << 16) + (X ? C::kS1 : C::kS0);
+    const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + (X ? C::kO1 : C::kO0);
+    uint64_t* s_full = bar_s_full + X;
+    uint64_t* p_full = bar_p_full + X;
+    float m = -INFINITY;  // running max of the scaled scores, log2 units
+    float l = 0.f;        // running row sum (relative to m)
+    int j = 0;
+    bool ok = true;
+    for (int step = 0; step < nsteps && ok; ++step) {
+      const int s = shard_of(step);
+      const int nt = (int)((cta_keys(s) + kBN - 1) / kBN);
+      const int64_t row_keys = !live ? 0 : (p.causal ? lay.visible_count(s, tq) : L);
+      for (int t = 0; t < nt; ++t, ++j) {
+        // all lanes leave together, so the warp-collective tcgen05.ld / st
+        // below always run converged
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, limit, p.status))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        float sc[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tS + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sc[c * 32 + i] = __uint_as_float(v[i]);
+        }
+        tmem_wait_ld();
+        const int64_t nvalid = row_keys - (int64_t)t * kBN;
+        if (nvalid < kBN) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c >= nvalid) sc[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, sc[c]);
+        const float m_tile = mx * p.scale_log2;
+        // Lazy rescale: the reference max only moves when it grows by more
+        // than 8 (a factor 256), so O is rescaled rarely; p <= 256 otherwise.
+        const bool grow = m_tile > m + 8.0f;
+        const float m_new = grow ? m_tile : m;
+        const bool need = grow && j > 0 && m != -INFINITY;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2(m - m_new) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < DP / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            tmem_st32(tO + c * 32, v);
+          }
+        }
+        if (grow) {
+          l *= (m == -INFINITY) ? 0.f : ex2(m - m_new);
+          m = m_new;
+        }
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(sc[c * 32 + 2 * i], p.scale_log2, -m_use));
+            const float p1 = ex2(fmaf(sc[c * 32 + 2 * i + 1], p.scale_log2, -m_use));
+            l += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(p_full);
+      }
+    }
+    // ---------------- epilogue: O / l, LSE ----------------
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bar_o_done, 0, limit, p.status))) {
+      fence_after_sync();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      const float lse = l > 0.f ? (((m == -INFINITY) ? 0.f : m) + __log2f(l)) * kLn2 : -INFINITY;
+      const int64_t orow = (p.ring ? (int64_t)r * L : 0) + row;
+      char* obase = reinterpret_cast<char*>(p.o) +
+                    (b * p.o_sb + orow * p.o_sn + (int64_t)h * p.o_sh) * (p.o_f32 ? 4 : 2);
+#pragma unroll
+      for (int c = 0; c < DP / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + c * 32, v);
+        tmem_wait_ld();
+        if (live) {
+          if (p.o_f32) {
+            float4* dst = reinterpret_cast<float4*>(obase) + c * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (c * 32 + 4 * i < p.d)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                                     __uint_as_float(v[4 * i + 2]) * inv,
+                                     __uint_as_float(v[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(obase) + c * 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (c * 32 + 8 * i >= p.d) continue;  // d = 24 stores 3 of the 4 vectors
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv);
+              u.y = pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv);
+              u.z = pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv);
+              u.w = pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv);
+              dst[i] = u;
+            }
+          }
+        }
+      }
+      if (live) p.lse[((int64_t)b * p.Hq + h) * p.lse_ld + orow] = lse;
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// A [B, P', L, H, d] view (P' = P in ring mode, 1 for a single shard) of a
+// bf16 operand, read in boxes of (box_cols, 1 head, 128 rows); columns past d
+// (head-dim padding) and rows past L are zero-filled by the TMA unit.
+rm_status encode_operand_map(CUtensorMap* map, const rm_tensor& t, int B, int shards, int64_t L,
+                             int H, int d, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return RM_ERR_CUDA;
+  const int64_t sn = t.stride_n * 2;
+  const int64_t sh = (H > 1 ? t.stride_h : d) * 2;
+  const int64_t sp = L * t.stride_n * 2;
+  const int64_t sb = (B > 1 ? t.stride_b : (int64_t)shards * L * t.stride_n) * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)shards,
+                        (cuuint64_t)B};
+  cuuint64_t strides[4] = {(cuuint64_t)sh, (cuuint64_t)sn, (cuuint64_t)(sp > 0 ? sp : 16),
+                           (cuuint64_t)(sb > 0 ? sb : 16)};
+  cuuint32_t box[5] = {(cuuint32_t)box_cols, 1, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle swz =
+      box_cols * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult rc = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, t.ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? RM_OK : RM_ERR_CUDA;
+}
+
+bool tc_supported_head_dim(int d) { return d == 24 || d == 32 || d == 64 || d == 128; }
+
+int tc_padded_head_dim(int d) { return d <= 32 ? 32 : d; }
+
+long long tc_wait_limit() {
+  static long long lim = [] {
+    const char* e = getenv("RM_WAIT_LIMIT_CYCLES");
+    long long v = e ? atoll(e) : 0;
+    return v > 0 ? v : kDefaultWaitLimit;
+  }();
+  return lim;
+}
+
+template <int DP>
+static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream) {
+  using C = FwdCfg<DP>;
+  const bool ring = q_rank < 0;
+  const int64_t L = a.N / a.P;
+  const int shards = ring ? a.P : 1;
+  CUtensorMap mq, mk, mv;
+  if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, C::kBoxCols, kBM) != RM_OK ||
+      encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN) != RM_OK ||
+      encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN) != RM_OK)
+    return RM_ERR_CUDA;
+  FwdParams p;
+  p.B = a.B;
+  p.d = a.d;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.P = a.P;
+  p.layout = a.layout;
+  p.causal = a.causal;
+  p.N = a.N;
+  p.L = L;
+  p.scale_log2 = a.scale * kLog2e;
+  p.ring = ring ? 1 : 0;
+  p.q_rank = q_rank;
+  p.kv_rank = kv_rank;
+  p.head_pairs = ((a.Hq / a.Hkv) % 2 == 0) ? 1 : 0;
+  p.o = a.o.ptr;
+  p.o_sb = a.o.stride_b;
+  p.o_sn = a.o.stride_n;
+  p.o_sh = a.o.stride_h;
+  p.o_f32 = a.o_f32;
+  p.lse = a.lse;
+  p.lse_ld = a.lse_ld;
+  p.status = a.status;
+  p.wait_limit = tc_wait_limit();
+  const int units = p.head_pairs ? ceil_div(L, kBM) : ceil_div(L, 2 * kBM);
+  dim3 grid((unsigned)units, (unsigned)(p.head_pairs ? a.Hq / 2 : a.Hq),
+            (unsigned)(ring ? a.B * a.P : a.B));
+  if (cudaFuncSetAttribute(tc_fwd_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmem) != cudaSuccess)
+    return RM_ERR_CUDA;
+  tc_fwd_kernel<DP><<<grid, kThreads, C::kSmem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? RM_OK : RM_ERR_CUDA;
+}
+
+rm_status tc_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream) {
+  if (a.B == 0 || a.N == 0) return RM_OK;
+  switch (tc_padded_head_dim(a.d)) {
+    case 32: return launch_fwd<32>(a, q_rank, kv_rank, stream);
+    case 64: return launch_fwd<64>(a, q_rank, kv_rank, stream);
+    case 128: return launch_fwd<128>(a, q_rank, kv_rank, stream);
+  }
+  return RM_ERR_UNSUPPORTED;
+}
+
+}  // namespace rm

@@ -1,0 +1,261 @@
+"""Thin Python binding of librm_attn.so (argument marshalling only).
+
+Every function here turns torch tensors into the plain pointers, sizes and
+strides of the C ABI in ``include/rm_attn.h`` and calls the entry point of the
+same name on the current CUDA stream; all computation happens in the CUDA
+kernels behind that ABI.  Importing this module loads the library and raises
+if it is missing -- there is no CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librm_attn.so")
+
+# ---- enums (mirror include/rm_attn.h) ----------------------------------------
+RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_WORKSPACE, RM_ERR_CUDA, RM_ERR_TIMEOUT = range(6)
+RM_F32, RM_BF16 = 0, 1
+LAYOUTS = {"contiguous": 0, "zigzag": 1, "striped": 2}
+MODES = {"fused": 0, "stepwise": 1}
+
+EXPORTED = (
+    "rm_attn_block_fwd", "rm_attn_block_bwd", "rm_attn_bwd_preprocess", "rm_lse_merge",
+    "rm_ring_workspace_size", "rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_layout_permute",
+    "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
+    "rm_debug_expire_wait",
+)
+
+
+class RmTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_n", ctypes.c_int64), ("stride_h", ctypes.c_int64)]
+
+
+class RmAttnDesc(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("N", ctypes.c_int64),
+                ("P", ctypes.c_int), ("layout", ctypes.c_int), ("causal", ctypes.c_int),
+                ("scale", ctypes.c_float), ("mode", ctypes.c_int)]
+
+
+class RmError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_status_name(status)}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m sequence_attention_rm_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    T, D = RmTensor, ctypes.POINTER(RmAttnDesc)
+    fp = ctypes.POINTER(ctypes.c_float)
+    sig = {
+        "rm_attn_block_fwd": [D, i, i, T, T, T, T, i, vp, vp],
+        "rm_attn_block_bwd": [D, i, i, T, T, T, T, vp, vp, T, T, T, vp],
+        "rm_attn_bwd_preprocess": [i, i, i64, i, i, T, T, vp, vp],
+        "rm_lse_merge": [i, i, i, i64, i, i, ctypes.POINTER(RmTensor), ctypes.POINTER(vp), T, vp, vp],
+        "rm_ring_workspace_size": [D, i, ctypes.POINTER(sz)],
+        "rm_ring_attn_fwd": [D, T, T, T, T, vp, vp, sz, vp],
+        "rm_ring_attn_bwd": [D, T, T, T, T, vp, T, T, T, T, vp, sz, vp],
+        "rm_layout_permute": [i, i, i64, i, i, i, i, i, vp, vp, vp],
+        "rm_seq_head_repack": [i, i, i64, i, i, i, vp, vp, vp],
+        "rm_get_device_status": [vp],
+        "rm_debug_expire_wait": [ctypes.c_uint32, vp],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.rm_status_string.argtypes = [ctypes.c_int]
+    lib.rm_status_string.restype = ctypes.c_char_p
+    lib.rm_last_error.argtypes = []
+    lib.rm_last_error.restype = ctypes.c_char_p
+    del fp
+    return lib
+
+
+_lib = load_library()
+
+
+def _status_name(s: int) -> str:
+    return _lib.rm_status_string(s).decode()
+
+
+def _check(status: int) -> None:
+    if status != RM_OK:
+        raise RmError(status, _lib.rm_last_error().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return RM_BF16
+    if t == torch.float32:
+        return RM_F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _bnhd(t: torch.Tensor) -> RmTensor:
+    """A [B, N, H, d] tensor with unit stride along d."""
+    if t.dim() != 4 or (t.shape[-1] > 1 and t.stride(-1) != 1):
+        raise ValueError("expected a [B, N, H, d] tensor with contiguous d")
+    return RmTensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def desc(dtype: torch.dtype, B: int, Hq: int, Hkv: int, d: int, N: int, P: int, layout: str,
+         causal: bool, scale: float | None = None, mode: str = "fused") -> RmAttnDesc:
+    return RmAttnDesc(_dtype_code(dtype), B, Hq, Hkv, d, N, P, LAYOUTS[layout], int(bool(causal)),
+                      0.0 if scale is None else float(scale), MODES[mode])
+
+
+# ---- entry points -----------------------------------------------------------
+def layout_permute(x: torch.Tensor, layout: str, P: int, inverse: bool = False,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Dense [B, N, H, d]: global order -> rank-major (inverse: back)."""
+    if not x.is_contiguous():
+        raise ValueError("layout_permute needs a dense tensor")
+    out = torch.empty_like(x) if out is None else out
+    B, N, H, d = x.shape
+    _check(_lib.rm_layout_permute(_dtype_code(x.dtype), B, N, H, d, LAYOUTS[layout], P,
+                                  int(inverse), _ptr(x), _ptr(out), _stream(stream)))
+    return out
+
+
+def seq_head_repack(x: torch.Tensor, P: int, head_to_seq: bool = False,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """seq->head: [P, L, H, d] -> [P, P*L, H/P, d]; head->seq is the inverse."""
+    if not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("seq_head_repack needs a dense 4-d tensor")
+    if not head_to_seq:
+        _, L, H, d = x.shape
+        shape = (P, P * L, H // P, d)
+    else:
+        _, NL, HP, d = x.shape
+        L, H = NL // P, HP * P
+        shape = (P, L, H, d)
+    out = torch.empty(shape, dtype=x.dtype, device=x.device) if out is None else out
+    _check(_lib.rm_seq_head_repack(_dtype_code(x.dtype), P, L, H, d, int(head_to_seq), _ptr(x),
+                                   _ptr(out), _stream(stream)))
+    return out
+
+
+def lse_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor],
+              out_dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None,
+              lse_out: torch.Tensor | None = None, stream=None):
+    """Merge fp32 partials [B, Nq, H, d] with LSE [B, H, Nq] -> (O, LSE)."""
+    n = len(o_parts)
+    B, Nq, H, d = o_parts[0].shape
+    parts = (RmTensor * n)(*[_bnhd(o) for o in o_parts])
+    lses = (ctypes.c_void_p * n)(*[l.data_ptr() for l in lse_parts])
+    out = torch.empty((B, Nq, H, d), dtype=out_dtype, device=o_parts[0].device) if out is None else out
+    lse_out = torch.empty((B, H, Nq), dtype=torch.float32, device=o_parts[0].device) \
+        if lse_out is None else lse_out
+    _check(_lib.rm_lse_merge(_dtype_code(out_dtype), B, H, Nq, d, n, parts, lses, _bnhd(out),
+                             _ptr(lse_out), _stream(stream)))
+    return out, lse_out
+
+
+def attn_block_fwd(q, k, v, *, N: int, P: int, layout: str, causal: bool, q_rank: int,
+                   kv_rank: int, scale: float | None = None, o_f32: bool = False, out=None,
+                   lse=None, stream=None):
+    """One Q shard [B, L, Hq, d] against one KV shard [B, L, Hkv, d] -> (O, LSE)."""
+    B, L, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    odt = torch.float32 if (o_f32 or q.dtype == torch.float32) else q.dtype
+    out = torch.empty((B, L, Hq, d), dtype=odt, device=q.device) if out is None else out
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(_lib.rm_attn_block_fwd(ctypes.byref(dsc), q_rank, kv_rank, _bnhd(q), _bnhd(k), _bnhd(v),
+                                  _bnhd(out), int(o_f32), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def attn_block_bwd(q, k, v, dout, lse_final, delta, dq_acc, dk_acc, dv_acc, *, N: int, P: int,
+                   layout: str, causal: bool, q_rank: int, kv_rank: int,
+                   scale: float | None = None, stream=None):
+    """Accumulate one shard pair's gradients into fp32 dq_acc / dk_acc / dv_acc."""
+    B, L, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    _check(_lib.rm_attn_block_bwd(ctypes.byref(dsc), q_rank, kv_rank, _bnhd(q), _bnhd(k), _bnhd(v),
+                                  _bnhd(dout), _ptr(lse_final), _ptr(delta), _bnhd(dq_acc),
+                                  _bnhd(dk_acc), _bnhd(dv_acc), _stream(stream)))
+
+
+def attn_bwd_preprocess(o, dout, delta=None, stream=None):
+    """delta [B, H, N] = rowsum(dout * o) in fp32."""
+    B, N, H, d = o.shape
+    delta = torch.empty((B, H, N), dtype=torch.float32, device=o.device) if delta is None else delta
+    _check(_lib.rm_attn_bwd_preprocess(_dtype_code(o.dtype), B, N, H, d, _bnhd(o), _bnhd(dout),
+                                       _ptr(delta), _stream(stream)))
+    return delta
+
+
+def ring_workspace_size(dsc: RmAttnDesc, backward: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.rm_ring_workspace_size(ctypes.byref(dsc), int(backward), ctypes.byref(n)))
+    return n.value
+
+
+def _workspace(nbytes: int, device, ws: torch.Tensor | None):
+    if nbytes == 0:
+        return ctypes.c_void_p(0), 0
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | None = None,
+                  mode: str = "fused", out=None, lse=None, ws=None, stream=None):
+    """Ring forward over P virtual ranks; q/k/v rank-major [B, N, H, d] -> (O, LSE [B, Hq, N])."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode)
+    out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    wp, wn = _workspace(ring_workspace_size(dsc, False), q.device, ws)
+    _check(_lib.rm_ring_attn_fwd(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(out),
+                                 _ptr(lse), wp, wn, _stream(stream)))
+    return out, lse
+
+
+def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
+                  scale: float | None = None, dq=None, dk=None, dv=None, ws=None, stream=None):
+    """Ring backward; returns (dq, dk, dv) in the input dtype, rank-major."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    wp, wn = _workspace(ring_workspace_size(dsc, True), q.device, ws)
+    _check(_lib.rm_ring_attn_bwd(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
+                                 _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
+                                 _stream(stream)))
+    return dq, dk, dv
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status word as an rm_status."""
+    return _lib.rm_get_device_status(_stream(stream))
+
+
+def debug_expire_wait(spin_limit: int, stream=None) -> None:
+    _check(_lib.rm_debug_expire_wait(spin_limit, _stream(stream)))
+
+
+def raw():
+    """The loaded ctypes library (for tests that call the C ABI directly)."""
+    return _lib

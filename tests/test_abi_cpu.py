@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rm_attn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:rm_status|const char\*)\s+(rm_\w+)\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def rm():
+    from sequence_attention_rm_b200 import rm as mod
+    return mod
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("rm_attn_block_fwd", "rm_attn_block_bwd", "rm_lse_merge", "rm_ring_attn_fwd",
+                 "rm_ring_attn_bwd", "rm_seq_head_repack", "rm_layout_permute",
+                 "rm_ring_workspace_size", "rm_get_device_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(rm):
+    lib = rm.raw()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) <= set(rm.EXPORTED) | {"rm_status_string", "rm_last_error"}
+
+
+def test_status_strings(rm):
+    lib = rm.raw()
+    assert lib.rm_status_string(0) == b"RM_OK"
+    assert lib.rm_status_string(5) == b"RM_ERR_TIMEOUT"
+
+
+def _desc(rm, **kw):
+    base = dict(dtype=rm.RM_BF16, B=1, Hq=16, Hkv=8, d=128, N=16384, P=2, layout=1, causal=1,
+                scale=0.0, mode=0)
+    base.update(kw)
+    return rm.RmAttnDesc(**base)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(d=96), 2),            # unsupported bf16 head dim
+    (dict(Hq=12, Hkv=8), 1),    # Hq % Hkv != 0
+    (dict(N=1000, P=3), 1),     # N % P != 0
+    (dict(N=4100, P=4), 1),     # zigzag needs N % 2P == 0
+    (dict(layout=7), 1),        # bad layout
+    (dict(P=0), 1),
+    (dict(dtype=9), 1),
+    (dict(dtype=0, d=130), 2),  # fp32 d > 128
+    (dict(mode=3), 1),
+])
+def test_desc_validation(rm, bad, status):
+    n = ctypes.c_size_t(0)
+    d = _desc(rm, **bad)
+    assert rm.raw().rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == status
+    assert rm.raw().rm_last_error()
+
+
+def test_workspace_sizes(rm):
+    n = ctypes.c_size_t(0)
+    lib = rm.raw()
+    d = _desc(rm)
+    assert lib.rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0
+    assert n.value == 0  # fused forward needs no workspace
+    assert lib.rm_ring_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == 0
+    # delta [B, Hq, N] + fp32 dQ accumulator [B, Hq, N, d]
+    assert n.value == 16 * 16384 * 4 + 16 * 16384 * 128 * 4
+    d = _desc(rm, mode=1)
+    assert lib.rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0
+    assert n.value == 2 * 16 * 16384 * 128 * 4 + 2 * 16 * 16384 * 4
+
+
+def test_entry_points_reject_bad_arguments_before_launch(rm):
+    lib = rm.raw()
+    nul = ctypes.c_void_p(0)
+    # layout permute: bad layout, N % P, overlapping buffers, NULL pointers
+    assert lib.rm_layout_permute(1, 1, 64, 2, 8, 9, 2, 0, nul, nul, nul) == 1
+    assert lib.rm_layout_permute(1, 1, 63, 2, 8, 0, 2, 0, nul, nul, nul) == 1
+    assert lib.rm_layout_permute(1, 1, 64, 2, 8, 0, 2, 0, nul, nul, nul) == 1
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert lib.rm_layout_permute(1, 1, 64, 2, 8, 0, 2, 0, p, p, nul) == 1  # overlap
+    assert lib.rm_layout_permute(1, 0, 64, 2, 8, 0, 2, 0, nul, nul, nul) == 0  # empty: no-op
+    # repack: head count must be a multiple of P (the Ulysses cap)
+    assert lib.rm_seq_head_repack(1, 4, 8, 6, 8, 0, nul, nul, nul) == 1
+    assert lib.rm_seq_head_repack(1, 4, 0, 8, 8, 0, nul, nul, nul) == 0
+    # merge: too many parts, bad head dim
+    T = rm.RmTensor
+    parts = (T * 1)(T(0, 0, 0, 0))
+    lses = (ctypes.c_void_p * 1)(0)
+    assert lib.rm_lse_merge(1, 1, 2, 8, 64, 17, parts, lses, T(0, 0, 0, 0), nul, nul) == 1
+    assert lib.rm_lse_merge(1, 1, 2, 8, 66, 1, parts, lses, T(0, 0, 0, 0), nul, nul) == 1
+    # ring forward: misaligned pointer / strides
+    d = _desc(rm, N=256, P=2)
+    bad_ptr = T(p.value + 8, 256 * 16 * 128, 16 * 128, 128)
+    ok = T(p.value, 256 * 16 * 128, 16 * 128, 128)
+    assert lib.rm_ring_attn_fwd(ctypes.byref(d), bad_ptr, ok, ok, ok, p, nul, 0, nul) == 1
+    bad_stride = T(p.value, 256 * 16 * 128, 16 * 128 + 3, 128)
+    assert lib.rm_ring_attn_fwd(ctypes.byref(d), ok, bad_stride, ok, ok, p, nul, 0, nul) == 1
+    # ring backward without a workspace
+    kv = T(p.value, 256 * 8 * 128, 8 * 128, 128)
+    assert lib.rm_ring_attn_bwd(ctypes.byref(d), ok, kv, kv, ok, p, ok, ok, kv, kv, nul, 0,
+                                nul) == 3
+    # block forward: rank out of range
+    assert lib.rm_attn_block_fwd(ctypes.byref(d), 2, 0, ok, kv, kv, ok, 0, p, nul) == 1
