@@ -1,0 +1,511 @@
+"""Benchmark of the ring-attention hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one "step"): the Llama-like causal ring -- B=1, 16 query heads / 8
+KV heads, d=128, N=16384 bf16 tokens, P=2 virtual ranks in the zigzag
+(load-balanced) layout, forward + backward:
+  layout permute of Q, K, V, dO to rank-major order -> fused ring forward ->
+  ring backward (delta preprocess, tcgen05 backward, dQ finalize) -> inverse
+  permute of O, LSE, dQ, dK, dV.
+Inputs are seeded synthetic tensors already resident in HBM; L2 (126 MB) is
+flushed between timed steps.  ``value`` is algorithmic TFLOP/s summed over all
+ranks: forward 4*d and backward 10*d flops per visible (query, key) pair,
+causal pairs only.  With --gpus N every rank runs an independent replica of
+the workload (the path has no data exchange on one GPU), so scaling is weak.
+
+Extra measurements on the same line: the LSE merge (8 partials per rank of the
+striped 128k shapes) and the Ulysses repack (Q and fused K|V of the 256k zigzag
+shapes) in GB/s against HBM, and the causal striped 128k forward against the
+bf16 tensor peak.
+
+``--impl reference`` times the CPU fp64 oracle instead, on a bounded sample of
+the same workload (2048 queries of one query head, forward and backward against
+every key they see), and prints the same metric with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sequence_attention_rm_b200 import synthetic  # noqa: E402
+
+METRIC = "ring-attn fwd+bwd TFLOP/s and % of BF16 peak at 1 B200; merge GB/s % HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def causal_pairs(w) -> int:
+    per_head = w.N * (w.N + 1) // 2 if w.causal else w.N * w.N
+    return per_head * w.Hq * w.B
+
+
+def flops_fwd(w) -> float:
+    return 4.0 * w.d * causal_pairs(w)
+
+
+def flops_bwd(w) -> float:
+    return 10.0 * w.d * causal_pairs(w)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (independent replicas; barrier + max-over-ranks timing)
+# ---------------------------------------------------------------------------
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz, mx, pw = float(parts[1]), float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            smax = mx
+            if pw > 300.0:  # under load
+                sm.append(mhz)
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:  # short runs: fall back to every sample
+            for line in getattr(self, "lines", []):
+                parts = [p.strip() for p in line.split(",")]
+                try:
+                    sm.append(float(parts[1]))
+                except (ValueError, IndexError):
+                    pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(getattr(self, "lines", []))}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Step:
+    """Pre-allocated buffers and the hot-path step of one workload."""
+
+    def __init__(self, rm, w, q, k, v, do):
+        self.rm, self.w = rm, w
+        self.q, self.k, self.v, self.do = q, k, v, do
+        e = lambda t: torch.empty_like(t)
+        self.qr, self.kr, self.vr, self.dor = e(q), e(k), e(v), e(do)
+        self.o, self.dq, self.dk, self.dv = e(q), e(q), e(k), e(v)
+        self.o_g, self.dq_g, self.dk_g, self.dv_g = e(q), e(q), e(k), e(v)
+        self.lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
+        self.lse_g = torch.empty_like(self.lse)
+        dsc = rm.desc(w.dtype, w.B, w.Hq, w.Hkv, w.d, w.N, w.P, w.layout, w.causal)
+        self.ws = torch.empty(max(rm.ring_workspace_size(dsc, True), 256), dtype=torch.uint8,
+                              device=q.device)
+        self.launches_per_step = 4 + 1 + 3 + 5
+
+    def run(self, ev=None):
+        rm, w = self.rm, self.w
+        lay, P = w.layout, w.P
+        if ev:
+            ev[0].record()
+        for src, dst in ((self.q, self.qr), (self.k, self.kr), (self.v, self.vr), (self.do, self.dor)):
+            rm.layout_permute(src, lay, P, out=dst)
+        if ev:
+            ev[1].record()
+        rm.ring_attn_fwd(self.qr, self.kr, self.vr, P=P, layout=lay, causal=w.causal,
+                         out=self.o, lse=self.lse)
+        if ev:
+            ev[2].record()
+        rm.ring_attn_bwd(self.qr, self.kr, self.vr, self.o, self.lse, self.dor, P=P, layout=lay,
+                         causal=w.causal, dq=self.dq, dk=self.dk, dv=self.dv, ws=self.ws)
+        if ev:
+            ev[3].record()
+        for src, dst in ((self.o, self.o_g), (self.dq, self.dq_g), (self.dk, self.dk_g),
+                         (self.dv, self.dv_g)):
+            rm.layout_permute(src, lay, P, inverse=True, out=dst)
+        # LSE [B, H, N]: the token axis is the last one; view it as [B*H, N, 1, 1]
+        rm.layout_permute(self.lse.view(w.B * w.Hq, w.N, 1, 1), lay, P, inverse=True,
+                          out=self.lse_g.view(w.B * w.Hq, w.N, 1, 1))
+        if ev:
+            ev[4].record()
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def time_events(pairs):
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def bench_ours(args, world, rank, local):
+    from sequence_attention_rm_b200 import rm
+
+    peaks, peak_src = load_peaks()
+    w = synthetic.LLAMA_ZIGZAG
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h, do_h = synthetic.attention_inputs(w)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    step = Step(rm, w, q, k, v, do)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush_l2(flush)
+            step.run(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    per = [time_events([(e[0], e[4]), (e[1], e[2]), (e[2], e[3]), (e[0], e[1]), (e[3], e[4])])
+           for e in evs]
+    step_ms = sum(p[0] for p in per)
+    fwd_ms = statistics.mean(p[1] for p in per)
+    bwd_ms = statistics.mean(p[2] for p in per)
+    perm_ms = statistics.mean(p[3] + p[4] for p in per)
+    step_ms_max = max_over_ranks(step_ms, world)
+    total_flops = (flops_fwd(w) + flops_bwd(w)) * args.steps * world
+    value = total_flops / (step_ms_max * 1e-3) / 1e12
+
+    # end-to-end: pinned host inputs in, results back to pinned host buffers
+    pin = lambda t: t.pin_memory()
+    hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
+    outs = [pin(torch.empty(t.shape, dtype=t.dtype)) for t in (step.o_g, step.dq_g, step.dk_g, step.dv_g, step.lse_g)]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for src, dst in ((hq, step.q), (hk, step.k), (hv, step.v), (hdo, step.do)):
+            dst.copy_(src, non_blocking=True)
+        step.run()
+        for src, dst in zip((step.o_g, step.dq_g, step.dk_g, step.dv_g, step.lse_g), outs):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "llama-causal-zigzag-16k: B=1 Hq=16 Hkv=8 d=128 N=16384 bf16 "
+                               "P=2 zigzag causal fwd+bwd",
+                   "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MiB write); inputs 192 MiB > L2"},
+    }
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    bwd_tflops = flops_bwd(w) / (bwd_ms * 1e-3) / 1e12
+    fwd_tflops = flops_fwd(w) / (fwd_ms * 1e-3) / 1e12
+    line["roofline"] = {
+        "bound": "tensor", "kernel": "tc_bwd_kernel (rm_ring_attn_bwd: + delta preprocess, dQ finalize)",
+        "achieved": round(bwd_tflops, 2), "peak": sustained, "unit": "TFLOP/s",
+        "frac": round(bwd_tflops / sustained, 4), "peak_source": f"{peak_src} bf16_tflops_sustained",
+        "traffic": None,
+        "frac_of_burst": round(bwd_tflops / peaks["bf16_tflops"], 4),
+    }
+    line["kernels_ms"] = {"permute_in_out": round(perm_ms, 4), "ring_fwd": round(fwd_ms, 4),
+                          "ring_bwd": round(bwd_ms, 4)}
+    line["ring_fwd_tflops"] = round(fwd_tflops, 2)
+    line["e2e"] = {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h}
+    line["gpu_launches"] = step.launches_per_step * args.steps
+    line["clocks"] = clk.summary()
+    del step, q, k, v, do
+    torch.cuda.empty_cache()
+
+    if not args.no_extras:
+        line["extras"] = extras(rm, peaks, peak_src, dev, flush)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample_heads)
+    return line
+
+
+def _time(fn, reps, flush):
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush_l2(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def extras(rm, peaks, peak_src, dev, flush):
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    # LSE merge, striped-128k shapes: per rank 8 fp32 partials [16384, 16, 128] + LSE, 8 ranks
+    Lr, H, d, P = 16384, 16, 128, 8
+    o_parts = [torch.randn(1, P * Lr, H, d, device=dev) for _ in range(P)]
+    lse_parts = [torch.randn(1, H, P * Lr, device=dev) for _ in range(P)]
+    o_out = torch.empty(1, P * Lr, H, d, dtype=torch.bfloat16, device=dev)
+    lse_out = torch.empty(1, H, P * Lr, device=dev)
+    fn = lambda: rm.lse_merge(o_parts, lse_parts, torch.bfloat16, out=o_out, lse_out=lse_out)
+    fn()
+    ms = _time(fn, 5, flush)
+    nbytes = P * (P * Lr * H * d * 4 + H * P * Lr * 4) + P * Lr * H * d * 2 + H * P * Lr * 4
+    out["lse_merge"] = {"shape": "8 partials x [1, 131072, 16, 128] fp32 -> bf16", "ms": round(ms, 4),
+                        "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
+                        "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    del o_parts, lse_parts, o_out, lse_out
+    # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and fused K|V [8 x 32768, 16, 128]
+    x = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
+    y = torch.empty(8, 8 * 32768, 2, 128, dtype=torch.bfloat16, device=dev)
+    fn = lambda: rm.seq_head_repack(x, 8, out=y)
+    fn()
+    ms = _time(fn, 5, flush)
+    nbytes = 2 * x.numel() * 2
+    out["repack"] = {"shape": "seq->head [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16", "ms": round(ms, 4),
+                     "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
+                     "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    del x, y
+    # the causal striped 128k forward (fused ring over 8 virtual ranks)
+    w3 = synthetic.STRIPED_128K
+    q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
+    k = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
+    v = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, w3.Hq, w3.N, device=dev)
+    fn = lambda: rm.ring_attn_fwd(q, k, v, P=8, layout="striped", causal=True, out=o, lse=lse)
+    fn()
+    ms = _time(fn, 3, flush)
+    tf = flops_fwd(w3) / (ms * 1e-3) / 1e12
+    out["striped_128k_fwd"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 2),
+                               "frac": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
+                               "peak_source": f"{peak_src} bf16_tflops (burst: one kernel timed alone)"}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+SAMPLE_ROWS = (4096, 6144)  # local query indices of virtual rank 0 in the sample
+
+
+def oracle_sample(heads: int = 1):
+    """The oracle's ring fwd+bwd for 2048 queries of virtual rank 0 of `heads`
+    query head(s) (with their KV head) of the Llama-like zigzag workload: the
+    queries' partials against both KV shards, their LSE merge, then their
+    backward contributions (their dQ, their share of dK / dV).  The rows are
+    rank 0's local indices 4096..6143, global positions 12288..14335 (the
+    second zigzag chunk), whose score rows are mostly visible.
+    Returns (seconds, algorithmic flops of the sample)."""
+    from oracle import attention as oatt
+    from oracle import layouts as olay
+    from oracle import merge as omerge
+    from oracle import ring as oring
+    w = synthetic.LLAMA_ZIGZAG
+    q, k, v, do = synthetic.attention_inputs(w)
+    hk = max(1, heads // (w.Hq // w.Hkv))
+    f = lambda t, n: t[:, :, :n].float().numpy().astype(np.float64)
+    qs, ks, vs, dos = f(q, heads), f(k, hk), f(v, hk), f(do, heads)
+    L, r = w.N // w.P, 0
+    j0, j1 = SAMPLE_ROWS
+    t0 = time.perf_counter()
+    perm = lambda x: olay.permute(x, w.layout, w.P)
+    qr, kr, vr, dor = perm(qs), perm(ks), perm(vs), perm(dos)
+    pos = [olay.rank_positions(w.layout, w.N, w.P, s) for s in range(w.P)]
+    rows = slice(r * L + j0, r * L + j1)
+    qpos = pos[r][j0:j1]
+    parts = []
+    for s in oring.schedule(w.P)[r]:
+        cols = slice(s * L, (s + 1) * L)
+        parts.append(oatt.attention_forward(qr[:, rows], kr[:, cols], vr[:, cols],
+                                            causal=w.causal, q_pos=qpos, k_pos=pos[s]))
+    o, lse = omerge.lse_merge([a for a, _ in parts], [b for _, b in parts])
+    delta = oatt.delta_from_output(dor[:, rows], o)
+    for s in oring.schedule(w.P)[r]:
+        cols = slice(s * L, (s + 1) * L)
+        oatt.attention_backward_block(qr[:, rows], kr[:, cols], vr[:, cols], dor[:, rows], lse,
+                                      delta, causal=w.causal, q_pos=qpos, k_pos=pos[s])
+    secs = time.perf_counter() - t0
+    # visible pairs: the query at global position t sees t + 1 keys
+    pairs = int((qpos + 1).sum()) * heads
+    return secs, 14.0 * w.d * pairs
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(heads: int):
+    secs, flops = oracle_sample(heads)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions "
+                      f"12288-14335, virtual rank 0) of {heads} of 16 query heads, N=16384 zigzag "
+                      f"P=2; {secs:.1f} s"}
+
+
+def bench_reference(args, world, rank):
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(args.cpu_sample_heads)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        s, f = oracle_sample(args.cpu_sample_heads)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    sample = (f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions 12288-14335, "
+              f"virtual rank 0) of {args.cpu_sample_heads} of 16 query heads, N=16384 zigzag P=2, "
+              f"per step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "llama-causal-zigzag-16k: B=1 Hq=16 Hkv=8 d=128 N=16384 bf16 "
+                               "P=2 zigzag causal fwd+bwd", "global_batch": 1, "seq_len": 16384,
+                   "parallelism": "single"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-heads", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = bench_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_init()
+    line = bench_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

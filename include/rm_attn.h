@@ -143,7 +143,8 @@ rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank,
 
 /* delta[b, h, t] = sum_c dout[b, t, h, c] * o[b, t, h, c] (fp32 accumulate),
  * the row term of the softmax derivative computed from the FINAL output.
- * o / dout in `dtype`, [B, N, H, d]; delta dense fp32 [B, H, N]. */
+ * o / dout in `dtype`, [B, N, H, d], d % 4 == 0, pointers aligned to 4
+ * elements and strides multiples of 4 elements; delta dense fp32 [B, H, N]. */
 rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
                                  rm_tensor o, rm_tensor dout, float* delta,
                                  void* stream);
@@ -157,7 +158,9 @@ rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
  * Parts with lse = -inf get weight 0; if all are -inf, O = 0, LSE = -inf.
  *   o_parts[i]  fp32 [B, Nq, H, d] (strided)     lse_parts[i] fp32 [B, H, Nq]
  *   o_out       out_dtype [B, Nq, H, d]          lse_out      fp32 [B, H, Nq]
- * 1 <= n_parts <= 16; d % 4 == 0, d <= 128; strides multiples of 4 elements.
+ * 1 <= n_parts <= 16; d % 4 == 0, d <= 128; o_parts 16-byte aligned with
+ * strides that are multiples of 4 elements; o_out aligned to 4 elements with
+ * strides that are multiples of 4 elements.
  * o_out may alias o_parts[0] exactly (in-place merge) when out_dtype is fp32;
  * lse_out may alias lse_parts[0]. */
 rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d,

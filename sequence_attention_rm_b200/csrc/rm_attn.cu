@@ -46,8 +46,6 @@ int current_device() {
   return dev < 0 || dev >= kMaxDevices ? 0 : dev;
 }
 
-bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
-
 int esize_of(rm_dtype t) { return t == RM_BF16 ? 2 : 4; }
 
 rm_status check_desc(const rm_attn_desc* d) {
@@ -81,17 +79,18 @@ float eff_scale(const rm_attn_desc* d) {
 }
 
 // A strided [B, rows, H, d] operand: pointer and strides must keep every row
-// 16-byte aligned (TMA and vector access).
-rm_status check_tensor(const char* name, rm_tensor t, int esize, int64_t rows, int heads,
-                       int d) {
+// `align` bytes aligned (16 for TMA operands; 4 elements for the row kernels).
+rm_status check_tensor(const char* name, rm_tensor t, int esize, int64_t rows, int heads, int d,
+                       int align = 16) {
   if (rows == 0) return RM_OK;
   if (!t.ptr) return fail(RM_ERR_INVALID_ARG, "%s: NULL pointer", name);
-  if (!aligned16(t.ptr)) return fail(RM_ERR_INVALID_ARG, "%s: pointer not 16-byte aligned", name);
+  if ((uintptr_t)t.ptr % align)
+    return fail(RM_ERR_INVALID_ARG, "%s: pointer not %d-byte aligned", name, align);
   if (t.stride_b < 0 || t.stride_n <= 0 || t.stride_h < 0)
     return fail(RM_ERR_INVALID_ARG, "%s: negative / zero stride", name);
-  if ((t.stride_b * esize) % 16 || (t.stride_n * esize) % 16 || (t.stride_h * esize) % 16)
-    return fail(RM_ERR_INVALID_ARG, "%s: strides * element size must be multiples of 16 bytes",
-                name);
+  if ((t.stride_b * esize) % align || (t.stride_n * esize) % align || (t.stride_h * esize) % align)
+    return fail(RM_ERR_INVALID_ARG, "%s: strides * element size must be multiples of %d bytes",
+                name, align);
   if (heads > 1 && t.stride_h < d)
     return fail(RM_ERR_INVALID_ARG, "%s: head stride smaller than d (overlapping heads)", name);
   return RM_OK;
@@ -284,7 +283,7 @@ rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d, int 
   a.n_parts = n_parts;
   a.lse_ld = Nq;
   for (int i = 0; i < n_parts; ++i) {
-    RM_TRY(check_tensor("o_parts[i]", o_parts[i], 4, rows, H, d));
+    RM_TRY(check_tensor("o_parts[i]", o_parts[i], 4, rows, H, d, 16));
     if (!lse_parts[i] || ((uintptr_t)lse_parts[i] & 3))
       return fail(RM_ERR_INVALID_ARG, "lse_parts[%d] NULL or misaligned", i);
     a.o_ptr[i] = (const float*)o_parts[i].ptr;
@@ -293,7 +292,7 @@ rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d, int 
     a.o_sh[i] = o_parts[i].stride_h;
     a.lse_ptr[i] = lse_parts[i];
   }
-  RM_TRY(check_tensor("o_out", o_out, out_dtype == RM_BF16 ? 2 : 4, rows, H, d));
+  RM_TRY(check_tensor("o_out", o_out, esize_of(out_dtype), rows, H, d, 4 * esize_of(out_dtype)));
   if (out_dtype == RM_BF16 && o_out.ptr == o_parts[0].ptr)
     return fail(RM_ERR_INVALID_ARG, "in-place merge needs an fp32 output");
   if (!lse_out || ((uintptr_t)lse_out & 3)) return fail(RM_ERR_INVALID_ARG, "lse_out NULL/misaligned");
@@ -313,8 +312,8 @@ rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
     return fail(RM_ERR_INVALID_ARG, "bad sizes (need d %% 4 == 0, 4 <= d <= 128)");
   const int64_t rows = (int64_t)B * N;
   if (rows == 0) return RM_OK;
-  RM_TRY(check_tensor("o", o, esize_of(dtype), rows, H, d));
-  RM_TRY(check_tensor("dout", dout, esize_of(dtype), rows, H, d));
+  RM_TRY(check_tensor("o", o, esize_of(dtype), rows, H, d, 4 * esize_of(dtype)));
+  RM_TRY(check_tensor("dout", dout, esize_of(dtype), rows, H, d, 4 * esize_of(dtype)));
   if (!delta || ((uintptr_t)delta & 3)) return fail(RM_ERR_INVALID_ARG, "delta NULL/misaligned");
   RM_CUDA(launch_bwd_preprocess(dtype == RM_BF16, B, N, H, d, o, dout, delta, nullptr,
                                 (cudaStream_t)stream),
@@ -402,6 +401,8 @@ rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank, r
     RM_CUDA(launch_simt_bwd(a, q_rank, kv_rank, st), "simt bwd launch");
     return RM_OK;
   }
+  if (desc->d != 128)
+    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", desc->d);
   return tc_bwd(a, q_rank, kv_rank, st);
 }
 
@@ -492,6 +493,8 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
   RM_TRY(check_tensor("dk", dk, es, rows, desc->Hkv, desc->d));
   RM_TRY(check_tensor("dv", dv, es, rows, desc->Hkv, desc->d));
   if (!lse) return fail(RM_ERR_INVALID_ARG, "lse NULL");
+  if (desc->dtype == RM_BF16 && desc->d != 128)
+    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", desc->d);
   const BwdWs w = bwd_ws(desc);
   if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
     return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);

@@ -147,3 +147,55 @@ def test_block_backward_fp32_accumulates(rm):
                               causal=causal, q_rank=r, kv_rank=s)
     for name, g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g_ref):
         assert_max_abs(np64(g), ref, 1e-5 * max(1, np.abs(ref).max()), name)
+
+
+BWD_CASES = [c for c in CASES if c[0] == torch.bfloat16 and c[5] == 128]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: f"B{c[1]}H{c[2]}/{c[3]}-N{c[4]}-P{c[6]}-{c[7]}-{'c' if c[8] else 'nc'}")
+def test_ring_backward_bf16(rm, case):
+    dtype, B, Hq, Hkv, N, d, P, layout, causal = case
+    q, k, v, do = _inputs(dtype, B, Hq, Hkv, N, d, 190 + N)
+    g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=causal)
+    perm = lambda x: rm.layout_permute(x.cuda(), layout, P)
+    qg, kg, vg, dog = perm(q), perm(k), perm(v), perm(do)
+    o, l = rm.ring_attn_fwd(qg, kg, vg, P=P, layout=layout, causal=causal)
+    grads = rm.ring_attn_bwd(qg, kg, vg, o, l, dog, P=P, layout=layout, causal=causal)
+    for name, g, ref in zip(("dq", "dk", "dv"), grads, g_ref):
+        assert g.dtype == torch.bfloat16
+        assert_grad_close(np64(rm.layout_permute(g, layout, P, inverse=True)), ref, what=name)
+
+
+def test_block_backward_bf16_every_pair(rm):
+    dtype, B, Hq, Hkv, N, d, P, layout, causal = CASES[4]
+    q, k, v, do = _inputs(dtype, B, Hq, Hkv, N, d, 321)
+    qr, kr, vr, dor = (olay.permute(np64(x), layout, P) for x in (q, k, v, do))
+    o_ref, l_ref = oring.ring_forward(qr, kr, vr, layout, P, causal)
+    g_ref = oring.ring_backward(qr, kr, vr, o_ref, l_ref, dor, layout, P, causal)
+    L = N // P
+    tb = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).cuda()
+    tf = lambda x: torch.from_numpy(np.ascontiguousarray(x)).float().cuda()
+    qg, kg, vg, dog = tb(qr), tb(kr), tb(vr), tb(dor)
+    lse, delta = tf(l_ref), tf(oatt.delta_from_output(dor, o_ref))
+    dq = torch.zeros(qg.shape, dtype=torch.float32, device="cuda")
+    dk = torch.zeros(kg.shape, dtype=torch.float32, device="cuda")
+    dv = torch.zeros(vg.shape, dtype=torch.float32, device="cuda")
+    for r in range(P):
+        rows = slice(r * L, (r + 1) * L)
+        for s in range(P):
+            cols = slice(s * L, (s + 1) * L)
+            rm.attn_block_bwd(qg[:, rows], kg[:, cols], vg[:, cols], dog[:, rows],
+                              lse[:, :, rows].contiguous(), delta[:, :, rows].contiguous(),
+                              dq[:, rows], dk[:, cols], dv[:, cols], N=N, P=P, layout=layout,
+                              causal=causal, q_rank=r, kv_rank=s)
+    for name, g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g_ref):
+        assert_grad_close(np64(g), ref, what=name)
+
+
+def test_bf16_backward_other_head_dims_are_rejected(rm):
+    q, k, v, do = _inputs(torch.bfloat16, 1, 2, 2, 256, 64, 5)
+    qg, kg, vg, dog = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, l = rm.ring_attn_fwd(qg, kg, vg, P=2, layout="contiguous", causal=True)
+    with pytest.raises(rm.RmError) as e:
+        rm.ring_attn_bwd(qg, kg, vg, o, l, dog, P=2, layout="contiguous", causal=True)
+    assert e.value.status == rm.RM_ERR_UNSUPPORTED

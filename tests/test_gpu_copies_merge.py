@@ -11,7 +11,7 @@ from oracle import layouts as olay
 from oracle import merge as omerge
 from oracle import repack as orepack
 from sequence_attention_rm_b200 import synthetic
-from tests._helpers import F32_TOL, assert_max_abs, gpu, np64
+from tests._helpers import BF16_O_TOL, F32_TOL, assert_max_abs, gpu, np64
 
 pytestmark = gpu
 
@@ -86,7 +86,8 @@ def test_lse_merge(rm, out_dtype, n, B, H, Nq, d):
         p[:, 1] = 0.0
     ref_o, ref_l = omerge.lse_merge([np64(o) for o in o_parts], [np64(l) for l in lse_parts])
     o, l = rm.lse_merge([o.cuda() for o in o_parts], [l.cuda() for l in lse_parts], out_dtype)
-    tol = F32_TOL if out_dtype == torch.float32 else 1e-2
+    # bf16 output: O values reach ~8 here, where one bf16 half-ulp is 2^-9 * 8
+    tol = F32_TOL if out_dtype == torch.float32 else BF16_O_TOL
     assert_max_abs(np64(o), ref_o, tol, "merged O")
     assert_max_abs(np64(l), ref_l, 1e-5, "merged LSE")
     assert np.all(np.isneginf(np64(l)[..., 1]))
