@@ -68,6 +68,11 @@ cudaError_t launch_simt_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
 // Backward, same rank convention; accumulates dq (+=) and dk/dv (+=).
 cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
 
+// Short sequences (L <= 16, d <= 64): one warp per (sequence, head), any dtype.
+bool small_seq_supported(int64_t L, int d);
+cudaError_t launch_small_seq_fwd(const AttnArgs& a, int q_rank, int kv_rank, int bf16,
+                                 cudaStream_t stream);
+
 cudaError_t launch_debug_expire_wait(uint32_t spin_limit, unsigned int* status,
                                      cudaStream_t stream);
 

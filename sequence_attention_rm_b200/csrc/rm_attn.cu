@@ -354,6 +354,11 @@ static rm_status block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm
                            int64_t lse_ld, cudaStream_t st) {
   AttnArgs a = attn_args(desc, lse_ld);
   a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = o_f32; a.lse = lse;
+  if (small_seq_supported(desc->N / desc->P, desc->d)) {
+    RM_CUDA(launch_small_seq_fwd(a, q_rank, kv_rank, desc->dtype == RM_BF16, st),
+            "short-sequence fwd launch");
+    return RM_OK;
+  }
   if (desc->dtype == RM_F32) {
     RM_CUDA(launch_simt_fwd(a, q_rank, kv_rank, st), "simt fwd launch");
     return RM_OK;
@@ -428,6 +433,8 @@ rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
     return fail(RM_ERR_UNSUPPORTED, "stepwise mode supports P <= %d", kMaxMergeParts);
   cudaStream_t st = (cudaStream_t)stream;
   const int64_t L = desc->N / desc->P;
+  if (desc->mode == RM_RING_FUSED && desc->P == 1 && small_seq_supported(desc->N, desc->d))
+    return block_fwd(desc, 0, 0, q, k, v, o, desc->dtype == RM_F32, lse, desc->N, st);
   if (desc->mode == RM_RING_FUSED) {
     AttnArgs a = attn_args(desc, desc->N);
     a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = desc->dtype == RM_F32; a.lse = lse;
