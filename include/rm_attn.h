@@ -195,6 +195,24 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
                            rm_tensor dout, rm_tensor dq, rm_tensor dk,
                            rm_tensor dv, void* ws, size_t ws_bytes, void* stream);
 
+/* Ring backward that allocates nothing.  The pages have no counterpart: this
+ * is for callers that cannot allocate device memory -- e.g. a runtime that
+ * reserved all of it for its own pool, or code that must not call cudaMalloc
+ * because that would synchronise the device.  Same arguments and results as
+ * rm_ring_attn_bwd, minus the workspace: the scratch comes from a fixed
+ * 64 MiB device array inside the library, so rm_ring_workspace_size(desc, 1)
+ * must be at most 64 MiB (else RM_ERR_WORKSPACE, nothing launched).
+ * The array is resolved on the first call on each device (with that device
+ * current); make that first call before any stream capture.  Every GPU that
+ * has made a call holds the 64 MiB until the process exits.  All calls share
+ * the one array per device: calls whose kernels overlap on the GPU (several
+ * streams, or several threads) race and give wrong results -- serialise them.
+ * Calls no cudaMalloc / cudaFree / allocating library routine. */
+rm_status rm_ring_attn_bwd_noalloc(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
+                                   rm_tensor v, rm_tensor o, const float* lse,
+                                   rm_tensor dout, rm_tensor dq, rm_tensor dk,
+                                   rm_tensor dv, void* stream);
+
 /* ---- bit-exact layout transforms ---------------------------------------- */
 
 /* Global token order <-> rank-major order (see pos(r, j) above) of a dense

@@ -10,6 +10,7 @@
 namespace rm {
 
 int num_sms();  // SM count of the current device (cached per device)
+void set_last_error(const char* msg);  // reason returned by rm_last_error()
 
 cudaError_t launch_layout_permute(int esize, int B, int64_t N, int H, int d, int layout, int P,
                                   int inverse, const void* in, void* out, cudaStream_t stream);

@@ -161,6 +161,9 @@ rm_tensor offset_rows(rm_tensor t, int64_t rows, int esize) {
 
 }  // namespace
 
+// Records a one-line reason for the calling thread's next rm_last_error().
+void set_last_error(const char* msg) { t_last_error = msg; }
+
 int num_sms() {
   int dev = current_device();
   std::lock_guard<std::mutex> lk(g_mu);

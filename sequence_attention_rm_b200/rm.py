@@ -28,7 +28,7 @@ EXPORTED = (
     "rm_attn_block_fwd", "rm_attn_block_bwd", "rm_attn_bwd_preprocess", "rm_lse_merge",
     "rm_ring_workspace_size", "rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_layout_permute",
     "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
-    "rm_debug_expire_wait",
+    "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc",
 )
 
 
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_seq_head_repack": [i, i, i64, i, i, i, vp, vp, vp],
         "rm_get_device_status": [vp],
         "rm_debug_expire_wait": [ctypes.c_uint32, vp],
+        "rm_ring_attn_bwd_noalloc": [D, T, T, T, T, vp, T, T, T, T, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -244,6 +245,21 @@ def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
     _check(_lib.rm_ring_attn_bwd(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
                                  _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
                                  _stream(stream)))
+    return dq, dk, dv
+
+
+def ring_attn_bwd_noalloc(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
+                          scale: float | None = None, dq=None, dk=None, dv=None, stream=None):
+    """rm_ring_attn_bwd without a workspace: the library's fixed device scratch
+    (at most 64 MiB of workspace) is used instead."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    _check(_lib.rm_ring_attn_bwd_noalloc(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
+                                         _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv),
+                                         _stream(stream)))
     return dq, dk, dv
 
 
