@@ -10,7 +10,8 @@
  *      [Mosaic, "How Ring Attention Works"; Ring Attention & Friends,
  *       "Flash Attention - Tiling with the Softmax Rescaling Trick"]
  *  - LSE merge of partial results, contiguous / head_tail (zigzag) layouts,
- *    the reverse-ring backward, the Ulysses head all-to-all
+ *    the backward that runs the ring in the opposite direction, the Ulysses
+ *    all-to-all on the head dimension
  *      [ringmaster (axolotl-ringmaster 0.2.0), "Why", "Status", "Layout"]
  *  - striped layout (token t on rank t mod P)
  *      [Ring Attention & Friends, "Striped Attention"]
@@ -128,7 +129,7 @@ rm_status rm_attn_block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank,
                             rm_tensor o, int o_f32, float* lse, void* stream);
 
 /* Backward contribution of one (q_rank, kv_rank) pair [ringmaster, "Status":
- * flash-style reverse-ring backward; the derivative of the definition]:
+ * the ring's backward; formulas are the derivative of the definition]:
  *   P_tu = exp(s_tu - lse_final_t);  dP = dO V^T;  dS = P o (dP - delta)
  *   dq_acc += scale dS K;  dk_acc += scale dS^T Q;  dv_acc += P^T dO
  * lse_final / delta: dense fp32 [B, Hq, L] of the query shard (the FINAL LSE
@@ -224,7 +225,7 @@ rm_status rm_layout_permute(rm_dtype dtype, int B, int64_t N, int H, int d,
                             const void* in, void* out, void* stream);
 
 /* Ulysses sequence <-> head repack as a local pack [ringmaster, "Why": the
- * all-to-all on the head dim, capped by the head count].
+ * all-to-all on the head dimension; P may not exceed the head count].
  * head_to_seq = 0 (seq -> head):
  *   in  [P][N_local][H][d]      (rank s's sequence shard of all heads)
  *   out [P][P*N_local][H/P][d]  out[r][s*N_local + t][h] = in[s][t][r*H/P + h]

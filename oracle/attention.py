@@ -5,7 +5,8 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 Definition followed (Mosaic page, "The Problem"): Attention(Q, K, V) =
 softmax(Q K^T / sqrt(d)) V, where the softmax runs over the key axis of each
 query row; the per-row normaliser of that softmax ("Ring Attention & Friends",
-slide "Vanilla Transformer": the row-wise softmax normalisation constant) is
+slide "Vanilla Transformer", which names the per-row constant that normalises
+the softmax) is
 reported as its natural logarithm, the LSE.
 
 Tensor layout (tokens-major, "bshd"): q [B, Nq, Hq, d], k [B, Nk, Hkv, d],
@@ -15,8 +16,8 @@ Readings of points the pages leave open:
 - scale is 1/sqrt(d) with d the true head dimension;
 - LSE is the natural log of sum_u exp(s_tu) over the visible keys;
 - causal: key at global position u is visible to the query at global position
-  t iff u <= t (diagonal inclusive; ringmaster "Status": dense causal
-  sequences).  Global positions are passed in explicitly so that the same
+  t iff u <= t (diagonal inclusive; ringmaster "Status" accepts causal
+  sequences without holes or arbitrary masks).  Global positions are passed in explicitly so that the same
   function serves any shard pair of any layout;
 - grouped-query attention: query head h reads KV head h // (Hq // Hkv)
   (contiguous groups; ringmaster "Quickstart" only names num_kv_heads);

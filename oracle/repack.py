@@ -5,8 +5,8 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 Ulysses (ringmaster "Why") wraps an attention kernel with an all-to-all on the
 head dimension: before attention each of the P ranks holds a sequence shard
 of all H heads; after the all-to-all each rank holds the whole sequence for
-H / P heads (so P may not exceed the head count: the "capped by KV-head count"
-rule).  On one device the all-to-all is a local pack:
+H / P heads (so P may not exceed the head count; the page limits the
+Ulysses degree by the number of KV heads).  On one device the all-to-all is a local pack:
 
     seq -> head:  out[r][s * L + t][h] = in[s][t][r * (H / P) + h]
 

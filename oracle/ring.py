@@ -4,11 +4,13 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 
 Schedule (Mosaic page, "How Ring Attention Works"): rank r starts with its own
 KV shard and, at each step, receives the shard of the rank before it in the
-ring (GPU 0 receives K3, V3 from GPU 3), so at step k = 0..P-1 rank r works
+ring (in the page's 4-GPU example, GPU 0's second chunk is GPU 3's), so at
+step k = 0..P-1 rank r works
 with KV shard (r - k) mod P.  Each step produces a partial (O, LSE) for the
 rank's query shard; the partials are merged with the LSE merge.
 
-Backward (ringmaster "Status": a flash-style reverse-ring backward): every
+Backward (ringmaster "Status" says the p2p ring has a FlashAttention-like
+backward that runs the ring in the opposite direction): every
 (query shard, KV shard) pair rebuilds its probabilities from the final LSE of
 its query rows and uses the row term D_t = dO_t . O_t of the final O; dQ of a
 rank sums over its steps, dK / dV of a shard sum over all ranks that used it

@@ -2,8 +2,8 @@
 // head dim 128.
 //
 // One CTA owns one 128-key tile of one KV head (ringmaster, "Status": the
-// flash-style reverse-ring backward -- the KV shard visits the ranks s, s+1,
-// ..., and every rank's queries add their contribution).  It walks, for every
+// backward runs the ring in the opposite direction -- the KV shard visits the
+// ranks s, s+1, ..., and every rank's queries add their contribution).  It walks, for every
 // query head of the GQA group and every rank in reverse-ring order, the
 // 64-query tiles that can see its keys, recomputing the probabilities from the
 // final LSE:
