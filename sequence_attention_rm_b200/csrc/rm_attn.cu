@@ -131,9 +131,8 @@ BwdWs bwd_ws(const rm_attn_desc* d) {
   const size_t rows_q = (size_t)d->B * d->N * d->Hq;
   w.delta = 0;
   w.dq = align_up(rows_q * 4);
-  // fp32 (SIMT) problems write dQ directly; the tensor-core backward
-  // accumulates dQ in fp32 [B, Hq, N, d] and writes dK / dV itself
-  w.total = d->dtype == RM_F32 ? w.dq : w.dq + align_up(rows_q * d->d * 4);
+  // both backward paths write dQ / dK / dV themselves: delta is all they keep
+  w.total = w.dq;
   return w;
 }
 
@@ -523,15 +522,12 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
     RM_CUDA(launch_simt_bwd(a, -1, -1, st), "simt ring bwd launch");
     return RM_OK;
   }
-  // delta from the final O, and the dQ accumulator ([B, Hq, N, d]) zeroed in the same pass
-  RM_CUDA(launch_bwd_preprocess(1, desc->B, desc->N, desc->Hq, desc->d, o, dout, delta, dq_acc,
+  // delta from the final O, then the dK/dV and dQ kernels write their outputs
+  RM_CUDA(launch_bwd_preprocess(1, desc->B, desc->N, desc->Hq, desc->d, o, dout, delta, nullptr,
                                 st),
           "bwd preprocess launch");
-  rm_tensor dq_t = dense_bhnd(dq_acc, desc->N, desc->Hq, desc->d);
-  a.dq = dq_t; a.dk = dk; a.dv = dv;
-  RM_TRY(tc_bwd(a, -1, -1, st));
-  RM_CUDA(launch_convert_f32(1, desc->B, desc->N, desc->Hq, desc->d, dq_t, dq, st), "dq out");
-  return RM_OK;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  return tc_bwd(a, -1, -1, st);
 }
 
 }  // extern "C"

@@ -12,9 +12,10 @@ bool tc_supported_head_dim(int d);
 // shard pair with shard-local operands.  o is bf16 unless a.o_f32.
 rm_status tc_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
 
-// Backward.  Same rank convention.  dq is an fp32 accumulator (+=, any
-// strides); dk / dv are fp32 accumulators (+=) when a.accumulate, else bf16
-// outputs written once (ring mode: every KV tile owns its complete sums).
+// Backward (head dim 128): a key-stationary dK/dV kernel and a
+// query-stationary dQ kernel.  Same rank convention.  With a.accumulate,
+// dq / dk / dv are fp32 accumulators (+=); otherwise bf16 outputs written once
+// (ring mode: every CTA owns complete sums).
 rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
 
 }  // namespace rm

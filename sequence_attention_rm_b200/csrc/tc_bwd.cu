@@ -1,28 +1,24 @@
 // Backward attention on the sm_100a tensor cores (bf16 in, fp32 accumulate),
-// head dim 128.
+// head dim 128, as two kernels that need no reductions in global memory:
 //
-// One CTA owns one 128-key tile of one KV head (ringmaster, "Status": the
-// backward runs the ring in the opposite direction -- the KV shard visits the
-// ranks s, s+1, ..., and every rank's queries add their contribution).  It walks, for every
-// query head of the GQA group and every rank in reverse-ring order, the
-// 64-query tiles that can see its keys, recomputing the probabilities from the
-// final LSE:
-//   S^T  = K Q^T            (TMEM, keys on lanes)
-//   dP^T = V dO^T           (TMEM)
-//   P^T  = exp(S^T * scale - LSE),  dS^T = P^T o (dP^T - D)
-//   dV  += P^T dO           (A = P^T from TMEM)
-//   dK  += dS^T Q           (A = dS^T from TMEM)
-//   dQ^T = K^T dS^T         (TMEM, head-dim on lanes) -> fp32 reductions to dQ
-// dK and dV stay in TMEM for the whole walk, so they need no atomics; dQ is
-// accumulated with coalesced fp32 reductions (consecutive lanes hold
-// consecutive head-dim columns of one query row).
-//
-// Warp roles (384 threads):
-//   warps 0-3  per-key math (P^T, dS^T), then the dK epilogue
-//   warps 4-7  dQ^T readout and reduction, then the dV epilogue
-//   warp  8    TMA producer: K, V once; Q, dO tiles into a 2-stage ring
-//   warp  9    MMA issuer
-// TMEM: dK [0,128) dV [128,256) S^T x2 [256,384) dP^T [384,448) dQ^T [448,512)
+//  tc_bwd_dkdv_kernel (key-stationary).  One CTA owns one 128-key tile of one
+//    KV head and keeps its dK and dV in TMEM while it walks, for every query
+//    head of the GQA group and every rank in reverse-ring order (s, s+1, ...;
+//    ringmaster, "Status": the backward runs the ring in the opposite
+//    direction), the 64-query tiles that can see its keys:
+//      S^T = K Q^T, dP^T = V dO^T             (TMEM, keys on lanes)
+//      P^T = exp(S^T * scale - LSE),  dS^T = P^T o (dP^T - D)
+//      dV += P^T dO   (A = P^T from TMEM)     dK += dS^T Q   (A = dS^T from smem)
+//  tc_bwd_dq_kernel (query-stationary).  One CTA owns two 128-row query tiles
+//    on one KV head (like the forward) and walks the 64-key tiles they see in
+//    ring order:
+//      S = Q K^T, dP = dO V^T                 (TMEM, queries on lanes)
+//      dS = exp(S * scale - LSE) o (dP - D)   (written over S as bf16)
+//      dQ += dS K     (A = dS from TMEM)
+//    and writes dQ once.
+// S and dP are recomputed by both kernels (7 MMAs per pair instead of 5); in
+// exchange dQ is never reduced through L2, whose fp32 reduce-add throughput
+// (about 1.2 TB/s) bound the fused design, and the result is deterministic.
 #include <cudaTypedefs.h>
 #include <stdlib.h>
 
@@ -39,45 +35,21 @@ namespace {
 
 using namespace tc;
 
-constexpr int D = 128;      // head dim
-constexpr int BK = 128;     // keys per CTA (TMEM lanes)
-constexpr int BQ = 64;      // queries per tile
-constexpr int kThreads = 384;
-constexpr int kWarpTma = 8;
-constexpr int kWarpMma = 9;
-constexpr int kRegsMath = 216;
-constexpr int kRegsOther = 64;
-static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
-
-// shared memory (bytes from a 1024-aligned base)
-constexpr int kKBox = BK * 128;             // 128 key rows x 128 B (64 cols)
-constexpr int kKTile = 2 * kKBox;           // d = 128: two boxes
-constexpr int kQBox = BQ * 128;             // 64 query rows x 128 B
-constexpr int kQTile = 2 * kQBox;
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + kKTile;
-constexpr int kOffQ = kOffV + kKTile;       // [2] stages
-constexpr int kOffDO = kOffQ + 2 * kQTile;  // [2] stages
-constexpr int kOffDS = kOffDO + 2 * kQTile; // dS^T bf16 [128 keys][64 queries], SW128
-constexpr int kDSBytes = BK * 128;
-constexpr int kOffVec = kOffDS + kDSBytes;  // LSE*log2e and D for 2 stages: [2][2][64] fp32
-constexpr int kOffBar = kOffVec + 2 * 2 * BQ * 4;
-constexpr int kSmem = kOffBar + 256 + 1024;
-
-constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384, kTdQ = 448;
+constexpr int D = 128;  // head dim
 
 struct BwdParams {
   int B, Hq, Hkv, P, layout, causal;
   int64_t N, L;
-  float scale;        // softmax scale
-  float scale_log2;   // scale * log2(e)
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
   int ring, q_rank, kv_rank;
-  const float* lse;   // natural-log LSE
+  int head_pairs;    // dQ kernel: the two query tiles are heads (2y, 2y+1)
+  const float* lse;  // natural-log LSE
   const float* delta;
   int64_t lse_ld;
-  float* dq;          // fp32, strided
+  void* dq;          // bf16 output (ring) or fp32 accumulator (block)
   int64_t dq_sb, dq_sn, dq_sh;
-  void* dk;           // bf16 output (ring) or fp32 accumulator (block)
+  void* dk;
   int64_t dk_sb, dk_sn, dk_sh;
   void* dv;
   int64_t dv_sb, dv_sn, dv_sh;
@@ -90,7 +62,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// K-major SW128 operand with rows of 128 B, two 64-column boxes box_bytes apart.
+// K-major SW128 operand with rows of 128 B, 64-column boxes box_bytes apart.
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, int k, uint32_t box_bytes) {
   const int col = k * 16;
   return smem_desc(base + (col / 64) * box_bytes + (col % 64) * 2, 16, 1024, kSwizzle128B);
@@ -102,66 +74,156 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t base, int k, uint32_t box_by
   return smem_desc(base + k * 16 * 128, box_bytes, 1024, kSwizzle128B);
 }
 
+// Writes 32 columns (acc * f) of one dK / dV / dQ row: bf16 output, or an fp32
+// accumulator read-modify-written.
+__device__ __forceinline__ void store_row(void* base, int accumulate, int c32,
+                                          const uint32_t (&v)[32], float f, bool zero) {
+  if (accumulate) {
+    float* dst = reinterpret_cast<float*>(base) + c32 * 32;
+#pragma unroll
+    for (int x = 0; x < 32; ++x) dst[x] += zero ? 0.f : __uint_as_float(v[x]) * f;
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + c32 * 32);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      float y[8];
+#pragma unroll
+      for (int z = 0; z < 8; ++z) y[z] = zero ? 0.f : __uint_as_float(v[8 * x + z]) * f;
+      dst[x] = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
+                          pack_bf16(y[6], y[7]));
+    }
+  }
+}
+
+// ===========================================================================
+// dK / dV (key-stationary)
+// ===========================================================================
+namespace kv {
+
+constexpr int BK = 128;     // keys per CTA (TMEM lanes)
+constexpr int BQ = 64;      // queries per tile
+constexpr int kQStages = 3;
+constexpr int kThreads = 384;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kRegsMath = 200;
+constexpr int kRegsOther = 96;
+static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
+
+constexpr int kKBox = BK * 128;             // 128 key rows x 128 B (64 cols)
+constexpr int kKTile = 2 * kKBox;
+constexpr int kQBox = BQ * 128;             // 64 query rows x 128 B
+constexpr int kQTile = 2 * kQBox;
+constexpr int kDSBytes = BK * 128;          // dS^T bf16 [128 keys][64 queries], SW128
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKTile;
+constexpr int kOffQ = kOffV + kKTile;              // [kQStages]
+constexpr int kOffDO = kOffQ + kQStages * kQTile;  // [kQStages]
+constexpr int kOffDS = kOffDO + kQStages * kQTile; // [2] (one per math warpgroup)
+constexpr int kOffVec = kOffDS + 2 * kDSBytes;     // [wg][2][lse2 | D][64] fp32
+constexpr int kOffBar = kOffVec + 2 * 2 * 2 * BQ * 4;
+constexpr int kSmem = kOffBar + 256 + 1024;
+static_assert(kSmem <= 232448, "shared memory");
+
+constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;  // S, dP: [2] x 64 columns
+
+// The CTA's walk: for every query head of the group, every rank in
+// reverse-ring order, the 64-query tiles that can see key i0.
+struct Walk {
+  LayoutMap lay;
+  int s, g, group, nranks, qtiles, ring, q_rank, P, causal;
+  int64_t tk_first;
+  __device__ __forceinline__ int rank_of(int step) const {
+    return ring ? (s + step) % P : q_rank;
+  }
+  // first query tile of rank r that can see key i0 (later tiles all can)
+  __device__ __forceinline__ int first_tile(int r) const {
+    if (!causal) return 0;
+    return (int)(lay.visible_count(r, tk_first - 1) / BQ);  // queries with pos < tk_first
+  }
+  __device__ __forceinline__ int count() const {
+    int n = 0;
+    for (int step = 0; step < nranks; ++step) n += qtiles - first_tile(rank_of(step));
+    return n * group;
+  }
+  __device__ __forceinline__ void at(int idx, int& h, int& r, int& t) const {
+    for (int hh = 0; hh < group; ++hh)
+      for (int step = 0; step < nranks; ++step) {
+        const int rr = rank_of(step);
+        const int ft = first_tile(rr);
+        if (idx < qtiles - ft) {
+          h = g * group + hh;
+          r = rr;
+          t = ft + idx;
+          return;
+        }
+        idx -= qtiles - ft;
+      }
+    h = g * group;
+    r = rank_of(0);
+    t = 0;
+  }
+};
+
+// Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
+// take alternate query tiles (P^T, dS^T of all 64 columns), then write dK
+// (warps 0-3) and dV (warps 4-7); warp 8 TMA producer (K, V once; Q, dO into
+// a 3-stage ring); warp 9 MMA issuer.  S^T / dP^T are double-buffered in TMEM,
+// one buffer per math warpgroup, so the tensor core computes tile i+1 while
+// tile i's math runs.
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+    tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* bar_kv = bars + 0;
-  uint64_t* bar_q_full = bars + 1;   // [2]
-  uint64_t* bar_q_empty = bars + 3;  // [2]
-  uint64_t* bar_s_full = bars + 5;   // [2] S^T buffers
-  uint64_t* bar_dp_full = bars + 7;
-  uint64_t* bar_p_full = bars + 8;   // P^T in TMEM (128 arrivals)
-  uint64_t* bar_ds_full = bars + 9;  // dS^T in TMEM and smem (128 arrivals)
-  uint64_t* bar_ds_empty = bars + 10;
-  uint64_t* bar_dq_full = bars + 11;
-  uint64_t* bar_dq_empty = bars + 12;  // dQ^T read out (128 arrivals)
-  uint64_t* bar_done = bars + 13;
-  uint64_t* bar_vec = bars + 14;      // [2] LSE / D staged (128 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  float* vec = reinterpret_cast<float*>(smem + kOffVec);  // [stage][0: lse2, 1: D][64]
+  uint64_t* bar_q_full = bars + 1;    // [3]
+  uint64_t* bar_q_empty = bars + 4;   // [3]
+  uint64_t* bar_sd_full = bars + 7;   // [2] S^T and dP^T of a tile in TMEM buffer x
+  uint64_t* bar_p_full = bars + 9;    // [2] P^T written (128 arrivals)
+  uint64_t* bar_ds_full = bars + 11;  // [2] dS^T in smem (128 arrivals)
+  uint64_t* bar_ds_empty = bars + 13; // [2] dK done reading dS^T
+  uint64_t* bar_vec = bars + 15;      // [wg][2] LSE / D staged (128 arrivals)
+  uint64_t* bar_done = bars + 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  float* vec = reinterpret_cast<float*>(smem + kOffVec);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const LayoutMap lay = make_layout(p.layout, p.N, p.P);
+  Walk W;
+  W.lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  const int s = p.ring ? (int)(blockIdx.z % p.P) : p.kv_rank;
+  W.s = p.ring ? (int)(blockIdx.z % p.P) : p.kv_rank;
   const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
-  const int g = blockIdx.y;
-  const int group = p.Hq / p.Hkv;
+  W.g = blockIdx.y;
+  W.group = p.Hq / p.Hkv;
+  W.nranks = p.ring ? p.P : 1;
+  W.qtiles = (int)((L + BQ - 1) / BQ);
+  W.ring = p.ring;
+  W.q_rank = p.q_rank;
+  W.P = p.P;
+  W.causal = p.causal;
   const int64_t i0 = (int64_t)blockIdx.x * BK;  // first key (local index in shard s)
-  const int64_t tk_first = lay.pos(s, i0);
-  const int nranks = p.ring ? p.P : 1;
-  const int qtiles = (int)((L + BQ - 1) / BQ);
+  W.tk_first = W.lay.pos(W.s, i0);
+  const int s = W.s, g = W.g;
   const long long limit = p.wait_limit;
-
-  // first query tile of rank r that can see key i0 (later tiles all can)
-  auto first_tile = [&](int r) -> int {
-    if (!p.causal) return 0;
-    const int64_t before = lay.visible_count(r, tk_first - 1);  // queries with pos < tk_first
-    return (int)(before / BQ);
-  };
-  auto rank_of = [&](int step) { return p.ring ? (s + step) % p.P : p.q_rank; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < kQStages; ++x) {
       mbar_init(bar_q_full + x, 1);
       mbar_init(bar_q_empty + x, 1);
-      mbar_init(bar_s_full + x, 1);
     }
-    mbar_init(bar_dp_full, 1);
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_ds_full, 128);
-    mbar_init(bar_ds_empty, 1);
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_empty, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_sd_full + x, 1);
+      mbar_init(bar_p_full + x, 128);
+      mbar_init(bar_ds_full + x, 128);
+      mbar_init(bar_ds_empty + x, 1);
+    }
+    for (int x = 0; x < 4; ++x) mbar_init(bar_vec + x, 128);
     mbar_init(bar_done, 1);
-    mbar_init(bar_vec + 0, 128);
-    mbar_init(bar_vec + 1, 128);
     fence_barrier_init();
   }
   if (warp == kWarpMma) {
@@ -172,11 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-
-  // total number of query tiles this CTA walks
-  int n = 0;
-  for (int hh = 0; hh < group; ++hh)
-    for (int step = 0; step < nranks; ++step) n += qtiles - first_tile(rank_of(step));
+  const int n = W.count();
 
   if (warp >= 8) {
     regs_dec<kRegsOther>();
@@ -192,303 +250,186 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_5d(smem + kOffV + x * kKBox, &tmV, bar_kv, x * 64, g, (int)i0, ks, b);
       }
       int i = 0;
-      bool ok = true;
-      for (int hh = 0; hh < group && ok; ++hh) {
-        const int h = g * group + hh;
-        for (int step = 0; step < nranks && ok; ++step) {
-          const int r = rank_of(step);
-          const int qs = p.ring ? r : 0;
-          for (int t = first_tile(r); t < qtiles; ++t, ++i) {
-            const int st = i & 1;
-            if (i >= 2 && !mbar_wait(bar_q_empty + st, ((i >> 1) - 1) & 1, limit, p.status)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(bar_q_full + st, 2 * kQTile);
-            for (int x = 0; x < 2; ++x) {
-              tma_load_5d(smem + kOffQ + st * kQTile + x * kQBox, &tmQ, bar_q_full + st, x * 64, h,
-                          t * BQ, qs, b);
-              tma_load_5d(smem + kOffDO + st * kQTile + x * kQBox, &tmDO, bar_q_full + st, x * 64,
-                          h, t * BQ, qs, b);
-            }
-          }
+      for (; i < n; ++i) {
+        const int st = i % kQStages;
+        if (i >= kQStages &&
+            !mbar_wait(bar_q_empty + st, ((i / kQStages) - 1) & 1, limit, p.status))
+          break;
+        int h, r, t;
+        W.at(i, h, r, t);
+        const int qs = p.ring ? r : 0;
+        mbar_arrive_expect_tx(bar_q_full + st, 2 * kQTile);
+        for (int x = 0; x < 2; ++x) {
+          tma_load_5d(smem + kOffQ + st * kQTile + x * kQBox, &tmQ, bar_q_full + st, x * 64, h,
+                      t * BQ, qs, b);
+          tma_load_5d(smem + kOffDO + st * kQTile + x * kQBox, &tmDO, bar_q_full + st, x * 64, h,
+                      t * BQ, qs, b);
         }
       }
+      // drain: every load issued has landed before the CTA exits
       mbar_wait(bar_kv, 0, limit, p.status);
-      for (int st = 0; st < 2 && i > st; ++st) {
-        const int uses = (i - st + 1) / 2;
+      for (int st = 0; st < kQStages && st < i; ++st) {
+        const int uses = (i - st + kQStages - 1) / kQStages;
         mbar_wait(bar_q_full + st, (uses - 1) & 1, limit, p.status);
       }
     } else if (warp == kWarpMma && lane == 0) {
-      constexpr uint32_t idST = idesc_bf16(BK, BQ, 0, 0);   // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16(BK, D, 0, 1);    // dV, dK (A from TMEM)
-      constexpr uint32_t idDQ = idesc_bf16(D, BQ, 1, 1);    // dQ^T = K^T dS^T
+      constexpr uint32_t idST = idesc_bf16(BK, BQ, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16(BK, D, 0, 1);   // dV (A in TMEM), dK (A in smem)
       const uint32_t kA = smem_u32(smem + kOffK), vA = smem_u32(smem + kOffV);
       const uint32_t qB = smem_u32(smem + kOffQ), doB = smem_u32(smem + kOffDO);
       const uint32_t dsB = smem_u32(smem + kOffDS);
-      auto issue_st = [&](int i) {  // S^T(i) and dP^T(i) into their TMEM buffers
-        const int st = i & 1;
+      // S^T(i) and dP^T(i) into TMEM buffer i & 1
+      auto issue_sd = [&](int i) -> bool {
+        const int qst = i % kQStages, x = i & 1;
+        if (!mbar_wait(bar_q_full + qst, (i / kQStages) & 1, limit, p.status)) return false;
+        fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTS + st * BQ, kdesc(kA, k, kKBox), kdesc(qB + st * kQTile, k, kQBox),
+          mma_ss(tmem + kTS + x * BQ, kdesc(kA, k, kKBox), kdesc(qB + qst * kQTile, k, kQBox),
                  idST, k > 0);
-        mma_commit(bar_s_full + st);
-      };
-      auto issue_dp = [&](int i) {
-        const int st = i & 1;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTdP, kdesc(vA, k, kKBox), kdesc(doB + st * kQTile, k, kQBox), idST,
-                 k > 0);
-        mma_commit(bar_dp_full);
+          mma_ss(tmem + kTdP + x * BQ, kdesc(vA, k, kKBox), kdesc(doB + qst * kQTile, k, kQBox),
+                 idST, k > 0);
+        mma_commit(bar_sd_full + x);
+        return true;
       };
       bool ok = mbar_wait(bar_kv, 0, limit, p.status);
-      if (ok && n > 0) {
-        ok = mbar_wait(bar_q_full + 0, 0, limit, p.status);
-        if (ok) {
-          fence_after_sync();
-          issue_st(0);
-          issue_dp(0);
-        }
-      }
+      for (int i = 0; ok && i < 2 && i < n; ++i) ok = issue_sd(i);
       for (int i = 0; ok && i < n; ++i) {
-        const int st = i & 1;
-        if (i + 1 < n) {
-          if (!mbar_wait(bar_q_full + ((i + 1) & 1), ((i + 1) >> 1) & 1, limit, p.status)) break;
-          fence_after_sync();
-          issue_st(i + 1);
-        }
-        if (!mbar_wait(bar_p_full, i & 1, limit, p.status)) break;
+        const int x = i & 1, qst = i % kQStages;
+        if (!mbar_wait(bar_p_full + x, (i >> 1) & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dV += P^T dO
-          mma_ts(tmem + kTdV, tmem + kTS + st * BQ + k * 8, mndesc(doB + st * kQTile, k, kQBox),
+          mma_ts(tmem + kTdV, tmem + kTS + x * BQ + k * 8, mndesc(doB + qst * kQTile, k, kQBox),
                  idKV, (i == 0 && k == 0) ? 0u : 1u);
-        if (!mbar_wait(bar_ds_full, i & 1, limit, p.status)) break;
+        if (!mbar_wait(bar_ds_full + x, (i >> 1) & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dK += dS^T Q
-          mma_ts(tmem + kTdK, tmem + kTdP + k * 8, mndesc(qB + st * kQTile, k, kQBox), idKV,
-                 (i == 0 && k == 0) ? 0u : 1u);
-        mma_commit(bar_q_empty + st);
-        if (i > 0 && !mbar_wait(bar_dq_empty, (i - 1) & 1, limit, p.status)) break;
-        fence_after_sync();
-#pragma unroll
-        for (int k = 0; k < BK / 16; ++k)  // dQ^T = K^T dS^T
-          mma_ss(tmem + kTdQ, mndesc(kA, k, kKBox), mndesc(dsB, k, kDSBytes), idDQ, k > 0);
-        mma_commit(bar_dq_full);
-        mma_commit(bar_ds_empty);
-        if (i + 1 < n) issue_dp(i + 1);
+          mma_ss(tmem + kTdK, kdesc(dsB + x * kDSBytes, k, kDSBytes),
+                 mndesc(qB + qst * kQTile, k, kQBox), idKV, (i == 0 && k == 0) ? 0u : 1u);
+        mma_commit(bar_q_empty + qst);
+        mma_commit(bar_ds_empty + x);
+        if (i + 2 < n && !issue_sd(i + 2)) break;
       }
       mma_commit(bar_done);
+      mbar_wait(bar_done, 0, limit, p.status);  // every MMA done before TMEM is freed
     }
   } else {
     regs_inc<kRegsMath>();
+    const int X = warp >> 2;                 // this warpgroup takes tiles i with i % 2 == X
     const int lane_base = (warp & 3) * 32;
     const uint32_t tl = (uint32_t)lane_base << 16;
-    if (warp < 4) {
-      // ---------------- per-key math ----------------
-      const int64_t key = i0 + lane_base + lane;
-      const bool key_live = key < L;
-      const int64_t tk = key_live ? lay.pos(s, key) : INT64_MAX;
-      int i = 0;
-      bool ok = true;
-      for (int hh = 0; hh < group && ok; ++hh) {
-        const int h = g * group + hh;
-        for (int step = 0; step < nranks && ok; ++step) {
-          const int r = rank_of(step);
-          const int64_t q0 = p.ring ? (int64_t)r * L : 0;
-          // queries of rank r before this key (causal: they do not see it)
-          const int64_t hidden = !p.causal ? 0 : (key_live ? lay.visible_count(r, tk - 1) : L);
-          for (int t = first_tile(r); t < qtiles; ++t, ++i) {
-            const int st = i & 1;
-            const int64_t j0 = (int64_t)t * BQ;
-            // stage LSE * log2(e) and D of the 64 queries (0 past the shard end)
-            {
-              const int c = threadIdx.x & 63;
-              const int which = threadIdx.x >> 6;  // 0: lse, 1: delta
-              const int64_t j = j0 + c;
-              float v = 0.f;
-              if (j < L) {
-                const int64_t idx = ((int64_t)b * p.Hq + h) * p.lse_ld + q0 + j;
-                v = which == 0 ? p.lse[idx] * kLog2e : p.delta[idx];
-              }
-              vec[(st * 2 + which) * BQ + c] = v;
-              mbar_arrive(bar_vec + st);
-              if (!__all_sync(0xffffffffu, mbar_wait(bar_vec + st, (i >> 1) & 1, limit, p.status))) {
-                ok = false;
-                break;
-              }
-            }
-            const float* lse2 = vec + (st * 2 + 0) * BQ;
-            const float* dd = vec + (st * 2 + 1) * BQ;
-            // visible query columns: [lo, hi)
-            const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, BQ);
-            const int hi = key_live ? (int)LayoutMap::min64(L - j0, BQ) : 0;
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + st, (i >> 1) & 1, limit, p.status))) {
-              ok = false;
-              break;
-            }
-            fence_after_sync();
-            float pt[BQ];
-            {
-              uint32_t v[32];
+    const int krow = lane_base + lane;       // key row of the tile (TMEM lane)
+    const int64_t key = i0 + krow;
+    const bool key_live = key < L;
+    const int64_t tk = key_live ? W.lay.pos(s, key) : 0;
+    const int tid = threadIdx.x & 127;
+    bool ok = true;
+    // LSE*log2(e) (tid < 64) or D (tid >= 64) of column tid & 63 of tile idx
+    auto fetch = [&](int idx) -> float {
+      if (idx >= n) return 0.f;
+      int h, r, t;
+      W.at(idx, h, r, t);
+      const int64_t j = (int64_t)t * BQ + (tid & 63);
+      if (j >= L) return 0.f;
+      const int64_t q0 = p.ring ? (int64_t)r * L : 0;
+      const int64_t off = ((int64_t)b * p.Hq + h) * p.lse_ld + q0 + j;
+      return tid < 64 ? p.lse[off] * kLog2e : p.delta[off];
+    };
+    float next = fetch(X);
+    for (int i = X; i < n; i += 2) {
+      const int y = (i >> 1) & 1;  // staging buffer of this warpgroup
+      float* vbuf = vec + (X * 2 + y) * 2 * BQ;
+      vbuf[tid] = next;
+      mbar_arrive(bar_vec + X * 2 + y);
+      next = fetch(i + 2);  // in flight during this tile
+      int h, r, t;
+      W.at(i, h, r, t);
+      const int64_t j0 = (int64_t)t * BQ;
+      // visible query columns [lo, hi) of this key in the tile
+      const int64_t hidden = !p.causal ? 0 : (key_live ? W.lay.visible_count(r, tk - 1) : L);
+      const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, BQ);
+      const int hi = key_live ? (int)LayoutMap::min64(L - j0, BQ) : 0;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_vec + X * 2 + y, (i >> 2) & 1, limit, p.status)) ||
+          !__all_sync(0xffffffffu, mbar_wait(bar_sd_full + X, (i >> 1) & 1, limit, p.status))) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      const float* lse2 = vbuf;
+      const float* dd = vbuf + BQ;
+      float pt[BQ];
 #pragma unroll
-              for (int c = 0; c < BQ / 32; ++c) {
-                tmem_ld32(tmem + tl + kTS + st * BQ + c * 32, v);
-                tmem_wait_ld();
+      for (int c = 0; c < BQ / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + tl + kTS + X * BQ + 32 * c, v);
+        tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                  const int col = c * 32 + x;
-                  const float e = ex2(fmaf(__uint_as_float(v[x]), p.scale_log2, -lse2[col]));
-                  pt[col] = (col >= lo && col < hi) ? e : 0.f;
-                }
-              }
-              uint32_t pk[32];
-#pragma unroll
-              for (int x = 0; x < BQ / 2; ++x) pk[x] = pack_bf16(pt[2 * x], pt[2 * x + 1]);
-              tmem_st32(tmem + tl + kTS + st * BQ, pk);
-              tmem_wait_st();
-            }
-            fence_before_sync();
-            mbar_arrive(bar_p_full);
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_dp_full, i & 1, limit, p.status))) {
-              ok = false;
-              break;
-            }
-            fence_after_sync();
-            uint32_t dsk[BQ / 2];
-            {
-              uint32_t v[32];
-#pragma unroll
-              for (int c = 0; c < BQ / 32; ++c) {
-                tmem_ld32(tmem + tl + kTdP + c * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                  const int col = c * 32 + x;
-                  const float d0 = pt[col] * (__uint_as_float(v[x]) - dd[col]);
-                  const float d1 = pt[col + 1] * (__uint_as_float(v[x + 1]) - dd[col + 1]);
-                  dsk[col / 2] = pack_bf16(d0, d1);
-                }
-              }
-              tmem_st32(tmem + tl + kTdP, dsk);
-            }
-            // dS^T row into smem for the dQ^T MMA (SW128: 16-byte chunk c of
-            // row k lands at chunk c ^ (k & 7) of its 128-byte row)
-            if (!__all_sync(0xffffffffu, i == 0 || mbar_wait(bar_ds_empty, (i - 1) & 1, limit, p.status))) {
-              ok = false;
-              break;
-            }
-            {
-              const int krow = lane_base + lane;
-              uint4* row = reinterpret_cast<uint4*>(smem + kOffDS + krow * 128);
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                row[c ^ (krow & 7)] = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
-            }
-            fence_proxy_async_smem();
-            tmem_wait_st();
-            fence_before_sync();
-            mbar_arrive(bar_ds_full);
-          }
+        for (int e = 0; e < 32; ++e) {
+          const int col = 32 * c + e;
+          const float ex = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -lse2[col]));
+          pt[col] = (col >= lo && col < hi) ? ex : 0.f;
         }
       }
-      // ---------------- dK epilogue ----------------
-      if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
-        fence_after_sync();
-        const int64_t krow = (p.ring ? (int64_t)s * L : 0) + key;
+      {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + tl + kTdK + c * 32, v);
-          tmem_wait_ld();
-          if (!key_live) continue;
-          if (p.accumulate) {
-            float* dst = reinterpret_cast<float*>(p.dk) + b * p.dk_sb + krow * p.dk_sn +
-                         (int64_t)g * p.dk_sh + c * 32;
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(pt[2 * e], pt[2 * e + 1]);
+        tmem_st32(tmem + tl + kTS + X * BQ, pk);
+        tmem_wait_st();
+      }
+      fence_before_sync();
+      mbar_arrive(bar_p_full + X);
+      uint32_t dsk[BQ / 2];
 #pragma unroll
-            for (int x = 0; x < 32; ++x) dst[x] += n > 0 ? __uint_as_float(v[x]) * p.scale : 0.f;
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dk) +
-                                                  b * p.dk_sb + krow * p.dk_sn + (int64_t)g * p.dk_sh +
-                                                  c * 32);
+      for (int c = 0; c < BQ / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + tl + kTdP + X * BQ + 32 * c, v);
+        tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              float f[8];
-#pragma unroll
-              for (int y = 0; y < 8; ++y) f[y] = n > 0 ? __uint_as_float(v[8 * x + y]) * p.scale : 0.f;
-              dst[x] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                  pack_bf16(f[6], f[7]));
-            }
-          }
+        for (int e = 0; e < 32; e += 2) {
+          const int col = 32 * c + e;
+          dsk[col / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - dd[col]),
+                                   pt[col + 1] * (__uint_as_float(v[e + 1]) - dd[col + 1]));
         }
       }
-    } else {
-      // ---------------- dQ^T readout: lane = head-dim column ----------------
-      const int col = lane_base + lane;
-      int i = 0;
-      bool ok = true;
-      for (int hh = 0; hh < group && ok; ++hh) {
-        const int h = g * group + hh;
-        for (int step = 0; step < nranks && ok; ++step) {
-          const int r = rank_of(step);
-          const int64_t q0 = p.ring ? (int64_t)r * L : 0;
-          for (int t = first_tile(r); t < qtiles; ++t, ++i) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_dq_full, i & 1, limit, p.status))) {
-              ok = false;
-              break;
-            }
-            fence_after_sync();
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tmem + tl + kTdQ, v0);
-            tmem_ld32(tmem + tl + kTdQ + 32, v1);
-            tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(bar_dq_empty);
-            const int64_t j0 = (int64_t)t * BQ;
-            float* base = p.dq + b * p.dq_sb + (int64_t)h * p.dq_sh + (q0 + j0) * p.dq_sn + col;
-            const int nq = (int)LayoutMap::min64(L - j0, BQ);
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-              if (x < nq) atomicAdd(base + x * p.dq_sn, __uint_as_float(v0[x]) * p.scale);
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-              if (32 + x < nq) atomicAdd(base + (32 + x) * p.dq_sn, __uint_as_float(v1[x]) * p.scale);
-          }
-        }
+      fence_before_sync();
+      // dS^T row of this key into smem (SW128: 16-byte chunk c of row k lands
+      // at chunk c ^ (k & 7) of its 128-byte row)
+      if (i >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(bar_ds_empty + X, ((i >> 1) - 1) & 1, limit, p.status))) {
+        ok = false;
+        break;
       }
-      // ---------------- dV epilogue: lane = key ----------------
-      if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
-        fence_after_sync();
-        const int64_t key = i0 + lane_base + lane;
-        const bool key_live = key < L;
-        const int64_t krow = (p.ring ? (int64_t)s * L : 0) + key;
+      {
+        uint4* row = reinterpret_cast<uint4*>(smem + kOffDS + X * kDSBytes + krow * 128);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + tl + kTdV + c * 32, v);
-          tmem_wait_ld();
-          if (!key_live) continue;
-          if (p.accumulate) {
-            float* dst = reinterpret_cast<float*>(p.dv) + b * p.dv_sb + krow * p.dv_sn +
-                         (int64_t)g * p.dv_sh + c * 32;
+        for (int c = 0; c < 8; ++c)
+          row[c ^ (krow & 7)] = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_ds_full + X);
+    }
+    // ---------------- epilogue: dK (warps 0-3), dV (warps 4-7); lane = key ----------------
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
+      fence_after_sync();
+      const uint32_t tcol = X == 0 ? kTdK : kTdV;
+      const float f = X == 0 ? p.scale : 1.0f;
+      const int es = p.accumulate ? 4 : 2;
+      const int64_t row = (p.ring ? (int64_t)s * L : 0) + key;
+      char* base = X == 0 ? reinterpret_cast<char*>(p.dk) +
+                                (b * p.dk_sb + row * p.dk_sn + (int64_t)g * p.dk_sh) * es
+                          : reinterpret_cast<char*>(p.dv) +
+                                (b * p.dv_sb + row * p.dv_sn + (int64_t)g * p.dv_sh) * es;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) dst[x] += n > 0 ? __uint_as_float(v[x]) : 0.f;
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dv) +
-                                                  b * p.dv_sb + krow * p.dv_sn + (int64_t)g * p.dv_sh +
-                                                  c * 32);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              float f[8];
-#pragma unroll
-              for (int y = 0; y < 8; ++y) f[y] = n > 0 ? __uint_as_float(v[8 * x + y]) : 0.f;
-              dst[x] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                  pack_bf16(f[6], f[7]));
-            }
-          }
-        }
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + tl + tcol + c * 32, v);
+        tmem_wait_ld();
+        if (key_live) store_row(base, p.accumulate, c, v, f, n == 0);
       }
     }
   }
@@ -500,6 +441,278 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+}  // namespace kv
+
+// ===========================================================================
+// dQ (query-stationary)
+// ===========================================================================
+namespace dq {
+
+constexpr int BM = 128;     // query rows per tile (TMEM lanes)
+constexpr int BN = 64;      // keys per KV tile
+constexpr int kStages = 2;
+constexpr int kThreads = 384;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kRegsMath = 216;
+constexpr int kRegsOther = 64;
+static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
+
+constexpr int kQBox = BM * 128;             // 128 query rows x 128 B
+constexpr int kQTile = 2 * kQBox;           // d = 128
+constexpr int kKBox = BN * 128;             // 64 key rows x 128 B
+constexpr int kKTile = 2 * kKBox;
+constexpr int kOffQ = 0;                    // [2] query tiles
+constexpr int kOffDO = kOffQ + 2 * kQTile;  // [2]
+constexpr int kOffK = kOffDO + 2 * kQTile;  // [kStages]
+constexpr int kOffV = kOffK + kStages * kKTile;
+constexpr int kOffBar = kOffV + kStages * kKTile;
+constexpr int kSmem = kOffBar + 256 + 1024;
+static_assert(kSmem <= 232448, "shared memory");
+
+// TMEM per query tile X: S [X*256, +64), dP [X*256 + 64, +64), dQ [X*256 + 128, +128)
+__device__ __forceinline__ uint32_t tS(int x) { return x * 256; }
+__device__ __forceinline__ uint32_t tdP(int x) { return x * 256 + 64; }
+__device__ __forceinline__ uint32_t tdQ(int x) { return x * 256 + 128; }
+
+// Warp roles (384 threads): warps 0-3 / 4-7 own query tiles A / B (one thread
+// per query row: dS = P o (dP - D) from S and dP, written over S as bf16;
+// then the dQ epilogue); warp 8 TMA producer (Q, dO once; K, V 64-key tiles
+// into a 2-stage ring); warp 9 MMA issuer.
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                     const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bar_q = bars + 0;
+  uint64_t* bar_kv_full = bars + 1;   // [2]
+  uint64_t* bar_kv_empty = bars + 3;  // [2]
+  uint64_t* bar_sd_full = bars + 5;   // [2] S and dP of query tile X in TMEM
+  uint64_t* bar_ds_full = bars + 7;   // [2] dS written (128 arrivals)
+  uint64_t* bar_done = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const LayoutMap lay = make_layout(p.layout, p.N, p.P);
+  const int64_t L = p.L;
+  const int r = p.ring ? (int)(blockIdx.z % p.P) : p.q_rank;
+  const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
+  const int unit = gridDim.x - 1 - blockIdx.x;  // later rows see more keys: start them first
+  int hA, hB;
+  int64_t rowA, rowB;
+  if (p.head_pairs) {
+    hA = 2 * blockIdx.y;
+    hB = hA + 1;
+    rowA = rowB = (int64_t)unit * BM;
+  } else {
+    hA = hB = blockIdx.y;
+    rowA = (int64_t)unit * 2 * BM;
+    rowB = rowA + BM;
+  }
+  const int g = hA / (p.Hq / p.Hkv);
+  const int64_t last_row = LayoutMap::min64((p.head_pairs ? rowA : rowB) + BM - 1, L - 1);
+  const int64_t t_last = lay.pos(r, last_row);
+  const int nsteps = p.ring ? p.P : 1;
+  const long long limit = p.wait_limit;
+  auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
+  auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_kv_full + x, 1);
+      mbar_init(bar_kv_empty + x, 1);
+      mbar_init(bar_sd_full + x, 1);
+      mbar_init(bar_ds_full + x, 128);
+    }
+    mbar_init(bar_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_dec<kRegsOther>();
+    if (warp == kWarpTma && lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDO);
+      const int qs = p.ring ? r : 0;
+      mbar_arrive_expect_tx(bar_q, 4 * kQTile);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_5d(smem + kOffQ + x * kQBox, &tmQ, bar_q, x * 64, hA, (int)rowA, qs, b);
+        tma_load_5d(smem + kOffQ + kQTile + x * kQBox, &tmQ, bar_q, x * 64, hB, (int)rowB, qs, b);
+        tma_load_5d(smem + kOffDO + x * kQBox, &tmDO, bar_q, x * 64, hA, (int)rowA, qs, b);
+        tma_load_5d(smem + kOffDO + kQTile + x * kQBox, &tmDO, bar_q, x * 64, hB, (int)rowB, qs, b);
+      }
+      int j = 0;
+      bool ok = true;
+      for (int step = 0; step < nsteps && ok; ++step) {
+        const int s = shard_of(step);
+        const int nt = (int)((cta_keys(s) + BN - 1) / BN);
+        const int ks = p.ring ? s : 0;
+        for (int t = 0; t < nt; ++t, ++j) {
+          const int st = j & 1;
+          if (j >= kStages && !mbar_wait(bar_kv_empty + st, ((j >> 1) - 1) & 1, limit, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_kv_full + st, 2 * kKTile);
+          for (int x = 0; x < 2; ++x) {
+            tma_load_5d(smem + kOffK + st * kKTile + x * kKBox, &tmK, bar_kv_full + st, x * 64, g,
+                        t * BN, ks, b);
+            tma_load_5d(smem + kOffV + st * kKTile + x * kKBox, &tmV, bar_kv_full + st, x * 64, g,
+                        t * BN, ks, b);
+          }
+        }
+      }
+      mbar_wait(bar_q, 0, limit, p.status);
+      for (int st = 0; st < kStages && j > st; ++st) {
+        const int uses = (j - st + 1) / 2;
+        mbar_wait(bar_kv_full + st, (uses - 1) & 1, limit, p.status);
+      }
+    } else if (warp == kWarpMma && lane == 0) {
+      constexpr uint32_t idSD = idesc_bf16(BM, BN, 0, 0);  // S, dP
+      constexpr uint32_t idQ = idesc_bf16(BM, D, 0, 1);    // dQ += dS K (A in TMEM)
+      const uint32_t qA = smem_u32(smem + kOffQ), doA = smem_u32(smem + kOffDO);
+      const uint32_t kB = smem_u32(smem + kOffK), vB = smem_u32(smem + kOffV);
+      int n = 0;
+      for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + BN - 1) / BN);
+      auto issue_sd = [&](int x, int st) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + tS(x), kdesc(qA + x * kQTile, k, kQBox), kdesc(kB + st * kKTile, k, kKBox),
+                 idSD, k > 0);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + tdP(x), kdesc(doA + x * kQTile, k, kQBox), kdesc(vB + st * kKTile, k, kKBox),
+                 idSD, k > 0);
+        mma_commit(bar_sd_full + x);
+      };
+      auto issue_dq = [&](int x, int st, bool first) {
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          mma_ts(tmem + tdQ(x), tmem + tS(x) + k * 8, mndesc(kB + st * kKTile, k, kKBox), idQ,
+                 (first && k == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(bar_q, 0, limit, p.status);
+      if (ok && n > 0) {
+        ok = mbar_wait(bar_kv_full + 0, 0, limit, p.status);
+        if (ok) {
+          fence_after_sync();
+          issue_sd(0, 0);
+          issue_sd(1, 0);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j & 1, nx = (j + 1) & 1;
+        if (!mbar_wait(bar_ds_full + 0, j & 1, limit, p.status)) break;
+        fence_after_sync();
+        issue_dq(0, st, j == 0);
+        if (j + 1 < n) {
+          if (!mbar_wait(bar_kv_full + nx, ((j + 1) >> 1) & 1, limit, p.status)) break;
+          fence_after_sync();
+          issue_sd(0, nx);
+        }
+        if (!mbar_wait(bar_ds_full + 1, j & 1, limit, p.status)) break;
+        fence_after_sync();
+        issue_dq(1, st, j == 0);
+        mma_commit(bar_kv_empty + st);
+        if (j + 1 < n) issue_sd(1, nx);
+      }
+      mma_commit(bar_done);
+      mbar_wait(bar_done, 0, limit, p.status);
+    }
+  } else {
+    regs_inc<kRegsMath>();
+    const int X = warp >> 2;
+    const int lane_base = (warp & 3) * 32;
+    const uint32_t tl = (uint32_t)lane_base << 16;
+    const int64_t row = (X ? rowB : rowA) + lane_base + lane;
+    const int h = X ? hB : hA;
+    const bool live = row < L;
+    const int64_t tq = live ? lay.pos(r, row) : -1;
+    const int64_t qrow = (p.ring ? (int64_t)r * L : 0) + row;
+    float lse2 = 0.f, dd = 0.f;
+    if (live) {
+      const int64_t off = ((int64_t)b * p.Hq + h) * p.lse_ld + qrow;
+      lse2 = p.lse[off] * kLog2e;
+      dd = p.delta[off];
+    }
+    int j = 0, n = 0;
+    bool ok = true;
+    for (int step = 0; step < nsteps && ok; ++step) {
+      const int s = shard_of(step);
+      const int nt = (int)((cta_keys(s) + BN - 1) / BN);
+      n += nt;
+      const int64_t row_keys = !live ? 0 : (p.causal ? lay.visible_count(s, tq) : L);
+      for (int t = 0; t < nt; ++t, ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_sd_full + X, j & 1, limit, p.status))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        const int64_t nvalid = row_keys - (int64_t)t * BN;  // visible keys of this tile: [0, nvalid)
+        uint32_t sv[32], dv[32], ds[16];
+        // dS over the 64 keys in two halves; each half's bf16 goes to the
+        // S columns that half has already been read from
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tmem + tl + tS(X) + 32 * c, sv);
+          tmem_ld32(tmem + tl + tdP(X) + 32 * c, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int col = 32 * c + e;
+            float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lse2));
+            float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.scale_log2, -lse2));
+            p0 = col < nvalid ? p0 : 0.f;
+            p1 = col + 1 < nvalid ? p1 : 0.f;
+            ds[e / 2] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dd),
+                                  p1 * (__uint_as_float(dv[e + 1]) - dd));
+          }
+          tmem_st16(tmem + tl + tS(X) + 16 * c, ds);
+        }
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(bar_ds_full + X);
+      }
+    }
+    // ---------------- epilogue: dQ = scale * acc ----------------
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
+      fence_after_sync();
+      const int es = p.accumulate ? 4 : 2;
+      char* base = reinterpret_cast<char*>(p.dq) +
+                   (b * p.dq_sb + qrow * p.dq_sn + (int64_t)h * p.dq_sh) * es;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + tl + tdQ(X) + c * 32, v);
+        tmem_wait_ld();
+        if (live) store_row(base, p.accumulate, c, v, p.scale, n == 0);
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dq
+
 }  // namespace
 
 rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream) {
@@ -508,12 +721,6 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   const bool ring = q_rank < 0;
   const int64_t L = a.N / a.P;
   const int shards = ring ? a.P : 1;
-  CUtensorMap mq, mk, mv, mdo;
-  if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, BQ) != RM_OK ||
-      encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, BK) != RM_OK ||
-      encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, BK) != RM_OK ||
-      encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, BQ) != RM_OK)
-    return RM_ERR_CUDA;
   BwdParams p;
   p.B = a.B;
   p.Hq = a.Hq;
@@ -528,10 +735,11 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.ring = ring ? 1 : 0;
   p.q_rank = q_rank;
   p.kv_rank = kv_rank;
+  p.head_pairs = ((a.Hq / a.Hkv) % 2 == 0) ? 1 : 0;
   p.lse = a.lse_in;
   p.delta = a.delta;
   p.lse_ld = a.lse_ld;
-  p.dq = reinterpret_cast<float*>(a.dq.ptr);
+  p.dq = a.dq.ptr;
   p.dq_sb = a.dq.stride_b;
   p.dq_sn = a.dq.stride_n;
   p.dq_sh = a.dq.stride_h;
@@ -546,12 +754,37 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.accumulate = a.accumulate;
   p.status = a.status;
   p.wait_limit = tc_wait_limit();
-  dim3 grid((unsigned)ceil_div(L, BK), (unsigned)a.Hkv, (unsigned)(ring ? a.B * a.P : a.B));
-  if (cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
-      cudaSuccess)
-    return RM_ERR_CUDA;
-  tc_bwd_kernel<<<grid, kThreads, kSmem, stream>>>(mq, mk, mv, mdo, p);
-  return cudaGetLastError() == cudaSuccess ? RM_OK : RM_ERR_CUDA;
+  {  // dK, dV
+    CUtensorMap mq, mk, mv, mdo;
+    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
+        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK)
+      return RM_ERR_CUDA;
+    dim3 grid((unsigned)ceil_div(L, kv::BK), (unsigned)a.Hkv, (unsigned)(ring ? a.B * a.P : a.B));
+    if (cudaFuncSetAttribute(kv::tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kv::kSmem) != cudaSuccess)
+      return RM_ERR_CUDA;
+    kv::tc_bwd_dkdv_kernel<<<grid, kv::kThreads, kv::kSmem, stream>>>(mq, mk, mv, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
+  }
+  {  // dQ
+    CUtensorMap mq, mk, mv, mdo;
+    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
+        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK)
+      return RM_ERR_CUDA;
+    const int units = p.head_pairs ? ceil_div(L, dq::BM) : ceil_div(L, 2 * dq::BM);
+    dim3 grid((unsigned)units, (unsigned)(p.head_pairs ? a.Hq / 2 : a.Hq),
+              (unsigned)(ring ? a.B * a.P : a.B));
+    if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dq::kSmem) != cudaSuccess)
+      return RM_ERR_CUDA;
+    dq::tc_bwd_dq_kernel<<<grid, dq::kThreads, dq::kSmem, stream>>>(mq, mk, mv, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
+  }
+  return RM_OK;
 }
 
 }  // namespace rm

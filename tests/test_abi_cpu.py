@@ -75,8 +75,8 @@ def test_workspace_sizes(rm):
     assert lib.rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0
     assert n.value == 0  # fused forward needs no workspace
     assert lib.rm_ring_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == 0
-    # delta [B, Hq, N] + fp32 dQ accumulator [B, Hq, N, d]
-    assert n.value == 16 * 16384 * 4 + 16 * 16384 * 128 * 4
+    # delta [B, Hq, N]: the backward kernels write dQ / dK / dV directly
+    assert n.value == 16 * 16384 * 4
     d = _desc(rm, mode=1)
     assert lib.rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0
     assert n.value == 2 * 16 * 16384 * 128 * 4 + 2 * 16 * 16384 * 4

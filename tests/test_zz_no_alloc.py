@@ -59,11 +59,13 @@ def test_no_alloc_backward_matches_the_workspace_backward(rm):
 
 def test_no_alloc_rejects_problems_beyond_its_scratch(rm):
     lib = rm.raw()
-    # workspace = delta + fp32 dQ accumulator = 16 * 16384 * (4 + 128 * 4) bytes > 64 MiB
-    dsc = rm.desc(torch.bfloat16, 1, 16, 8, 128, 16384, 2, "zigzag", True)
+    # workspace = delta [B, Hq, N] fp32 = 16 * 2^21 * 4 bytes = 128 MiB > 64 MiB
+    n = 1 << 21
+    dsc = rm.desc(torch.bfloat16, 1, 16, 8, 128, n, 2, "zigzag", True)
+    assert rm.ring_workspace_size(dsc, True) > 64 << 20
     T = rm.RmTensor
     x = torch.empty(16, device="cuda")
-    t = T(x.data_ptr(), 16384 * 16 * 128, 16 * 128, 128)
+    t = T(x.data_ptr(), n * 16 * 128, 16 * 128, 128)
     nul = ctypes.c_void_p(0)
     status = lib.rm_ring_attn_bwd_noalloc(ctypes.byref(dsc), t, t, t, t, nul, t, t, t, t, nul)
     assert status == rm.RM_ERR_WORKSPACE
