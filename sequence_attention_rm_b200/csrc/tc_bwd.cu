@@ -62,17 +62,21 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// K-major SW128 operand with rows of 128 B, 64-column boxes box_bytes apart.
-__device__ __forceinline__ uint64_t kdesc(uint32_t base, int k, uint32_t box_bytes) {
-  const int col = k * 16;
-  return smem_desc(base + (col / 64) * box_bytes + (col % 64) * 2, 16, 1024, kSwizzle128B);
+// K-major SW128 operand with rows of 128 B, 64-column boxes box_bytes apart:
+// base descriptor, and the byte offset of K-step k (16 elements).
+__device__ __forceinline__ uint64_t kdesc0(uint32_t base) {
+  return smem_desc(base, 16, 1024, kSwizzle128B);
+}
+__device__ __forceinline__ uint32_t koff(int k, uint32_t box_bytes) {
+  return (k * 16 / 64) * box_bytes + (k * 16 % 64) * 2;
 }
 // MN-major SW128 operand: rows of 128 B along the contiguous (M or N) axis, the
 // K axis along rows; K-step k starts 16 rows later; 64-element blocks of the
 // contiguous axis are box_bytes apart.
-__device__ __forceinline__ uint64_t mndesc(uint32_t base, int k, uint32_t box_bytes) {
-  return smem_desc(base + k * 16 * 128, box_bytes, 1024, kSwizzle128B);
+__device__ __forceinline__ uint64_t mndesc0(uint32_t base, uint32_t box_bytes) {
+  return smem_desc(base, box_bytes, 1024, kSwizzle128B);
 }
+__device__ __forceinline__ uint32_t mnoff(int k) { return k * 16 * 128; }
 
 // Writes 32 columns (acc * f) of one dK / dV / dQ row: bf16 output, or an fp32
 // accumulator read-modify-written.
@@ -146,23 +150,34 @@ struct Walk {
     for (int step = 0; step < nranks; ++step) n += qtiles - first_tile(rank_of(step));
     return n * group;
   }
-  __device__ __forceinline__ void at(int idx, int& h, int& r, int& t) const {
-    for (int hh = 0; hh < group; ++hh)
-      for (int step = 0; step < nranks; ++step) {
-        const int rr = rank_of(step);
-        const int ft = first_tile(rr);
-        if (idx < qtiles - ft) {
-          h = g * group + hh;
-          r = rr;
-          t = ft + idx;
-          return;
-        }
-        idx -= qtiles - ft;
+  // A position in the walk, advanced one tile at a time (no rescans).
+  struct Cursor {
+    int hh, step, r, t;
+  };
+  __device__ __forceinline__ void settle(Cursor& c) const {
+    while (c.t >= qtiles && c.hh < group) {
+      if (++c.step == nranks) {
+        c.step = 0;
+        ++c.hh;
       }
-    h = g * group;
-    r = rank_of(0);
-    t = 0;
+      c.r = rank_of(c.step);
+      c.t = first_tile(c.r);
+    }
   }
+  __device__ __forceinline__ Cursor begin() const {
+    Cursor c;
+    c.hh = 0;
+    c.step = 0;
+    c.r = rank_of(0);
+    c.t = first_tile(c.r);
+    settle(c);
+    return c;
+  }
+  __device__ __forceinline__ void next(Cursor& c) const {
+    ++c.t;
+    settle(c);
+  }
+  __device__ __forceinline__ int head(const Cursor& c) const { return g * group + c.hh; }
 };
 
 // Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
@@ -250,14 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_5d(smem + kOffV + x * kKBox, &tmV, bar_kv, x * 64, g, (int)i0, ks, b);
       }
       int i = 0;
-      for (; i < n; ++i) {
+      Walk::Cursor cur = W.begin();
+      for (; i < n; ++i, W.next(cur)) {
         const int st = i % kQStages;
         if (i >= kQStages &&
             !mbar_wait(bar_q_empty + st, ((i / kQStages) - 1) & 1, limit, p.status))
           break;
-        int h, r, t;
-        W.at(i, h, r, t);
-        const int qs = p.ring ? r : 0;
+        const int h = W.head(cur), t = cur.t;
+        const int qs = p.ring ? cur.r : 0;
         mbar_arrive_expect_tx(bar_q_full + st, 2 * kQTile);
         for (int x = 0; x < 2; ++x) {
           tma_load_5d(smem + kOffQ + st * kQTile + x * kQBox, &tmQ, bar_q_full + st, x * 64, h,
@@ -275,9 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma && lane == 0) {
       constexpr uint32_t idST = idesc_bf16(BK, BQ, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKV = idesc_bf16(BK, D, 0, 1);   // dV (A in TMEM), dK (A in smem)
-      const uint32_t kA = smem_u32(smem + kOffK), vA = smem_u32(smem + kOffV);
-      const uint32_t qB = smem_u32(smem + kOffQ), doB = smem_u32(smem + kOffDO);
-      const uint32_t dsB = smem_u32(smem + kOffDS);
+      const uint64_t kAd = kdesc0(smem_u32(smem + kOffK)), vAd = kdesc0(smem_u32(smem + kOffV));
+      const uint64_t qBd = kdesc0(smem_u32(smem + kOffQ)), doBd = kdesc0(smem_u32(smem + kOffDO));
+      const uint64_t qMNd = mndesc0(smem_u32(smem + kOffQ), kQBox);
+      const uint64_t doMNd = mndesc0(smem_u32(smem + kOffDO), kQBox);
+      const uint64_t dsAd = kdesc0(smem_u32(smem + kOffDS));
       // S^T(i) and dP^T(i) into TMEM buffer i & 1
       auto issue_sd = [&](int i) -> bool {
         const int qst = i % kQStages, x = i & 1;
@@ -285,12 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTS + x * BQ, kdesc(kA, k, kKBox), kdesc(qB + qst * kQTile, k, kQBox),
-                 idST, k > 0);
+          mma_ss(tmem + kTS + x * BQ, desc_add(kAd, koff(k, kKBox)),
+                 desc_add(qBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTdP + x * BQ, kdesc(vA, k, kKBox), kdesc(doB + qst * kQTile, k, kQBox),
-                 idST, k > 0);
+          mma_ss(tmem + kTdP + x * BQ, desc_add(vAd, koff(k, kKBox)),
+                 desc_add(doBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
         mma_commit(bar_sd_full + x);
         return true;
       };
@@ -302,14 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dV += P^T dO
-          mma_ts(tmem + kTdV, tmem + kTS + x * BQ + k * 8, mndesc(doB + qst * kQTile, k, kQBox),
-                 idKV, (i == 0 && k == 0) ? 0u : 1u);
+          mma_ts(tmem + kTdV, tmem + kTS + x * BQ + k * 8,
+                 desc_add(doMNd, qst * kQTile + mnoff(k)), idKV, (i == 0 && k == 0) ? 0u : 1u);
         if (!mbar_wait(bar_ds_full + x, (i >> 1) & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dK += dS^T Q
-          mma_ss(tmem + kTdK, kdesc(dsB + x * kDSBytes, k, kDSBytes),
-                 mndesc(qB + qst * kQTile, k, kQBox), idKV, (i == 0 && k == 0) ? 0u : 1u);
+          mma_ss(tmem + kTdK, desc_add(dsAd, x * kDSBytes + koff(k, kDSBytes)),
+                 desc_add(qMNd, qst * kQTile + mnoff(k)), idKV, (i == 0 && k == 0) ? 0u : 1u);
         mma_commit(bar_q_empty + qst);
         mma_commit(bar_ds_empty + x);
         if (i + 2 < n && !issue_sd(i + 2)) break;
@@ -328,39 +345,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t tk = key_live ? W.lay.pos(s, key) : 0;
     const int tid = threadIdx.x & 127;
     bool ok = true;
-    // LSE*log2(e) (tid < 64) or D (tid >= 64) of column tid & 63 of tile idx
-    auto fetch = [&](int idx) -> float {
+    // LSE*log2(e) (tid < 64) or D (tid >= 64) of column tid & 63 of the tile at c
+    auto fetch = [&](const Walk::Cursor& c, int idx) -> float {
       if (idx >= n) return 0.f;
-      int h, r, t;
-      W.at(idx, h, r, t);
-      const int64_t j = (int64_t)t * BQ + (tid & 63);
+      const int64_t j = (int64_t)c.t * BQ + (tid & 63);
       if (j >= L) return 0.f;
-      const int64_t q0 = p.ring ? (int64_t)r * L : 0;
-      const int64_t off = ((int64_t)b * p.Hq + h) * p.lse_ld + q0 + j;
+      const int64_t q0 = p.ring ? (int64_t)c.r * L : 0;
+      const int64_t off = ((int64_t)b * p.Hq + W.head(c)) * p.lse_ld + q0 + j;
       return tid < 64 ? p.lse[off] * kLog2e : p.delta[off];
     };
-    float next = fetch(X);
+    // this warpgroup's tiles: cur walks X, X+2, ...; ahead runs two tiles in front
+    Walk::Cursor cur = W.begin();
+    if (X == 1) W.next(cur);
+    Walk::Cursor ahead = cur;
+    W.next(ahead);
+    W.next(ahead);
+    float next = fetch(cur, X);
     for (int i = X; i < n; i += 2) {
       const int y = (i >> 1) & 1;  // staging buffer of this warpgroup
       float* vbuf = vec + (X * 2 + y) * 2 * BQ;
       vbuf[tid] = next;
       mbar_arrive(bar_vec + X * 2 + y);
-      next = fetch(i + 2);  // in flight during this tile
-      int h, r, t;
-      W.at(i, h, r, t);
+      next = fetch(ahead, i + 2);  // in flight during this tile
+      const int r = cur.r, t = cur.t;
       const int64_t j0 = (int64_t)t * BQ;
       // visible query columns [lo, hi) of this key in the tile
       const int64_t hidden = !p.causal ? 0 : (key_live ? W.lay.visible_count(r, tk - 1) : L);
       const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, BQ);
       const int hi = key_live ? (int)LayoutMap::min64(L - j0, BQ) : 0;
+      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == BQ);
+      W.next(cur);
+      W.next(cur);
+      W.next(ahead);
+      W.next(ahead);
       if (!__all_sync(0xffffffffu, mbar_wait(bar_vec + X * 2 + y, (i >> 2) & 1, limit, p.status)) ||
           !__all_sync(0xffffffffu, mbar_wait(bar_sd_full + X, (i >> 1) & 1, limit, p.status))) {
         ok = false;
         break;
       }
       fence_after_sync();
-      const float* lse2 = vbuf;
-      const float* dd = vbuf + BQ;
+      const float4* lse4 = reinterpret_cast<const float4*>(vbuf);
+      const float4* dd4 = reinterpret_cast<const float4*>(vbuf + BQ);
       float pt[BQ];
 #pragma unroll
       for (int c = 0; c < BQ / 32; ++c) {
@@ -368,11 +393,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + tl + kTS + X * BQ + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = 32 * c + e;
-          const float ex = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -lse2[col]));
-          pt[col] = (col >= lo && col < hi) ? ex : 0.f;
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = lse4[(32 * c + e) / 4];
+          pt[32 * c + e + 0] = ex2(fmaf(__uint_as_float(v[e + 0]), p.scale_log2, -l4.x));
+          pt[32 * c + e + 1] = ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -l4.y));
+          pt[32 * c + e + 2] = ex2(fmaf(__uint_as_float(v[e + 2]), p.scale_log2, -l4.z));
+          pt[32 * c + e + 3] = ex2(fmaf(__uint_as_float(v[e + 3]), p.scale_log2, -l4.w));
         }
+      }
+      if (!full) {
+#pragma unroll
+        for (int col = 0; col < BQ; ++col) pt[col] = (col >= lo && col < hi) ? pt[col] : 0.f;
       }
       {
         uint32_t pk[32];
@@ -390,10 +421,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + tl + kTdP + X * BQ + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 32; e += 4) {
           const int col = 32 * c + e;
-          dsk[col / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - dd[col]),
-                                   pt[col + 1] * (__uint_as_float(v[e + 1]) - dd[col + 1]));
+          const float4 d4 = dd4[col / 4];
+          dsk[col / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - d4.x),
+                                   pt[col + 1] * (__uint_as_float(v[e + 1]) - d4.y));
+          dsk[col / 2 + 1] = pack_bf16(pt[col + 2] * (__uint_as_float(v[e + 2]) - d4.z),
+                                       pt[col + 3] * (__uint_as_float(v[e + 3]) - d4.w));
         }
       }
       fence_before_sync();
@@ -454,8 +488,8 @@ constexpr int kStages = 2;
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
-constexpr int kRegsMath = 216;
-constexpr int kRegsOther = 64;
+constexpr int kRegsMath = 192;
+constexpr int kRegsOther = 112;
 static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
 
 constexpr int kQBox = BM * 128;             // 128 query rows x 128 B
@@ -584,25 +618,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma && lane == 0) {
       constexpr uint32_t idSD = idesc_bf16(BM, BN, 0, 0);  // S, dP
       constexpr uint32_t idQ = idesc_bf16(BM, D, 0, 1);    // dQ += dS K (A in TMEM)
-      const uint32_t qA = smem_u32(smem + kOffQ), doA = smem_u32(smem + kOffDO);
-      const uint32_t kB = smem_u32(smem + kOffK), vB = smem_u32(smem + kOffV);
+      const uint64_t qAd = kdesc0(smem_u32(smem + kOffQ)), doAd = kdesc0(smem_u32(smem + kOffDO));
+      const uint64_t kBd = kdesc0(smem_u32(smem + kOffK)), vBd = kdesc0(smem_u32(smem + kOffV));
+      const uint64_t kMNd = mndesc0(smem_u32(smem + kOffK), kKBox);
       int n = 0;
       for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + BN - 1) / BN);
       auto issue_sd = [&](int x, int st) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + tS(x), kdesc(qA + x * kQTile, k, kQBox), kdesc(kB + st * kKTile, k, kKBox),
-                 idSD, k > 0);
+          mma_ss(tmem + tS(x), desc_add(qAd, x * kQTile + koff(k, kQBox)),
+                 desc_add(kBd, st * kKTile + koff(k, kKBox)), idSD, k > 0);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + tdP(x), kdesc(doA + x * kQTile, k, kQBox), kdesc(vB + st * kKTile, k, kKBox),
-                 idSD, k > 0);
+          mma_ss(tmem + tdP(x), desc_add(doAd, x * kQTile + koff(k, kQBox)),
+                 desc_add(vBd, st * kKTile + koff(k, kKBox)), idSD, k > 0);
         mma_commit(bar_sd_full + x);
       };
       auto issue_dq = [&](int x, int st, bool first) {
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tmem + tdQ(x), tmem + tS(x) + k * 8, mndesc(kB + st * kKTile, k, kKBox), idQ,
+          mma_ts(tmem + tdQ(x), tmem + tS(x) + k * 8, desc_add(kMNd, st * kKTile + mnoff(k)), idQ,
                  (first && k == 0) ? 0u : 1u);
       };
       bool ok = mbar_wait(bar_q, 0, limit, p.status);

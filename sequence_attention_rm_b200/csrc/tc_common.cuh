@@ -225,6 +225,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// The descriptor of the same operand `byte_off` bytes further on.  Shared
+// addresses are below 256 KB, so the 14-bit start-address field (16-byte
+// units) never carries into the next field.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t byte_off) {
+  return desc + (uint64_t)(byte_off >> 4);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulate.
 // a_mn / b_mn: operand stored MN-major (1) instead of K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
