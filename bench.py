@@ -213,6 +213,33 @@ class Step:
             ev[4].record()
 
 
+# Algorithmic flops per launch of each attention kernel, per visible (query,
+# key) pair: the contractions the kernel performs for its outputs.
+FLOPS_PER_PAIR = {"tc_fwd_kernel": 4, "tc_bwd_dkdv_kernel": 8, "tc_bwd_dq_kernel": 6}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from the committed
+# ncu captures of the current kernels (profiles/); None until captured.
+TRAFFIC = {}
+
+
+def kernel_table(records, steps, step_ms, w):
+    agg = {}
+    for name, ms in records:
+        a = agg.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += ms
+    out = {}
+    for name, (n, tot) in agg.items():
+        ms = tot / n
+        e = {"launches_per_step": round(n / steps, 2), "ms": round(ms, 4),
+             "share": round(tot / steps / step_ms, 4)}
+        if name in FLOPS_PER_PAIR:
+            flops = FLOPS_PER_PAIR[name] * w.d * causal_pairs(w)
+            e["flops"] = flops
+            e["TFLOP/s"] = round(flops / (ms * 1e-3) / 1e12, 2)
+        out[name] = e
+    return out
+
+
 def flush_l2(buf):
     buf.zero_()
 
@@ -238,12 +265,15 @@ def bench_ours(args, world, rank, local):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
+    rm.profile_enable(True)  # per-launch CUDA events on the launching stream
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush_l2(flush)
             step.run(evs[i])
         torch.cuda.synchronize()
     barrier(world)
+    records = rm.profile_records()
+    rm.profile_enable(False)
     per = [time_events([(e[0], e[4]), (e[1], e[2]), (e[2], e[3]), (e[0], e[1]), (e[3], e[4])])
            for e in evs]
     step_ms = sum(p[0] for p in per)
@@ -253,6 +283,7 @@ def bench_ours(args, world, rank, local):
     step_ms_max = max_over_ranks(step_ms, world)
     total_flops = (flops_fwd(w) + flops_bwd(w)) * args.steps * world
     value = total_flops / (step_ms_max * 1e-3) / 1e12
+    kernels = kernel_table(records, args.steps, step_ms / args.steps, w)
 
     # end-to-end: pinned host inputs in, results back to pinned host buffers
     pin = lambda t: t.pin_memory()
@@ -303,19 +334,23 @@ def bench_ours(args, world, rank, local):
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     bwd_tflops = flops_bwd(w) / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = flops_fwd(w) / (fwd_ms * 1e-3) / 1e12
+    top = max(kernels, key=lambda k: kernels[k]["share"])
+    tk = kernels[top]
     line["roofline"] = {
-        "bound": "tensor", "kernel": "tc_bwd_kernel (rm_ring_attn_bwd: + delta preprocess, dQ finalize)",
-        "achieved": round(bwd_tflops, 2), "peak": sustained, "unit": "TFLOP/s",
-        "frac": round(bwd_tflops / sustained, 4), "peak_source": f"{peak_src} bf16_tflops_sustained",
-        "traffic": None,
-        "frac_of_burst": round(bwd_tflops / peaks["bf16_tflops"], 4),
+        "bound": "tensor", "kernel": top, "achieved": tk["TFLOP/s"], "peak": sustained,
+        "unit": "TFLOP/s", "frac": round(tk["TFLOP/s"] / sustained, 4),
+        "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": TRAFFIC.get(top),
+        "frac_of_burst": round(tk["TFLOP/s"] / peaks["bf16_tflops"], 4),
+        "flops_per_launch": tk["flops"], "ms_per_launch": tk["ms"],
     }
-    line["kernels_ms"] = {"permute_in_out": round(perm_ms, 4), "ring_fwd": round(fwd_ms, 4),
-                          "ring_bwd": round(bwd_ms, 4)}
+    line["kernels"] = kernels
+    line["calls_ms"] = {"permute_in_out": round(perm_ms, 4), "ring_fwd": round(fwd_ms, 4),
+                        "ring_bwd": round(bwd_ms, 4)}
     line["ring_fwd_tflops"] = round(fwd_tflops, 2)
+    line["ring_bwd_tflops"] = round(bwd_tflops, 2)
     line["e2e"] = {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h}
-    line["gpu_launches"] = step.launches_per_step * args.steps
+    line["gpu_launches"] = len(records)
     line["clocks"] = clk.summary()
     del step, q, k, v, do
     torch.cuda.empty_cache()
@@ -454,15 +489,15 @@ def bench_reference(args, world, rank):
     if rank != 0:
         return None
     for _ in range(args.warmup):
-        oracle_sample(args.cpu_sample_heads)
+        oracle_sample(args.ref_sample_heads)
     secs, flops = 0.0, 0.0
     for _ in range(args.steps):
-        s, f = oracle_sample(args.cpu_sample_heads)
+        s, f = oracle_sample(args.ref_sample_heads)
         secs += s
         flops += f
     value = flops / secs / 1e12
     sample = (f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions 12288-14335, "
-              f"virtual rank 0) of {args.cpu_sample_heads} of 16 query heads, N=16384 zigzag P=2, "
+              f"virtual rank 0) of {args.ref_sample_heads} of 16 query heads, N=16384 zigzag P=2, "
               f"per step")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
@@ -487,7 +522,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-heads", type=int, default=2)
+    ap.add_argument("--cpu-sample-heads", type=int, default=16,
+                    help="query heads in the oracle sample of cpu_baseline")
+    ap.add_argument("--ref-sample-heads", type=int, default=4,
+                    help="query heads in each --impl reference step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

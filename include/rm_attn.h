@@ -250,6 +250,19 @@ const char* rm_last_error(void);
  * RM_ERR_TIMEOUT in the device status word.  Faults and hangs nothing. */
 rm_status rm_debug_expire_wait(uint32_t spin_limit, void* stream);
 
+/* ---- launch timing ------------------------------------------------------ */
+
+/* Opt-in per-kernel timing.  rm_profile_enable(1) clears earlier records and
+ * starts bracketing every kernel launch of the library with two CUDA events
+ * recorded on the launching stream; rm_profile_enable(0) stops (and also
+ * clears).  rm_profile_count gives the number of launches recorded;
+ * rm_profile_get(i, &name, &ms) waits for launch i to finish and returns the
+ * kernel's name (static string) and its device time in milliseconds.  The
+ * library owns the events; records are process-wide. */
+rm_status rm_profile_enable(int on);
+int rm_profile_count(void);
+rm_status rm_profile_get(int i, const char** name, float* ms);
+
 #if defined(__GNUC__)
 #pragma GCC visibility pop
 #endif

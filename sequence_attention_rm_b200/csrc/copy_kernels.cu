@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(256) gather_runs_kernel(const char* __restrict
 // Row map of the token permutation: output row (b, r*L + j) <- input row
 // (b, pos(r, j)) (forward) or the reverse.
 struct PermuteMap {
+  static constexpr const char* kName = "layout_permute";
   LayoutMap lay;
   int64_t N;
   int64_t row_bytes;
@@ -66,6 +67,7 @@ struct PermuteMap {
 // Ntot = P * N_local and run = (H/P) * d elements:
 //   seq -> head: out[r][n] <- in[n][r];   head -> seq: out[n][r] <- in[r][n].
 struct RepackMap {
+  static constexpr const char* kName = "seq_head_repack";
   int64_t ntot;
   int P;
   int64_t run_bytes;
@@ -93,6 +95,7 @@ cudaError_t launch_gather(const void* src, void* dst, int64_t rows, int64_t run_
   const int64_t warps = rows < warps_cap ? rows : warps_cap;
   const int blocks = (int)((warps + (threads / 32) - 1) / (threads / 32));
   uintptr_t a = (uintptr_t)src | (uintptr_t)dst;
+  ProfScope ps(Map::kName, stream);
   if (run_bytes % 16 == 0 && a % 16 == 0) {
     gather_runs_kernel<uint4, 4, Map><<<blocks, threads, 0, stream>>>(
         (const char*)src, (char*)dst, rows, (int)(run_bytes / 16), map);

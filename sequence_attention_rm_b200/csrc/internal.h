@@ -10,6 +10,18 @@
 namespace rm {
 
 int num_sms();  // SM count of the current device (cached per device)
+
+// Opt-in launch timing (rm_profile_enable): brackets a launch with events.
+namespace prof {
+int begin(const char* name, cudaStream_t s);
+void end(int idx, cudaStream_t s);
+}  // namespace prof
+struct ProfScope {
+  int idx;
+  cudaStream_t s;
+  ProfScope(const char* name, cudaStream_t st) : idx(prof::begin(name, st)), s(st) {}
+  ~ProfScope() { prof::end(idx, s); }
+};
 void set_last_error(const char* msg);  // reason returned by rm_last_error()
 
 cudaError_t launch_layout_permute(int esize, int B, int64_t N, int H, int d, int layout, int P,

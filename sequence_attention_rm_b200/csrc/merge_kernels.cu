@@ -200,6 +200,7 @@ cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stre
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(a.d);
   int grid = grid_for_rows(rows, g.rows_per_warp);
+  ProfScope ps("lse_merge", stream);
   return out_bf16 ? merge_dispatch<__nv_bfloat16>(a, g, grid, stream)
                   : merge_dispatch<float>(a, g, grid, stream);
 }
@@ -211,6 +212,7 @@ cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, r
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(d);
   int grid = grid_for_rows(rows, g.rows_per_warp);
+  ProfScope ps("bwd_preprocess", stream);
   if (in_bf16)
     bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
         B, N, H, d, o, dout, delta, zero_fill, g.lanes, g.rows_per_warp);
@@ -226,6 +228,7 @@ cudaError_t launch_convert_f32(int out_bf16, int B, int64_t N, int H, int d, rm_
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(d);
   int grid = grid_for_rows(rows, g.rows_per_warp);
+  ProfScope ps("convert_f32", stream);
   if (out_bf16)
     convert_f32_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes,
                                                                 g.rows_per_warp);

@@ -323,6 +323,7 @@ cudaError_t launch_simt_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   if (L == 0 || a.B == 0 || a.Hq == 0) return cudaSuccess;
   dim3 grid((unsigned)ceil_div(L, kRows), (unsigned)a.Hq,
             (unsigned)(q_rank < 0 ? a.B * a.P : a.B));
+  ProfScope ps("simt_fwd", stream);
   if (a.d <= 32) simt_fwd_kernel<32><<<grid, kThreads, 0, stream>>>(a, q_rank, kv_rank);
   else if (a.d <= 64) simt_fwd_kernel<64><<<grid, kThreads, 0, stream>>>(a, q_rank, kv_rank);
   else simt_fwd_kernel<128><<<grid, kThreads, 0, stream>>>(a, q_rank, kv_rank);
@@ -335,6 +336,7 @@ cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   const unsigned z = (unsigned)(q_rank < 0 ? a.B * a.P : a.B);
   dim3 gq((unsigned)ceil_div(L, kRows), (unsigned)a.Hq, z);
   dim3 gk((unsigned)ceil_div(L, kRows), (unsigned)a.Hkv, z);
+  ProfScope ps("simt_bwd", stream);
   if (a.d <= 32) {
     simt_bwd_dq_kernel<32><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
     simt_bwd_dkdv_kernel<32><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);

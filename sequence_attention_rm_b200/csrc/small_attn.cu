@@ -97,6 +97,7 @@ cudaError_t launch_small_seq_fwd(const AttnArgs& a, int q_rank, int kv_rank, int
   if (pairs == 0) return cudaSuccess;
   const int64_t blocks = (pairs + kWarps - 1) / kWarps;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  ProfScope ps("small_seq_fwd", stream);
   if (bf16)
     small_seq_attn_kernel<__nv_bfloat16><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(a, q_rank, kv_rank);
   else

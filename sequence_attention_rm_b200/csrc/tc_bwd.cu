@@ -800,6 +800,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
     if (cudaFuncSetAttribute(kv::tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kv::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;
+    ProfScope ps("tc_bwd_dkdv_kernel", stream);
     kv::tc_bwd_dkdv_kernel<<<grid, kv::kThreads, kv::kSmem, stream>>>(mq, mk, mv, mdo, p);
     if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
   }
@@ -816,6 +817,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
     if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dq::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;
+    ProfScope ps("tc_bwd_dq_kernel", stream);
     dq::tc_bwd_dq_kernel<<<grid, dq::kThreads, dq::kSmem, stream>>>(mq, mk, mv, mdo, p);
     if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
   }

@@ -515,6 +515,7 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   if (cudaFuncSetAttribute(tc_fwd_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)
     return RM_ERR_CUDA;
+  ProfScope ps("tc_fwd_kernel", stream);
   tc_fwd_kernel<DP><<<grid, kThreads, C::kSmem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? RM_OK : RM_ERR_CUDA;
 }

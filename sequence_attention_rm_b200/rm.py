@@ -28,7 +28,8 @@ EXPORTED = (
     "rm_attn_block_fwd", "rm_attn_block_bwd", "rm_attn_bwd_preprocess", "rm_lse_merge",
     "rm_ring_workspace_size", "rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_layout_permute",
     "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
-    "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc",
+    "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
+    "rm_profile_get",
 )
 
 
@@ -70,6 +71,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_get_device_status": [vp],
         "rm_debug_expire_wait": [ctypes.c_uint32, vp],
         "rm_ring_attn_bwd_noalloc": [D, T, T, T, T, vp, T, T, T, T, vp],
+        "rm_profile_enable": [i],
+        "rm_profile_count": [],
+        "rm_profile_get": [i, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -270,6 +274,22 @@ def get_device_status(stream=None) -> int:
 
 def debug_expire_wait(spin_limit: int, stream=None) -> None:
     _check(_lib.rm_debug_expire_wait(spin_limit, _stream(stream)))
+
+
+def profile_enable(on: bool) -> None:
+    """Start (clearing earlier records) or stop per-launch event timing."""
+    _check(_lib.rm_profile_enable(int(on)))
+
+
+def profile_records():
+    """[(kernel name, device ms)] of the launches recorded since enabling."""
+    out = []
+    for i in range(_lib.rm_profile_count()):
+        name = ctypes.c_char_p()
+        ms = ctypes.c_float()
+        _check(_lib.rm_profile_get(i, ctypes.byref(name), ctypes.byref(ms)))
+        out.append((name.value.decode(), ms.value))
+    return out
 
 
 def raw():

@@ -120,3 +120,16 @@ def test_bounded_wait_reports_timeout_and_context_survives(rm):
     x = torch.arange(16, device="cuda", dtype=torch.float32).reshape(1, 4, 1, 4)
     y = rm.layout_permute(x, "striped", 2)      # the context still works
     assert torch.equal(rm.layout_permute(y, "striped", 2, inverse=True), x)
+
+
+def test_launch_profiler_records_each_launch(rm):
+    x = synthetic.tensor(31, (1, 256, 4, 64), torch.bfloat16).cuda()
+    rm.profile_enable(True)
+    y = rm.layout_permute(x, "zigzag", 2)
+    rm.seq_head_repack(y.view(2, 128, 4, 64), 2)
+    recs = rm.profile_records()
+    rm.profile_enable(False)
+    assert [n for n, _ in recs] == ["layout_permute", "seq_head_repack"]
+    assert all(ms > 0 for _, ms in recs)
+    rm.layout_permute(x, "zigzag", 2)
+    assert rm.profile_records() == []  # disabled: nothing recorded
