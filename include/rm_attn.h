@@ -239,7 +239,8 @@ rm_status rm_seq_head_repack(rm_dtype dtype, int P, int64_t N_local, int H,
 
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: RM_ERR_TIMEOUT if a bounded wait expired in any kernel
- * since the last call, RM_ERR_CUDA if the synchronisation failed, else RM_OK. */
+ * since the last call, RM_ERR_CUDA if the synchronisation failed or a kernel
+ * found its shared memory misaligned (it then skipped its work), else RM_OK. */
 rm_status rm_get_device_status(void* stream);
 
 const char* rm_status_string(rm_status s);

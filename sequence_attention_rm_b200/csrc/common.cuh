@@ -56,13 +56,16 @@ __host__ __device__ inline LayoutMap make_layout(int layout, int64_t N, int P) {
 }
 
 // ---- device status word (bounded-wait expiry) ------------------------------
-enum : uint32_t { kStatusTimeout = 1u };
+enum : uint32_t { kStatusTimeout = 1u, kStatusSmemAlign = 2u };
 
 // Host: address of the status word on the current device.
 unsigned int* status_word();
 
 __device__ __forceinline__ void report_timeout(unsigned int* status) {
   if (status) atomicOr(status, kStatusTimeout);
+}
+__device__ __forceinline__ void report_status(unsigned int* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
 }
 
 // ---- small math helpers -----------------------------------------------------

@@ -216,6 +216,8 @@ rm_status rm_get_device_status(void* stream) {
   RM_CUDA(cudaMemsetAsync(p, 0, sizeof(v), st), "status clear");
   RM_CUDA(cudaStreamSynchronize(st), "status sync");
   if (v & kStatusTimeout) return fail(RM_ERR_TIMEOUT, "a device-side bounded wait expired");
+  if (v & kStatusSmemAlign)
+    return fail(RM_ERR_CUDA, "a kernel found its dynamic shared memory not 1024-byte aligned");
   return RM_OK;
 }
 

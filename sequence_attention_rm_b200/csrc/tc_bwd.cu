@@ -106,7 +106,7 @@ namespace kv {
 
 constexpr int BK = 128;     // keys per CTA (TMEM lanes)
 constexpr int BQ = 64;      // queries per tile
-constexpr int kQStages = 3;
+constexpr int kQStages = 4;
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
@@ -126,10 +126,23 @@ constexpr int kOffDO = kOffQ + kQStages * kQTile;  // [kQStages]
 constexpr int kOffDS = kOffDO + kQStages * kQTile; // [2] (one per math warpgroup)
 constexpr int kOffVec = kOffDS + 2 * kDSBytes;     // [wg][2][lse2 | D][64] fp32
 constexpr int kOffBar = kOffVec + 2 * 2 * 2 * BQ * 4;
-constexpr int kSmem = kOffBar + 256 + 1024;
+constexpr int kSmem = kOffBar + 256;  // the base must be 1024-aligned (checked)
 static_assert(kSmem <= 232448, "shared memory");
 
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;  // S, dP: [2] x 64 columns
+
+// mbarrier slots (8 bytes each) in the 256-byte barrier area
+constexpr int kBarKV = 0;
+constexpr int kBarQFull = kBarKV + 1;
+constexpr int kBarQEmpty = kBarQFull + kQStages;
+constexpr int kBarSD = kBarQEmpty + kQStages;
+constexpr int kBarP = kBarSD + 2;
+constexpr int kBarDSFull = kBarP + 2;
+constexpr int kBarDSEmpty = kBarDSFull + 2;
+constexpr int kBarVec = kBarDSEmpty + 2;
+constexpr int kBarDone = kBarVec + 4;
+constexpr int kBarTmem = kBarDone + 1;
+static_assert((kBarTmem + 1) * 8 <= 256, "barrier area");
 
 // The CTA's walk: for every query head of the group, every rank in
 // reverse-ring order, the 64-query tiles that can see key i0.
@@ -190,19 +203,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // SW128 tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) report_status(p.status, kStatusSmemAlign);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* bar_kv = bars + 0;
-  uint64_t* bar_q_full = bars + 1;    // [3]
-  uint64_t* bar_q_empty = bars + 4;   // [3]
-  uint64_t* bar_sd_full = bars + 7;   // [2] S^T and dP^T of a tile in TMEM buffer x
-  uint64_t* bar_p_full = bars + 9;    // [2] P^T written (128 arrivals)
-  uint64_t* bar_ds_full = bars + 11;  // [2] dS^T in smem (128 arrivals)
-  uint64_t* bar_ds_empty = bars + 13; // [2] dK done reading dS^T
-  uint64_t* bar_vec = bars + 15;      // [wg][2] LSE / D staged (128 arrivals)
-  uint64_t* bar_done = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* bar_kv = bars + kBarKV;
+  uint64_t* bar_q_full = bars + kBarQFull;    // [kQStages]
+  uint64_t* bar_q_empty = bars + kBarQEmpty;  // [kQStages]
+  uint64_t* bar_sd_full = bars + kBarSD;      // [2] S^T and dP^T of a tile in TMEM buffer x
+  uint64_t* bar_p_full = bars + kBarP;        // [2] P^T written (128 arrivals)
+  uint64_t* bar_ds_full = bars + kBarDSFull;  // [2] dS^T in smem (128 arrivals)
+  uint64_t* bar_ds_empty = bars + kBarDSEmpty;  // [2] dK done reading dS^T
+  uint64_t* bar_vec = bars + kBarVec;         // [wg][2] LSE / D staged (128 arrivals)
+  uint64_t* bar_done = bars + kBarDone;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarTmem);
   float* vec = reinterpret_cast<float*>(smem + kOffVec);
 
   const int warp = threadIdx.x >> 5;
@@ -484,7 +501,7 @@ namespace dq {
 
 constexpr int BM = 128;     // query rows per tile (TMEM lanes)
 constexpr int BN = 64;      // keys per KV tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
@@ -501,8 +518,18 @@ constexpr int kOffDO = kOffQ + 2 * kQTile;  // [2]
 constexpr int kOffK = kOffDO + 2 * kQTile;  // [kStages]
 constexpr int kOffV = kOffK + kStages * kKTile;
 constexpr int kOffBar = kOffV + kStages * kKTile;
-constexpr int kSmem = kOffBar + 256 + 1024;
+constexpr int kSmem = kOffBar + 256 + 1024;  // + slack to align the base to 1024
 static_assert(kSmem <= 232448, "shared memory");
+
+// mbarrier slots (8 bytes each) in the 256-byte barrier area
+constexpr int kBarQ = 0;
+constexpr int kBarKVFull = kBarQ + 1;
+constexpr int kBarKVEmpty = kBarKVFull + kStages;
+constexpr int kBarSD = kBarKVEmpty + kStages;
+constexpr int kBarDS = kBarSD + 2;
+constexpr int kBarDone = kBarDS + 2;
+constexpr int kBarTmem = kBarDone + 1;
+static_assert((kBarTmem + 1) * 8 <= 256, "barrier area");
 
 // TMEM per query tile X: S [X*256, +64), dP [X*256 + 64, +64), dQ [X*256 + 128, +128)
 __device__ __forceinline__ uint32_t tS(int x) { return x * 256; }
@@ -520,13 +547,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* bar_kv_full = bars + 1;   // [2]
-  uint64_t* bar_kv_empty = bars + 3;  // [2]
-  uint64_t* bar_sd_full = bars + 5;   // [2] S and dP of query tile X in TMEM
-  uint64_t* bar_ds_full = bars + 7;   // [2] dS written (128 arrivals)
-  uint64_t* bar_done = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* bar_q = bars + kBarQ;
+  uint64_t* bar_kv_full = bars + kBarKVFull;    // [kStages]
+  uint64_t* bar_kv_empty = bars + kBarKVEmpty;  // [kStages]
+  uint64_t* bar_sd_full = bars + kBarSD;        // [2] S and dP of query tile X in TMEM
+  uint64_t* bar_ds_full = bars + kBarDS;        // [2] dS written (128 arrivals)
+  uint64_t* bar_done = bars + kBarDone;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarTmem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -556,9 +583,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < kStages; ++x) {
       mbar_init(bar_kv_full + x, 1);
       mbar_init(bar_kv_empty + x, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
       mbar_init(bar_sd_full + x, 1);
       mbar_init(bar_ds_full + x, 128);
     }
@@ -596,8 +625,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nt = (int)((cta_keys(s) + BN - 1) / BN);
         const int ks = p.ring ? s : 0;
         for (int t = 0; t < nt; ++t, ++j) {
-          const int st = j & 1;
-          if (j >= kStages && !mbar_wait(bar_kv_empty + st, ((j >> 1) - 1) & 1, limit, p.status)) {
+          const int st = j % kStages;
+          if (j >= kStages &&
+              !mbar_wait(bar_kv_empty + st, ((j / kStages) - 1) & 1, limit, p.status)) {
             ok = false;
             break;
           }
@@ -612,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_wait(bar_q, 0, limit, p.status);
       for (int st = 0; st < kStages && j > st; ++st) {
-        const int uses = (j - st + 1) / 2;
+        const int uses = (j - st + kStages - 1) / kStages;
         mbar_wait(bar_kv_full + st, (uses - 1) & 1, limit, p.status);
       }
     } else if (warp == kWarpMma && lane == 0) {
@@ -650,12 +680,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1, nx = (j + 1) & 1;
+        const int st = j % kStages, nx = (j + 1) % kStages;
         if (!mbar_wait(bar_ds_full + 0, j & 1, limit, p.status)) break;
         fence_after_sync();
         issue_dq(0, st, j == 0);
         if (j + 1 < n) {
-          if (!mbar_wait(bar_kv_full + nx, ((j + 1) >> 1) & 1, limit, p.status)) break;
+          if (!mbar_wait(bar_kv_full + nx, ((j + 1) / kStages) & 1, limit, p.status)) break;
           fence_after_sync();
           issue_sd(0, nx);
         }

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  static_assert(kStages == 2, "the barrier slots below assume a 2-stage K/V ring");
   uint64_t* bar_q = bars + 0;
   uint64_t* bar_k_full = bars + 1;    // [kStages]
   uint64_t* bar_v_full = bars + 3;    // [kStages]
