@@ -11,33 +11,47 @@ namespace rm {
 namespace {
 
 // Copies `rows` runs of `run_vecs` vectors.  Run i goes from src + so(i) to
-// dst + dof(i) (byte offsets from the map).  One warp owns one run at a time
-// (the map is evaluated once per run, not per vector); each lane keeps UNROLL
-// independent 16/4/2-byte loads in flight before storing them.
-template <typename VEC, int UNROLL, typename Map>
-__global__ void __launch_bounds__(256) gather_runs_kernel(const char* __restrict__ src,
+// dst + dof(i) (byte offsets from the map).  The work is cut into items of
+// one run's 32-vector chunk, one vector per lane; a warp takes K consecutive
+// items per pass and keeps all K loads in flight before the stores.  The map
+// (integer divisions) is evaluated once per item by lane u of the warp and
+// broadcast with shuffles, so its cost is shared by the 32 lanes.
+template <typename VEC, int K, typename Map>
+__global__ void __launch_bounds__(256, 4) gather_runs_kernel(const char* __restrict__ src,
                                                           char* __restrict__ dst, int64_t rows,
                                                           int run_vecs, Map map) {
+  static_assert(K <= 32, "one item per lane for the map evaluation");
   const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-       row += warps) {
-    int64_t so, dof;
-    map(row, so, dof);
-    const VEC* s = reinterpret_cast<const VEC*>(src + so);
-    VEC* d = reinterpret_cast<VEC*>(dst + dof);
-    for (int v0 = 0; v0 < run_vecs; v0 += 32 * UNROLL) {
-      VEC buf[UNROLL];
-#pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        int v = v0 + u * 32 + lane;
-        if (v < run_vecs) buf[u] = __ldcs(s + v);
+  const int chunks = (run_vecs + 31) >> 5;
+  const int64_t items = rows * chunks;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * K;
+       base < items; base += nwarps * K) {
+    // lane u < K evaluates item base + u
+    int64_t my_so = 0, my_dof = 0;
+    int my_v0 = 0;
+    {
+      const int64_t it = base + (lane < K ? lane : 0);
+      if (it < items) {
+        const int64_t row = chunks == 1 ? it : it / chunks;
+        my_v0 = (int)(it - row * chunks) * 32;
+        map(row, my_so, my_dof);
       }
+    }
+    VEC buf[K];
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        int v = v0 + u * 32 + lane;
-        if (v < run_vecs) __stcs(d + v, buf[u]);
-      }
+    for (int u = 0; u < K; ++u) {
+      const int64_t so = __shfl_sync(0xffffffffu, my_so, u);
+      const int v = __shfl_sync(0xffffffffu, my_v0, u) + lane;
+      if (base + u < items && v < run_vecs)
+        buf[u] = __ldcs(reinterpret_cast<const VEC*>(src + so) + v);
+    }
+#pragma unroll
+    for (int u = 0; u < K; ++u) {
+      const int64_t dof = __shfl_sync(0xffffffffu, my_dof, u);
+      const int v = __shfl_sync(0xffffffffu, my_v0, u) + lane;
+      if (base + u < items && v < run_vecs)
+        __stcs(reinterpret_cast<VEC*>(dst + dof) + v, buf[u]);
     }
   }
 }
@@ -91,21 +105,25 @@ cudaError_t launch_gather(const void* src, void* dst, int64_t rows, int64_t run_
                           cudaStream_t stream) {
   if (rows == 0 || run_bytes == 0) return cudaSuccess;
   const int threads = 256;
-  const int64_t warps_cap = (int64_t)num_sms() * 16 * (threads / 32);
-  const int64_t warps = rows < warps_cap ? rows : warps_cap;
+  constexpr int K = 8;
+  const uintptr_t a = (uintptr_t)src | (uintptr_t)dst;
+  const int vsz = (run_bytes % 16 == 0 && a % 16 == 0) ? 16 : (run_bytes % 4 == 0 && a % 4 == 0) ? 4 : 2;
+  const int64_t run_vecs = run_bytes / vsz;
+  const int64_t items = rows * ((run_vecs + 31) / 32);
+  const int64_t warps_cap = (int64_t)num_sms() * 4 * (threads / 32);  // 4 resident blocks per SM
+  const int64_t warps_need = (items + K - 1) / K;
+  const int64_t warps = warps_need < warps_cap ? warps_need : warps_cap;
   const int blocks = (int)((warps + (threads / 32) - 1) / (threads / 32));
-  uintptr_t a = (uintptr_t)src | (uintptr_t)dst;
   ProfScope ps(Map::kName, stream);
-  if (run_bytes % 16 == 0 && a % 16 == 0) {
-    gather_runs_kernel<uint4, 4, Map><<<blocks, threads, 0, stream>>>(
-        (const char*)src, (char*)dst, rows, (int)(run_bytes / 16), map);
-  } else if (run_bytes % 4 == 0 && a % 4 == 0) {
-    gather_runs_kernel<uint32_t, 8, Map><<<blocks, threads, 0, stream>>>(
-        (const char*)src, (char*)dst, rows, (int)(run_bytes / 4), map);
-  } else {
-    gather_runs_kernel<uint16_t, 8, Map><<<blocks, threads, 0, stream>>>(
-        (const char*)src, (char*)dst, rows, (int)(run_bytes / 2), map);
-  }
+  if (vsz == 16)
+    gather_runs_kernel<uint4, K, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)run_vecs, map);
+  else if (vsz == 4)
+    gather_runs_kernel<uint32_t, K, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)run_vecs, map);
+  else
+    gather_runs_kernel<uint16_t, K, Map><<<blocks, threads, 0, stream>>>(
+        (const char*)src, (char*)dst, rows, (int)run_vecs, map);
   return cudaGetLastError();
 }
 
