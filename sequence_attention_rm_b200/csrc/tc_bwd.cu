@@ -105,47 +105,52 @@ __device__ __forceinline__ void store_row(void* base, int accumulate, int c32,
 namespace kv {
 
 constexpr int BK = 128;     // keys per CTA (TMEM lanes)
-constexpr int BQ = 64;      // queries per tile
-constexpr int kQStages = 4;
+constexpr int BQ = 128;     // queries per tile (the N of S^T, dP^T)
+constexpr int kHalf = BQ / 2;  // query columns per math warpgroup
+constexpr int kQStages = 2;
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kRegsMath = 200;
-constexpr int kRegsOther = 96;
+constexpr int kRegsOther = 104;
 static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
 
 constexpr int kKBox = BK * 128;             // 128 key rows x 128 B (64 cols)
 constexpr int kKTile = 2 * kKBox;
-constexpr int kQBox = BQ * 128;             // 64 query rows x 128 B
+constexpr int kQBox = BQ * 128;             // 128 query rows x 128 B
 constexpr int kQTile = 2 * kQBox;
-constexpr int kDSBytes = BK * 128;          // dS^T bf16 [128 keys][64 queries], SW128
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKTile;
 constexpr int kOffQ = kOffV + kKTile;              // [kQStages]
 constexpr int kOffDO = kOffQ + kQStages * kQTile;  // [kQStages]
-constexpr int kOffDS = kOffDO + kQStages * kQTile; // [2] (one per math warpgroup)
-constexpr int kOffVec = kOffDS + 2 * kDSBytes;     // [wg][2][lse2 | D][64] fp32
-constexpr int kOffBar = kOffVec + 2 * 2 * 2 * BQ * 4;
+constexpr int kOffVec = kOffDO + kQStages * kQTile; // [wg][2][lse2 | D][64] fp32
+constexpr int kOffBar = kOffVec + 2 * 2 * 2 * kHalf * 4;
 constexpr int kSmem = kOffBar + 256;  // the base must be 1024-aligned (checked)
 static_assert(kSmem <= 232448, "shared memory");
 
-constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;  // S, dP: [2] x 64 columns
+// TMEM columns: dK, dV accumulators; S^T (P^T written over it as bf16) and
+// dP^T (dS^T written over it as bf16), single-buffered.
+constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;
 
 // mbarrier slots (8 bytes each) in the 256-byte barrier area
 constexpr int kBarKV = 0;
 constexpr int kBarQFull = kBarKV + 1;
 constexpr int kBarQEmpty = kBarQFull + kQStages;
-constexpr int kBarSD = kBarQEmpty + kQStages;
-constexpr int kBarP = kBarSD + 2;
-constexpr int kBarDSFull = kBarP + 2;
-constexpr int kBarDSEmpty = kBarDSFull + 2;
-constexpr int kBarVec = kBarDSEmpty + 2;
+constexpr int kBarS = kBarQEmpty + kQStages;
+constexpr int kBarDP = kBarS + 1;
+constexpr int kBarP = kBarDP + 1;
+constexpr int kBarDS = kBarP + 1;
+constexpr int kBarVec = kBarDS + 1;
 constexpr int kBarDone = kBarVec + 4;
 constexpr int kBarTmem = kBarDone + 1;
 static_assert((kBarTmem + 1) * 8 <= 256, "barrier area");
 
+// TMEM column of the bf16 A operand (P^T or dS^T) for K-step k (16 queries):
+// warpgroup k / 4 packed its 64 queries into the first 32 columns of its half.
+__device__ __forceinline__ uint32_t a_col(int k) { return kHalf * (k >> 2) + 8 * (k & 3); }
+
 // The CTA's walk: for every query head of the group, every rank in
-// reverse-ring order, the 64-query tiles that can see key i0.
+// reverse-ring order, the query tiles that can see key i0.
 struct Walk {
   LayoutMap lay;
   int s, g, group, nranks, qtiles, ring, q_rank, P, causal;
@@ -194,11 +199,17 @@ struct Walk {
 };
 
 // Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
-// take alternate query tiles (P^T, dS^T of all 64 columns), then write dK
-// (warps 0-3) and dV (warps 4-7); warp 8 TMA producer (K, V once; Q, dO into
-// a 3-stage ring); warp 9 MMA issuer.  S^T / dP^T are double-buffered in TMEM,
-// one buffer per math warpgroup, so the tensor core computes tile i+1 while
-// tile i's math runs.
+// split every 128-query tile by columns (queries 0-63 / 64-127) over all 128
+// key lanes, then write dK (warps 0-3) and dV (warps 4-7); warp 8 TMA producer
+// (K, V once; Q, dO into a 2-stage ring); warp 9 MMA issuer.  All four
+// contractions are M=128, N=128: S^T, dP^T from shared memory; dV and dK take
+// P^T and dS^T from TMEM, so only Q and dO are read from shared memory for
+// them.  The tensor pipe runs, per tile i,
+//   dV(i) [needs P^T(i)], S^T(i+1), dK(i) [needs dS^T(i)], dP^T(i+1)
+// so that while the warpgroups turn S^T(i+1) into P^T(i+1) it computes dK(i)
+// and dP^T(i+1); the in-order pipe makes the single S / dP buffers safe
+// (S^T(i+1) is issued after dV(i) read P^T(i), dP^T(i+1) after dK(i) read
+// dS^T(i)).
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -213,10 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kv = bars + kBarKV;
   uint64_t* bar_q_full = bars + kBarQFull;    // [kQStages]
   uint64_t* bar_q_empty = bars + kBarQEmpty;  // [kQStages]
-  uint64_t* bar_sd_full = bars + kBarSD;      // [2] S^T and dP^T of a tile in TMEM buffer x
-  uint64_t* bar_p_full = bars + kBarP;        // [2] P^T written (128 arrivals)
-  uint64_t* bar_ds_full = bars + kBarDSFull;  // [2] dS^T in smem (128 arrivals)
-  uint64_t* bar_ds_empty = bars + kBarDSEmpty;  // [2] dK done reading dS^T
+  uint64_t* bar_s_full = bars + kBarS;        // S^T of the tile in TMEM
+  uint64_t* bar_dp_full = bars + kBarDP;      // dP^T of the tile in TMEM
+  uint64_t* bar_p_full = bars + kBarP;        // P^T written (256 arrivals)
+  uint64_t* bar_ds_full = bars + kBarDS;      // dS^T written (256 arrivals)
   uint64_t* bar_vec = bars + kBarVec;         // [wg][2] LSE / D staged (128 arrivals)
   uint64_t* bar_done = bars + kBarDone;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarTmem);
@@ -248,12 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_q_full + x, 1);
       mbar_init(bar_q_empty + x, 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(bar_sd_full + x, 1);
-      mbar_init(bar_p_full + x, 128);
-      mbar_init(bar_ds_full + x, 128);
-      mbar_init(bar_ds_empty + x, 1);
-    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_p_full, 256);
+    mbar_init(bar_ds_full, 256);
     for (int x = 0; x < 4; ++x) mbar_init(bar_vec + x, 128);
     mbar_init(bar_done, 1);
     fence_barrier_init();
@@ -306,108 +315,107 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kWarpMma && lane == 0) {
       constexpr uint32_t idST = idesc_bf16(BK, BQ, 0, 0);  // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16(BK, D, 0, 1);   // dV (A in TMEM), dK (A in smem)
+      constexpr uint32_t idKV = idesc_bf16(BK, D, 0, 1);   // dV, dK (A in TMEM, B MN-major)
       const uint64_t kAd = kdesc0(smem_u32(smem + kOffK)), vAd = kdesc0(smem_u32(smem + kOffV));
       const uint64_t qBd = kdesc0(smem_u32(smem + kOffQ)), doBd = kdesc0(smem_u32(smem + kOffDO));
       const uint64_t qMNd = mndesc0(smem_u32(smem + kOffQ), kQBox);
       const uint64_t doMNd = mndesc0(smem_u32(smem + kOffDO), kQBox);
-      const uint64_t dsAd = kdesc0(smem_u32(smem + kOffDS));
-      // S^T(i) and dP^T(i) into TMEM buffer i & 1
-      auto issue_sd = [&](int i) -> bool {
-        const int qst = i % kQStages, x = i & 1;
+      auto issue_s = [&](int i) -> bool {  // S^T(i) = K Q(i)^T
+        const int qst = i % kQStages;
         if (!mbar_wait(bar_q_full + qst, (i / kQStages) & 1, limit, p.status)) return false;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTS + x * BQ, desc_add(kAd, koff(k, kKBox)),
+          mma_ss(tmem + kTS, desc_add(kAd, koff(k, kKBox)),
                  desc_add(qBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + kTdP + x * BQ, desc_add(vAd, koff(k, kKBox)),
-                 desc_add(doBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
-        mma_commit(bar_sd_full + x);
+        mma_commit(bar_s_full);
         return true;
       };
-      bool ok = mbar_wait(bar_kv, 0, limit, p.status);
-      for (int i = 0; ok && i < 2 && i < n; ++i) ok = issue_sd(i);
+      auto issue_dp = [&](int i) {  // dP^T(i) = V dO(i)^T (Q / dO of tile i already landed)
+        const int qst = i % kQStages;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + kTdP, desc_add(vAd, koff(k, kKBox)),
+                 desc_add(doBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
+        mma_commit(bar_dp_full);
+      };
+      bool ok = n == 0 || (mbar_wait(bar_kv, 0, limit, p.status) && issue_s(0));
+      if (ok && n > 0) issue_dp(0);
       for (int i = 0; ok && i < n; ++i) {
-        const int x = i & 1, qst = i % kQStages;
-        if (!mbar_wait(bar_p_full + x, (i >> 1) & 1, limit, p.status)) break;
+        const int qst = i % kQStages;
+        if (!mbar_wait(bar_p_full, i & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dV += P^T dO
-          mma_ts(tmem + kTdV, tmem + kTS + x * BQ + k * 8,
-                 desc_add(doMNd, qst * kQTile + mnoff(k)), idKV, (i == 0 && k == 0) ? 0u : 1u);
-        if (!mbar_wait(bar_ds_full + x, (i >> 1) & 1, limit, p.status)) break;
+          mma_ts(tmem + kTdV, tmem + kTS + a_col(k), desc_add(doMNd, qst * kQTile + mnoff(k)),
+                 idKV, (i == 0 && k == 0) ? 0u : 1u);
+        if (i + 1 < n && !issue_s(i + 1)) break;
+        if (!mbar_wait(bar_ds_full, i & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dK += dS^T Q
-          mma_ss(tmem + kTdK, desc_add(dsAd, x * kDSBytes + koff(k, kDSBytes)),
-                 desc_add(qMNd, qst * kQTile + mnoff(k)), idKV, (i == 0 && k == 0) ? 0u : 1u);
+          mma_ts(tmem + kTdK, tmem + kTdP + a_col(k), desc_add(qMNd, qst * kQTile + mnoff(k)),
+                 idKV, (i == 0 && k == 0) ? 0u : 1u);
         mma_commit(bar_q_empty + qst);
-        mma_commit(bar_ds_empty + x);
-        if (i + 2 < n && !issue_sd(i + 2)) break;
+        if (i + 1 < n) issue_dp(i + 1);
       }
       mma_commit(bar_done);
       mbar_wait(bar_done, 0, limit, p.status);  // every MMA done before TMEM is freed
     }
   } else {
     regs_inc<kRegsMath>();
-    const int X = warp >> 2;                 // this warpgroup takes tiles i with i % 2 == X
+    const int X = warp >> 2;                 // this warpgroup's query columns: [64X, 64X + 64)
     const int lane_base = (warp & 3) * 32;
     const uint32_t tl = (uint32_t)lane_base << 16;
     const int krow = lane_base + lane;       // key row of the tile (TMEM lane)
     const int64_t key = i0 + krow;
     const bool key_live = key < L;
     const int64_t tk = key_live ? W.lay.pos(s, key) : 0;
+    // queries of rank r with position < tk cannot see this key
     const int tid = threadIdx.x & 127;
+    const uint32_t cS = kTS + kHalf * X, cdP = kTdP + kHalf * X;
     bool ok = true;
-    // LSE*log2(e) (tid < 64) or D (tid >= 64) of column tid & 63 of the tile at c
+    // LSE*log2(e) (tid < 64) or D (tid >= 64) of column 64X + (tid & 63) of the tile at c
     auto fetch = [&](const Walk::Cursor& c, int idx) -> float {
       if (idx >= n) return 0.f;
-      const int64_t j = (int64_t)c.t * BQ + (tid & 63);
+      const int64_t j = (int64_t)c.t * BQ + kHalf * X + (tid & 63);
       if (j >= L) return 0.f;
       const int64_t q0 = p.ring ? (int64_t)c.r * L : 0;
       const int64_t off = ((int64_t)b * p.Hq + W.head(c)) * p.lse_ld + q0 + j;
       return tid < 64 ? p.lse[off] * kLog2e : p.delta[off];
     };
-    // this warpgroup's tiles: cur walks X, X+2, ...; ahead runs two tiles in front
     Walk::Cursor cur = W.begin();
-    if (X == 1) W.next(cur);
     Walk::Cursor ahead = cur;
     W.next(ahead);
-    W.next(ahead);
-    float next = fetch(cur, X);
-    for (int i = X; i < n; i += 2) {
-      const int y = (i >> 1) & 1;  // staging buffer of this warpgroup
-      float* vbuf = vec + (X * 2 + y) * 2 * BQ;
+    float next = fetch(cur, 0);
+    for (int i = 0; i < n; ++i) {
+      const int y = i & 1;  // staging buffer
+      float* vbuf = vec + (X * 2 + y) * 2 * kHalf;
       vbuf[tid] = next;
       mbar_arrive(bar_vec + X * 2 + y);
-      next = fetch(ahead, i + 2);  // in flight during this tile
+      next = fetch(ahead, i + 1);  // in flight during this tile
       const int r = cur.r, t = cur.t;
-      const int64_t j0 = (int64_t)t * BQ;
-      // visible query columns [lo, hi) of this key in the tile
+      const int64_t j0 = (int64_t)t * BQ + kHalf * X;
+      // visible query columns [lo, hi) of this key in this warpgroup's half
       const int64_t hidden = !p.causal ? 0 : (key_live ? W.lay.visible_count(r, tk - 1) : L);
-      const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, BQ);
-      const int hi = key_live ? (int)LayoutMap::min64(L - j0, BQ) : 0;
-      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == BQ);
-      W.next(cur);
+      const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, kHalf);
+      const int hi = key_live ? (int)LayoutMap::clamp64(L - j0, 0, kHalf) : 0;
+      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kHalf);
       W.next(cur);
       W.next(ahead);
-      W.next(ahead);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_vec + X * 2 + y, (i >> 2) & 1, limit, p.status)) ||
-          !__all_sync(0xffffffffu, mbar_wait(bar_sd_full + X, (i >> 1) & 1, limit, p.status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_vec + X * 2 + y, (i >> 1) & 1, limit, p.status)) ||
+          !__all_sync(0xffffffffu, mbar_wait(bar_s_full, i & 1, limit, p.status))) {
         ok = false;
         break;
       }
       fence_after_sync();
       const float4* lse4 = reinterpret_cast<const float4*>(vbuf);
-      const float4* dd4 = reinterpret_cast<const float4*>(vbuf + BQ);
-      float pt[BQ];
+      const float4* dd4 = reinterpret_cast<const float4*>(vbuf + kHalf);
+      float pt[kHalf];
 #pragma unroll
-      for (int c = 0; c < BQ / 32; ++c) {
+      for (int c = 0; c < kHalf / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + tl + kTS + X * BQ + 32 * c, v);
+        tmem_ld32(tmem + tl + cS + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -420,49 +428,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!full) {
 #pragma unroll
-        for (int col = 0; col < BQ; ++col) pt[col] = (col >= lo && col < hi) ? pt[col] : 0.f;
+        for (int col = 0; col < kHalf; ++col) pt[col] = (col >= lo && col < hi) ? pt[col] : 0.f;
       }
       {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(pt[2 * e], pt[2 * e + 1]);
-        tmem_st32(tmem + tl + kTS + X * BQ, pk);
+        tmem_st32(tmem + tl + cS, pk);
         tmem_wait_st();
       }
       fence_before_sync();
-      mbar_arrive(bar_p_full + X);
-      uint32_t dsk[BQ / 2];
+      mbar_arrive(bar_p_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dp_full, i & 1, limit, p.status))) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      // dS^T over the 64 columns in two halves; each half's bf16 goes to the
+      // dP^T columns that have already been read
 #pragma unroll
-      for (int c = 0; c < BQ / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + tl + kTdP + X * BQ + 32 * c, v);
+      for (int c = 0; c < kHalf / 32; ++c) {
+        uint32_t v[32], dsk[16];
+        tmem_ld32(tmem + tl + cdP + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int col = 32 * c + e;
           const float4 d4 = dd4[col / 4];
-          dsk[col / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - d4.x),
-                                   pt[col + 1] * (__uint_as_float(v[e + 1]) - d4.y));
-          dsk[col / 2 + 1] = pack_bf16(pt[col + 2] * (__uint_as_float(v[e + 2]) - d4.z),
-                                       pt[col + 3] * (__uint_as_float(v[e + 3]) - d4.w));
+          dsk[e / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - d4.x),
+                                 pt[col + 1] * (__uint_as_float(v[e + 1]) - d4.y));
+          dsk[e / 2 + 1] = pack_bf16(pt[col + 2] * (__uint_as_float(v[e + 2]) - d4.z),
+                                     pt[col + 3] * (__uint_as_float(v[e + 3]) - d4.w));
         }
+        tmem_st16(tmem + tl + cdP + 16 * c, dsk);
       }
+      tmem_wait_st();
       fence_before_sync();
-      // dS^T row of this key into smem (SW128: 16-byte chunk c of row k lands
-      // at chunk c ^ (k & 7) of its 128-byte row)
-      if (i >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(bar_ds_empty + X, ((i >> 1) - 1) & 1, limit, p.status))) {
-        ok = false;
-        break;
-      }
-      {
-        uint4* row = reinterpret_cast<uint4*>(smem + kOffDS + X * kDSBytes + krow * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          row[c ^ (krow & 7)] = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_ds_full + X);
+      mbar_arrive(bar_ds_full);
     }
     // ---------------- epilogue: dK (warps 0-3), dV (warps 4-7); lane = key ----------------
     if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
