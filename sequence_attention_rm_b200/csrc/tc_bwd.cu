@@ -43,7 +43,6 @@ struct BwdParams {
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int ring, q_rank, kv_rank;
-  int head_pairs;    // dQ kernel: the two query tiles are heads (2y, 2y+1)
   const float* lse;  // natural-log LSE
   const float* delta;
   int64_t lse_ld;
@@ -57,10 +56,6 @@ struct BwdParams {
   unsigned int* status;
   long long wait_limit;
 };
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
 
 // K-major SW128 operand with rows of 128 B, 64-column boxes box_bytes apart:
 // base descriptor, and the byte offset of K-step k (16 elements).
@@ -107,7 +102,8 @@ namespace kv {
 constexpr int BK = 128;     // keys per CTA (TMEM lanes)
 constexpr int BQ = 128;     // queries per tile (the N of S^T, dP^T)
 constexpr int kHalf = BQ / 2;  // query columns per math warpgroup
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;   // Q is read by S^T(i) and dK(i): the longer-lived operand
+constexpr int kDOStages = 2;  // dO by dP^T(i) and dV(i)
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
@@ -122,8 +118,8 @@ constexpr int kQTile = 2 * kQBox;
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKTile;
 constexpr int kOffQ = kOffV + kKTile;              // [kQStages]
-constexpr int kOffDO = kOffQ + kQStages * kQTile;  // [kQStages]
-constexpr int kOffVec = kOffDO + kQStages * kQTile; // [wg][2][lse2 | D][64] fp32
+constexpr int kOffDO = kOffQ + kQStages * kQTile;  // [kDOStages]
+constexpr int kOffVec = kOffDO + kDOStages * kQTile; // [wg][2][lse2 | D][64] fp32
 constexpr int kOffBar = kOffVec + 2 * 2 * 2 * kHalf * 4;
 constexpr int kSmem = kOffBar + 256;  // the base must be 1024-aligned (checked)
 static_assert(kSmem <= 232448, "shared memory");
@@ -136,7 +132,9 @@ constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;
 constexpr int kBarKV = 0;
 constexpr int kBarQFull = kBarKV + 1;
 constexpr int kBarQEmpty = kBarQFull + kQStages;
-constexpr int kBarS = kBarQEmpty + kQStages;
+constexpr int kBarDOFull = kBarQEmpty + kQStages;
+constexpr int kBarDOEmpty = kBarDOFull + kDOStages;
+constexpr int kBarS = kBarDOEmpty + kDOStages;
 constexpr int kBarDP = kBarS + 1;
 constexpr int kBarP = kBarDP + 1;
 constexpr int kBarDS = kBarP + 1;
@@ -201,7 +199,8 @@ struct Walk {
 // Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
 // split every 128-query tile by columns (queries 0-63 / 64-127) over all 128
 // key lanes, then write dK (warps 0-3) and dV (warps 4-7); warp 8 TMA producer
-// (K, V once; Q, dO into a 2-stage ring); warp 9 MMA issuer.  All four
+// (K, V once; Q into a 3-stage ring, dO into a 2-stage ring); warp 9 MMA
+// issuer.  All four
 // contractions are M=128, N=128: S^T, dP^T from shared memory; dV and dK take
 // P^T and dS^T from TMEM, so only Q and dO are read from shared memory for
 // them.  The tensor pipe runs, per tile i,
@@ -224,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kv = bars + kBarKV;
   uint64_t* bar_q_full = bars + kBarQFull;    // [kQStages]
   uint64_t* bar_q_empty = bars + kBarQEmpty;  // [kQStages]
+  uint64_t* bar_do_full = bars + kBarDOFull;    // [kDOStages]
+  uint64_t* bar_do_empty = bars + kBarDOEmpty;  // [kDOStages]
   uint64_t* bar_s_full = bars + kBarS;        // S^T of the tile in TMEM
   uint64_t* bar_dp_full = bars + kBarDP;      // dP^T of the tile in TMEM
   uint64_t* bar_p_full = bars + kBarP;        // P^T written (256 arrivals)
@@ -259,6 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_q_full + x, 1);
       mbar_init(bar_q_empty + x, 1);
     }
+    for (int x = 0; x < kDOStages; ++x) {
+      mbar_init(bar_do_full + x, 1);
+      mbar_init(bar_do_empty + x, 1);
+    }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_full, 256);
@@ -290,28 +295,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_5d(smem + kOffK + x * kKBox, &tmK, bar_kv, x * 64, g, (int)i0, ks, b);
         tma_load_5d(smem + kOffV + x * kKBox, &tmV, bar_kv, x * 64, g, (int)i0, ks, b);
       }
-      int i = 0;
+      int nq = 0, ndo = 0;  // Q / dO tiles issued
       Walk::Cursor cur = W.begin();
-      for (; i < n; ++i, W.next(cur)) {
-        const int st = i % kQStages;
-        if (i >= kQStages &&
-            !mbar_wait(bar_q_empty + st, ((i / kQStages) - 1) & 1, limit, p.status))
-          break;
+      for (int i = 0; i < n; ++i, W.next(cur)) {
+        const int sq = i % kQStages, sd = i % kDOStages;
         const int h = W.head(cur), t = cur.t;
         const int qs = p.ring ? cur.r : 0;
-        mbar_arrive_expect_tx(bar_q_full + st, 2 * kQTile);
-        for (int x = 0; x < 2; ++x) {
-          tma_load_5d(smem + kOffQ + st * kQTile + x * kQBox, &tmQ, bar_q_full + st, x * 64, h,
+        if (i >= kQStages &&
+            !mbar_wait(bar_q_empty + sq, ((i / kQStages) - 1) & 1, limit, p.status))
+          break;
+        mbar_arrive_expect_tx(bar_q_full + sq, kQTile);
+        for (int x = 0; x < 2; ++x)
+          tma_load_5d(smem + kOffQ + sq * kQTile + x * kQBox, &tmQ, bar_q_full + sq, x * 64, h,
                       t * BQ, qs, b);
-          tma_load_5d(smem + kOffDO + st * kQTile + x * kQBox, &tmDO, bar_q_full + st, x * 64, h,
+        ++nq;
+        if (i >= kDOStages &&
+            !mbar_wait(bar_do_empty + sd, ((i / kDOStages) - 1) & 1, limit, p.status))
+          break;
+        mbar_arrive_expect_tx(bar_do_full + sd, kQTile);
+        for (int x = 0; x < 2; ++x)
+          tma_load_5d(smem + kOffDO + sd * kQTile + x * kQBox, &tmDO, bar_do_full + sd, x * 64, h,
                       t * BQ, qs, b);
-        }
+        ++ndo;
       }
       // drain: every load issued has landed before the CTA exits
       mbar_wait(bar_kv, 0, limit, p.status);
-      for (int st = 0; st < kQStages && st < i; ++st) {
-        const int uses = (i - st + kQStages - 1) / kQStages;
+      for (int st = 0; st < kQStages && st < nq; ++st) {
+        const int uses = (nq - st + kQStages - 1) / kQStages;
         mbar_wait(bar_q_full + st, (uses - 1) & 1, limit, p.status);
+      }
+      for (int st = 0; st < kDOStages && st < ndo; ++st) {
+        const int uses = (ndo - st + kDOStages - 1) / kDOStages;
+        mbar_wait(bar_do_full + st, (uses - 1) & 1, limit, p.status);
       }
     } else if (warp == kWarpMma && lane == 0) {
       constexpr uint32_t idST = idesc_bf16(BK, BQ, 0, 0);  // S^T, dP^T
@@ -331,24 +346,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_s_full);
         return true;
       };
-      auto issue_dp = [&](int i) {  // dP^T(i) = V dO(i)^T (Q / dO of tile i already landed)
-        const int qst = i % kQStages;
+      auto issue_dp = [&](int i) -> bool {  // dP^T(i) = V dO(i)^T
+        const int sd = i % kDOStages;
+        if (!mbar_wait(bar_do_full + sd, (i / kDOStages) & 1, limit, p.status)) return false;
+        fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + kTdP, desc_add(vAd, koff(k, kKBox)),
-                 desc_add(doBd, qst * kQTile + koff(k, kQBox)), idST, k > 0);
+                 desc_add(doBd, sd * kQTile + koff(k, kQBox)), idST, k > 0);
         mma_commit(bar_dp_full);
+        return true;
       };
-      bool ok = n == 0 || (mbar_wait(bar_kv, 0, limit, p.status) && issue_s(0));
-      if (ok && n > 0) issue_dp(0);
+      bool ok = n == 0 || (mbar_wait(bar_kv, 0, limit, p.status) && issue_s(0) && issue_dp(0));
       for (int i = 0; ok && i < n; ++i) {
-        const int qst = i % kQStages;
+        const int qst = i % kQStages, sd = i % kDOStages;
         if (!mbar_wait(bar_p_full, i & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dV += P^T dO
-          mma_ts(tmem + kTdV, tmem + kTS + a_col(k), desc_add(doMNd, qst * kQTile + mnoff(k)),
+          mma_ts(tmem + kTdV, tmem + kTS + a_col(k), desc_add(doMNd, sd * kQTile + mnoff(k)),
                  idKV, (i == 0 && k == 0) ? 0u : 1u);
+        mma_commit(bar_do_empty + sd);
         if (i + 1 < n && !issue_s(i + 1)) break;
         if (!mbar_wait(bar_ds_full, i & 1, limit, p.status)) break;
         fence_after_sync();
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + kTdK, tmem + kTdP + a_col(k), desc_add(qMNd, qst * kQTile + mnoff(k)),
                  idKV, (i == 0 && k == 0) ? 0u : 1u);
         mma_commit(bar_q_empty + qst);
-        if (i + 1 < n) issue_dp(i + 1);
+        if (i + 1 < n && !issue_dp(i + 1)) break;
       }
       mma_commit(bar_done);
       mbar_wait(bar_done, 0, limit, p.status);  // every MMA done before TMEM is freed
@@ -501,59 +519,78 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 namespace dq {
 
-constexpr int BM = 128;     // query rows per tile (TMEM lanes)
-constexpr int BN = 64;      // keys per KV tile
-constexpr int kStages = 3;
+constexpr int BM = 128;     // query rows per CTA (TMEM lanes)
+constexpr int BN = 128;     // keys per KV tile (the N of S, dP)
+constexpr int kHalf = BN / 2;  // key columns per math warpgroup
+constexpr int kKStages = 3;    // K is read by S(j) and dQ(j): the longer-lived operand
+constexpr int kVStages = 2;    // V only by dP(j)
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
-constexpr int kRegsMath = 192;
-constexpr int kRegsOther = 112;
+constexpr int kRegsMath = 200;
+constexpr int kRegsOther = 104;
 static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
 
 constexpr int kQBox = BM * 128;             // 128 query rows x 128 B
 constexpr int kQTile = 2 * kQBox;           // d = 128
-constexpr int kKBox = BN * 128;             // 64 key rows x 128 B
+constexpr int kKBox = BN * 128;             // 128 key rows x 128 B
 constexpr int kKTile = 2 * kKBox;
-constexpr int kOffQ = 0;                    // [2] query tiles
-constexpr int kOffDO = kOffQ + 2 * kQTile;  // [2]
-constexpr int kOffK = kOffDO + 2 * kQTile;  // [kStages]
-constexpr int kOffV = kOffK + kStages * kKTile;
-constexpr int kOffBar = kOffV + kStages * kKTile;
-constexpr int kSmem = kOffBar + 256 + 1024;  // + slack to align the base to 1024
+constexpr int kOffQ = 0;
+constexpr int kOffDO = kOffQ + kQTile;
+constexpr int kOffK = kOffDO + kQTile;      // [kKStages]
+constexpr int kOffV = kOffK + kKStages * kKTile;  // [kVStages]
+constexpr int kOffBar = kOffV + kVStages * kKTile;
+constexpr int kSmem = kOffBar + 256;  // the base must be 1024-aligned (checked)
 static_assert(kSmem <= 232448, "shared memory");
+
+// TMEM columns: S double-buffered (dS written over it as bf16), dP, dQ.
+constexpr uint32_t kTS = 0, kTdP = 256, kTdQ = 384;
 
 // mbarrier slots (8 bytes each) in the 256-byte barrier area
 constexpr int kBarQ = 0;
-constexpr int kBarKVFull = kBarQ + 1;
-constexpr int kBarKVEmpty = kBarKVFull + kStages;
-constexpr int kBarSD = kBarKVEmpty + kStages;
-constexpr int kBarDS = kBarSD + 2;
-constexpr int kBarDone = kBarDS + 2;
+constexpr int kBarKFull = kBarQ + 1;
+constexpr int kBarKEmpty = kBarKFull + kKStages;
+constexpr int kBarVFull = kBarKEmpty + kKStages;
+constexpr int kBarVEmpty = kBarVFull + kVStages;
+constexpr int kBarS = kBarVEmpty + kVStages;  // [2]
+constexpr int kBarDP = kBarS + 2;
+constexpr int kBarDS = kBarDP + 1;
+constexpr int kBarDone = kBarDS + 1;
 constexpr int kBarTmem = kBarDone + 1;
 static_assert((kBarTmem + 1) * 8 <= 256, "barrier area");
 
-// TMEM per query tile X: S [X*256, +64), dP [X*256 + 64, +64), dQ [X*256 + 128, +128)
-__device__ __forceinline__ uint32_t tS(int x) { return x * 256; }
-__device__ __forceinline__ uint32_t tdP(int x) { return x * 256 + 64; }
-__device__ __forceinline__ uint32_t tdQ(int x) { return x * 256 + 128; }
+// TMEM column of the bf16 A operand dS for K-step k (16 keys): warpgroup k / 4
+// packed its 64 keys into the first 32 columns of its half.
+__device__ __forceinline__ uint32_t a_col(int k) { return kHalf * (k >> 2) + 8 * (k & 3); }
 
-// Warp roles (384 threads): warps 0-3 / 4-7 own query tiles A / B (one thread
-// per query row: dS = P o (dP - D) from S and dP, written over S as bf16;
-// then the dQ epilogue); warp 8 TMA producer (Q, dO once; K, V 64-key tiles
-// into a 2-stage ring); warp 9 MMA issuer.
+// Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
+// split every 128-key tile by columns (keys 0-63 / 64-127) over the 128 query
+// rows (one thread per row: dS = P o (dP - D), written over S as bf16), then
+// write dQ; warp 8 TMA producer (Q, dO once; K tiles into a 3-stage ring, V
+// tiles into a 2-stage ring);
+// warp 9 MMA issuer.  S is double-buffered in TMEM, dP single-buffered; the
+// tensor pipe runs, per tile j,
+//   dQ(j) [needs dS(j)], dP(j+1), S(j+2)
+// so the exponentials of tile j+1 overlap dQ(j) and dP(j+1).
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                      const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // SW128 tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) report_status(p.status, kStatusSmemAlign);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* bar_q = bars + kBarQ;
-  uint64_t* bar_kv_full = bars + kBarKVFull;    // [kStages]
-  uint64_t* bar_kv_empty = bars + kBarKVEmpty;  // [kStages]
-  uint64_t* bar_sd_full = bars + kBarSD;        // [2] S and dP of query tile X in TMEM
-  uint64_t* bar_ds_full = bars + kBarDS;        // [2] dS written (128 arrivals)
+  uint64_t* bar_k_full = bars + kBarKFull;    // [kKStages]
+  uint64_t* bar_k_empty = bars + kBarKEmpty;  // [kKStages]
+  uint64_t* bar_v_full = bars + kBarVFull;    // [kVStages]
+  uint64_t* bar_v_empty = bars + kBarVEmpty;  // [kVStages]
+  uint64_t* bar_s_full = bars + kBarS;          // [2] S of a tile in TMEM buffer
+  uint64_t* bar_dp_full = bars + kBarDP;        // dP of the tile in TMEM
+  uint64_t* bar_ds_full = bars + kBarDS;        // dS written (256 arrivals)
   uint64_t* bar_done = bars + kBarDone;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarTmem);
 
@@ -563,36 +600,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t L = p.L;
   const int r = p.ring ? (int)(blockIdx.z % p.P) : p.q_rank;
   const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
-  const int unit = gridDim.x - 1 - blockIdx.x;  // later rows see more keys: start them first
-  int hA, hB;
-  int64_t rowA, rowB;
-  if (p.head_pairs) {
-    hA = 2 * blockIdx.y;
-    hB = hA + 1;
-    rowA = rowB = (int64_t)unit * BM;
-  } else {
-    hA = hB = blockIdx.y;
-    rowA = (int64_t)unit * 2 * BM;
-    rowB = rowA + BM;
-  }
-  const int g = hA / (p.Hq / p.Hkv);
-  const int64_t last_row = LayoutMap::min64((p.head_pairs ? rowA : rowB) + BM - 1, L - 1);
+  const int64_t row0 = (int64_t)(gridDim.x - 1 - blockIdx.x) * BM;  // later rows see more keys: start them first
+  const int h = blockIdx.y;
+  const int g = h / (p.Hq / p.Hkv);
+  const int64_t last_row = LayoutMap::min64(row0 + BM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
   const int nsteps = p.ring ? p.P : 1;
   const long long limit = p.wait_limit;
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
   auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
+  int n = 0;  // key tiles of the whole walk
+  for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int x = 0; x < kStages; ++x) {
-      mbar_init(bar_kv_full + x, 1);
-      mbar_init(bar_kv_empty + x, 1);
+    for (int x = 0; x < kKStages; ++x) {
+      mbar_init(bar_k_full + x, 1);
+      mbar_init(bar_k_empty + x, 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(bar_sd_full + x, 1);
-      mbar_init(bar_ds_full + x, 128);
+    for (int x = 0; x < kVStages; ++x) {
+      mbar_init(bar_v_full + x, 1);
+      mbar_init(bar_v_empty + x, 1);
     }
+    mbar_init(bar_s_full + 0, 1);
+    mbar_init(bar_s_full + 1, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_ds_full, 256);
     mbar_init(bar_done, 1);
     fence_barrier_init();
   }
@@ -613,100 +646,103 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDO);
       const int qs = p.ring ? r : 0;
-      mbar_arrive_expect_tx(bar_q, 4 * kQTile);
+      mbar_arrive_expect_tx(bar_q, 2 * kQTile);
       for (int x = 0; x < 2; ++x) {
-        tma_load_5d(smem + kOffQ + x * kQBox, &tmQ, bar_q, x * 64, hA, (int)rowA, qs, b);
-        tma_load_5d(smem + kOffQ + kQTile + x * kQBox, &tmQ, bar_q, x * 64, hB, (int)rowB, qs, b);
-        tma_load_5d(smem + kOffDO + x * kQBox, &tmDO, bar_q, x * 64, hA, (int)rowA, qs, b);
-        tma_load_5d(smem + kOffDO + kQTile + x * kQBox, &tmDO, bar_q, x * 64, hB, (int)rowB, qs, b);
+        tma_load_5d(smem + kOffQ + x * kQBox, &tmQ, bar_q, x * 64, h, (int)row0, qs, b);
+        tma_load_5d(smem + kOffDO + x * kQBox, &tmDO, bar_q, x * 64, h, (int)row0, qs, b);
       }
-      int j = 0;
+      int nk = 0, nv = 0;  // K / V tiles issued
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int s = shard_of(step);
         const int nt = (int)((cta_keys(s) + BN - 1) / BN);
         const int ks = p.ring ? s : 0;
-        for (int t = 0; t < nt; ++t, ++j) {
-          const int st = j % kStages;
-          if (j >= kStages &&
-              !mbar_wait(bar_kv_empty + st, ((j / kStages) - 1) & 1, limit, p.status)) {
+        for (int t = 0; t < nt; ++t) {
+          const int sk = nk % kKStages, sv = nv % kVStages;
+          if (nk >= kKStages &&
+              !mbar_wait(bar_k_empty + sk, ((nk / kKStages) - 1) & 1, limit, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar_kv_full + st, 2 * kKTile);
-          for (int x = 0; x < 2; ++x) {
-            tma_load_5d(smem + kOffK + st * kKTile + x * kKBox, &tmK, bar_kv_full + st, x * 64, g,
+          mbar_arrive_expect_tx(bar_k_full + sk, kKTile);
+          for (int x = 0; x < 2; ++x)
+            tma_load_5d(smem + kOffK + sk * kKTile + x * kKBox, &tmK, bar_k_full + sk, x * 64, g,
                         t * BN, ks, b);
-            tma_load_5d(smem + kOffV + st * kKTile + x * kKBox, &tmV, bar_kv_full + st, x * 64, g,
-                        t * BN, ks, b);
+          ++nk;
+          if (nv >= kVStages &&
+              !mbar_wait(bar_v_empty + sv, ((nv / kVStages) - 1) & 1, limit, p.status)) {
+            ok = false;
+            break;
           }
+          mbar_arrive_expect_tx(bar_v_full + sv, kKTile);
+          for (int x = 0; x < 2; ++x)
+            tma_load_5d(smem + kOffV + sv * kKTile + x * kKBox, &tmV, bar_v_full + sv, x * 64, g,
+                        t * BN, ks, b);
+          ++nv;
         }
       }
+      // drain: every load issued has landed before the CTA exits
       mbar_wait(bar_q, 0, limit, p.status);
-      for (int st = 0; st < kStages && j > st; ++st) {
-        const int uses = (j - st + kStages - 1) / kStages;
-        mbar_wait(bar_kv_full + st, (uses - 1) & 1, limit, p.status);
+      for (int st = 0; st < kKStages && nk > st; ++st) {
+        const int uses = (nk - st + kKStages - 1) / kKStages;
+        mbar_wait(bar_k_full + st, (uses - 1) & 1, limit, p.status);
+      }
+      for (int st = 0; st < kVStages && nv > st; ++st) {
+        const int uses = (nv - st + kVStages - 1) / kVStages;
+        mbar_wait(bar_v_full + st, (uses - 1) & 1, limit, p.status);
       }
     } else if (warp == kWarpMma && lane == 0) {
       constexpr uint32_t idSD = idesc_bf16(BM, BN, 0, 0);  // S, dP
-      constexpr uint32_t idQ = idesc_bf16(BM, D, 0, 1);    // dQ += dS K (A in TMEM)
+      constexpr uint32_t idQ = idesc_bf16(BM, D, 0, 1);    // dQ += dS K (A in TMEM, B MN-major)
       const uint64_t qAd = kdesc0(smem_u32(smem + kOffQ)), doAd = kdesc0(smem_u32(smem + kOffDO));
       const uint64_t kBd = kdesc0(smem_u32(smem + kOffK)), vBd = kdesc0(smem_u32(smem + kOffV));
       const uint64_t kMNd = mndesc0(smem_u32(smem + kOffK), kKBox);
-      int n = 0;
-      for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + BN - 1) / BN);
-      auto issue_sd = [&](int x, int st) {
+      auto issue_s = [&](int j) -> bool {  // S(j) = Q K(j)^T into buffer j & 1
+        const int sk = j % kKStages;
+        if (!mbar_wait(bar_k_full + sk, (j / kKStages) & 1, limit, p.status)) return false;
+        fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + tS(x), desc_add(qAd, x * kQTile + koff(k, kQBox)),
-                 desc_add(kBd, st * kKTile + koff(k, kKBox)), idSD, k > 0);
+          mma_ss(tmem + kTS + (j & 1) * BN, desc_add(qAd, koff(k, kQBox)),
+                 desc_add(kBd, sk * kKTile + koff(k, kKBox)), idSD, k > 0);
+        mma_commit(bar_s_full + (j & 1));
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V(j)^T
+        const int sv = j % kVStages;
+        if (!mbar_wait(bar_v_full + sv, (j / kVStages) & 1, limit, p.status)) return false;
+        fence_after_sync();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem + tdP(x), desc_add(doAd, x * kQTile + koff(k, kQBox)),
-                 desc_add(vBd, st * kKTile + koff(k, kKBox)), idSD, k > 0);
-        mma_commit(bar_sd_full + x);
+          mma_ss(tmem + kTdP, desc_add(doAd, koff(k, kQBox)),
+                 desc_add(vBd, sv * kKTile + koff(k, kKBox)), idSD, k > 0);
+        mma_commit(bar_dp_full);
+        mma_commit(bar_v_empty + sv);
+        return true;
       };
-      auto issue_dq = [&](int x, int st, bool first) {
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tmem + tdQ(x), tmem + tS(x) + k * 8, desc_add(kMNd, st * kKTile + mnoff(k)), idQ,
-                 (first && k == 0) ? 0u : 1u);
-      };
-      bool ok = mbar_wait(bar_q, 0, limit, p.status);
-      if (ok && n > 0) {
-        ok = mbar_wait(bar_kv_full + 0, 0, limit, p.status);
-        if (ok) {
-          fence_after_sync();
-          issue_sd(0, 0);
-          issue_sd(1, 0);
-        }
-      }
+      bool ok = n == 0 || (mbar_wait(bar_q, 0, limit, p.status) && issue_s(0) && issue_dp(0));
+      if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kStages, nx = (j + 1) % kStages;
-        if (!mbar_wait(bar_ds_full + 0, j & 1, limit, p.status)) break;
+        const int sk = j % kKStages;
+        if (!mbar_wait(bar_ds_full, j & 1, limit, p.status)) break;
         fence_after_sync();
-        issue_dq(0, st, j == 0);
-        if (j + 1 < n) {
-          if (!mbar_wait(bar_kv_full + nx, ((j + 1) / kStages) & 1, limit, p.status)) break;
-          fence_after_sync();
-          issue_sd(0, nx);
-        }
-        if (!mbar_wait(bar_ds_full + 1, j & 1, limit, p.status)) break;
-        fence_after_sync();
-        issue_dq(1, st, j == 0);
-        mma_commit(bar_kv_empty + st);
-        if (j + 1 < n) issue_sd(1, nx);
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)  // dQ += dS K
+          mma_ts(tmem + kTdQ, tmem + kTS + (j & 1) * BN + a_col(k),
+                 desc_add(kMNd, sk * kKTile + mnoff(k)), idQ, (j == 0 && k == 0) ? 0u : 1u);
+        mma_commit(bar_k_empty + sk);
+        if (j + 1 < n && !issue_dp(j + 1)) break;
+        if (j + 2 < n && !issue_s(j + 2)) break;
       }
       mma_commit(bar_done);
       mbar_wait(bar_done, 0, limit, p.status);
     }
   } else {
     regs_inc<kRegsMath>();
-    const int X = warp >> 2;
+    const int X = warp >> 2;                 // this warpgroup's key columns: [64X, 64X + 64)
     const int lane_base = (warp & 3) * 32;
     const uint32_t tl = (uint32_t)lane_base << 16;
-    const int64_t row = (X ? rowB : rowA) + lane_base + lane;
-    const int h = X ? hB : hA;
+    const int64_t row = row0 + lane_base + lane;
     const bool live = row < L;
     const int64_t tq = live ? lay.pos(r, row) : -1;
     const int64_t qrow = (p.ring ? (int64_t)r * L : 0) + row;
@@ -716,55 +752,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       lse2 = p.lse[off] * kLog2e;
       dd = p.delta[off];
     }
-    int j = 0, n = 0;
+    int j = 0;
     bool ok = true;
     for (int step = 0; step < nsteps && ok; ++step) {
       const int s = shard_of(step);
       const int nt = (int)((cta_keys(s) + BN - 1) / BN);
-      n += nt;
       const int64_t row_keys = !live ? 0 : (p.causal ? lay.visible_count(s, tq) : L);
       for (int t = 0; t < nt; ++t, ++j) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_sd_full + X, j & 1, limit, p.status))) {
+        const uint32_t cS = kTS + (j & 1) * BN + kHalf * X, cdP = kTdP + kHalf * X;
+        // visible keys of this warpgroup's half: [0, nvalid)
+        const int64_t nvalid = row_keys - (int64_t)t * BN - kHalf * X;
+        const bool full = __all_sync(0xffffffffu, nvalid >= kHalf);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, limit, p.status))) {
           ok = false;
           break;
         }
         fence_after_sync();
-        const int64_t nvalid = row_keys - (int64_t)t * BN;  // visible keys of this tile: [0, nvalid)
-        uint32_t sv[32], dv[32], ds[16];
-        // dS over the 64 keys in two halves; each half's bf16 goes to the
-        // S columns that half has already been read from
+        float pt[kHalf];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_ld32(tmem + tl + tS(X) + 32 * c, sv);
-          tmem_ld32(tmem + tl + tdP(X) + 32 * c, dv);
+        for (int c = 0; c < kHalf / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + tl + cS + 32 * c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int col = 32 * c + e;
-            float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lse2));
-            float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.scale_log2, -lse2));
-            p0 = col < nvalid ? p0 : 0.f;
-            p1 = col + 1 < nvalid ? p1 : 0.f;
-            ds[e / 2] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dd),
-                                  p1 * (__uint_as_float(dv[e + 1]) - dd));
-          }
-          tmem_st16(tmem + tl + tS(X) + 16 * c, ds);
+          for (int e = 0; e < 32; ++e)
+            pt[32 * c + e] = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -lse2));
+        }
+        if (!full) {
+#pragma unroll
+          for (int col = 0; col < kHalf; ++col) pt[col] = col < nvalid ? pt[col] : 0.f;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_dp_full, j & 1, limit, p.status))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        // dS over the 64 columns in two halves, written over S (already read)
+#pragma unroll
+        for (int c = 0; c < kHalf / 32; ++c) {
+          uint32_t v[32], ds[16];
+          tmem_ld32(tmem + tl + cdP + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            ds[e / 2] = pack_bf16(pt[32 * c + e] * (__uint_as_float(v[e]) - dd),
+                                  pt[32 * c + e + 1] * (__uint_as_float(v[e + 1]) - dd));
+          tmem_st16(tmem + tl + cS + 16 * c, ds);
         }
         tmem_wait_st();
         fence_before_sync();
-        mbar_arrive(bar_ds_full + X);
+        mbar_arrive(bar_ds_full);
       }
     }
-    // ---------------- epilogue: dQ = scale * acc ----------------
+    // ---------------- epilogue: dQ = scale * acc, columns [64X, 64X + 64) ----------------
     if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
       fence_after_sync();
       const int es = p.accumulate ? 4 : 2;
       char* base = reinterpret_cast<char*>(p.dq) +
                    (b * p.dq_sb + qrow * p.dq_sn + (int64_t)h * p.dq_sh) * es;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 2 * X; c < 2 * X + 2; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + tl + tdQ(X) + c * 32, v);
+        tmem_ld32(tmem + tl + kTdQ + c * 32, v);
         tmem_wait_ld();
         if (live) store_row(base, p.accumulate, c, v, p.scale, n == 0);
       }
@@ -802,7 +851,6 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.ring = ring ? 1 : 0;
   p.q_rank = q_rank;
   p.kv_rank = kv_rank;
-  p.head_pairs = ((a.Hq / a.Hkv) % 2 == 0) ? 1 : 0;
   p.lse = a.lse_in;
   p.delta = a.delta;
   p.lse_ld = a.lse_ld;
@@ -843,9 +891,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
         encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK)
       return RM_ERR_CUDA;
-    const int units = p.head_pairs ? ceil_div(L, dq::BM) : ceil_div(L, 2 * dq::BM);
-    dim3 grid((unsigned)units, (unsigned)(p.head_pairs ? a.Hq / 2 : a.Hq),
-              (unsigned)(ring ? a.B * a.P : a.B));
+    dim3 grid((unsigned)ceil_div(L, dq::BM), (unsigned)a.Hq, (unsigned)(ring ? a.B * a.P : a.B));
     if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dq::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;
