@@ -124,8 +124,9 @@ constexpr int kOffBar = kOffVec + 2 * 2 * 2 * kHalf * 4;
 constexpr int kSmem = kOffBar + 256;  // the base must be 1024-aligned (checked)
 static_assert(kSmem <= 232448, "shared memory");
 
-// TMEM columns: dK, dV accumulators; S^T (P^T written over it as bf16) and
-// dP^T (dS^T written over it as bf16), single-buffered.
+// TMEM columns: dK, dV accumulators; S^T, released as soon as the math
+// warpgroups have read it; dP^T, over which each warpgroup writes, in its own
+// 64-column half, P^T (bf16, first 32 columns) and dS^T (bf16, last 32).
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384;
 
 // mbarrier slots (8 bytes each) in the 256-byte barrier area
@@ -135,7 +136,8 @@ constexpr int kBarQEmpty = kBarQFull + kQStages;
 constexpr int kBarDOFull = kBarQEmpty + kQStages;
 constexpr int kBarDOEmpty = kBarDOFull + kDOStages;
 constexpr int kBarS = kBarDOEmpty + kDOStages;
-constexpr int kBarDP = kBarS + 1;
+constexpr int kBarSFree = kBarS + 1;
+constexpr int kBarDP = kBarSFree + 1;
 constexpr int kBarP = kBarDP + 1;
 constexpr int kBarDS = kBarP + 1;
 constexpr int kBarVec = kBarDS + 1;
@@ -143,9 +145,10 @@ constexpr int kBarDone = kBarVec + 4;
 constexpr int kBarTmem = kBarDone + 1;
 static_assert((kBarTmem + 1) * 8 <= 256, "barrier area");
 
-// TMEM column of the bf16 A operand (P^T or dS^T) for K-step k (16 queries):
-// warpgroup k / 4 packed its 64 queries into the first 32 columns of its half.
-__device__ __forceinline__ uint32_t a_col(int k) { return kHalf * (k >> 2) + 8 * (k & 3); }
+// TMEM column (from kTdP) of the bf16 A operand P^T / dS^T for K-step k (16
+// queries): warpgroup k / 4 packed its 64 queries into 32 columns of its half.
+__device__ __forceinline__ uint32_t p_col(int k) { return kHalf * (k >> 2) + 8 * (k & 3); }
+__device__ __forceinline__ uint32_t ds_col(int k) { return p_col(k) + 32; }
 
 // The CTA's walk: for every query head of the group, every rank in
 // reverse-ring order, the query tiles that can see key i0.
@@ -200,15 +203,13 @@ struct Walk {
 // split every 128-query tile by columns (queries 0-63 / 64-127) over all 128
 // key lanes, then write dK (warps 0-3) and dV (warps 4-7); warp 8 TMA producer
 // (K, V once; Q into a 3-stage ring, dO into a 2-stage ring); warp 9 MMA
-// issuer.  All four
-// contractions are M=128, N=128: S^T, dP^T from shared memory; dV and dK take
-// P^T and dS^T from TMEM, so only Q and dO are read from shared memory for
-// them.  The tensor pipe runs, per tile i,
-//   dV(i) [needs P^T(i)], S^T(i+1), dK(i) [needs dS^T(i)], dP^T(i+1)
-// so that while the warpgroups turn S^T(i+1) into P^T(i+1) it computes dK(i)
-// and dP^T(i+1); the in-order pipe makes the single S / dP buffers safe
-// (S^T(i+1) is issued after dV(i) read P^T(i), dP^T(i+1) after dK(i) read
-// dS^T(i)).
+// issuer.  All four contractions are M=128, N=128: S^T, dP^T from shared
+// memory; dV and dK take P^T and dS^T from TMEM, so only Q and dO are read
+// from shared memory for them.  The warpgroups copy S^T(i) into registers and
+// release its columns at once, so the tensor pipe runs, per tile i,
+//   dV(i) [needs P^T(i)], dK(i) [needs dS^T(i)], dP^T(i+1), S^T(i+2)
+// and the exponentials of tile i+1 overlap all four; the in-order pipe makes
+// the single dP^T buffer safe (dP^T(i+1) is issued after dK(i) read dS^T(i)).
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_do_full = bars + kBarDOFull;    // [kDOStages]
   uint64_t* bar_do_empty = bars + kBarDOEmpty;  // [kDOStages]
   uint64_t* bar_s_full = bars + kBarS;        // S^T of the tile in TMEM
+  uint64_t* bar_s_free = bars + kBarSFree;    // S^T read by the warpgroups (256 arrivals)
   uint64_t* bar_dp_full = bars + kBarDP;      // dP^T of the tile in TMEM
   uint64_t* bar_p_full = bars + kBarP;        // P^T written (256 arrivals)
   uint64_t* bar_ds_full = bars + kBarDS;      // dS^T written (256 arrivals)
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_do_empty + x, 1);
     }
     mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_free, 256);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_full, 256);
     mbar_init(bar_ds_full, 256);
@@ -358,24 +361,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       bool ok = n == 0 || (mbar_wait(bar_kv, 0, limit, p.status) && issue_s(0) && issue_dp(0));
+      if (ok && n > 1) ok = mbar_wait(bar_s_free, 0, limit, p.status) && issue_s(1);
       for (int i = 0; ok && i < n; ++i) {
         const int qst = i % kQStages, sd = i % kDOStages;
         if (!mbar_wait(bar_p_full, i & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dV += P^T dO
-          mma_ts(tmem + kTdV, tmem + kTS + a_col(k), desc_add(doMNd, sd * kQTile + mnoff(k)),
+          mma_ts(tmem + kTdV, tmem + kTdP + p_col(k), desc_add(doMNd, sd * kQTile + mnoff(k)),
                  idKV, (i == 0 && k == 0) ? 0u : 1u);
         mma_commit(bar_do_empty + sd);
-        if (i + 1 < n && !issue_s(i + 1)) break;
         if (!mbar_wait(bar_ds_full, i & 1, limit, p.status)) break;
         fence_after_sync();
 #pragma unroll
         for (int k = 0; k < BQ / 16; ++k)  // dK += dS^T Q
-          mma_ts(tmem + kTdK, tmem + kTdP + a_col(k), desc_add(qMNd, qst * kQTile + mnoff(k)),
+          mma_ts(tmem + kTdK, tmem + kTdP + ds_col(k), desc_add(qMNd, qst * kQTile + mnoff(k)),
                  idKV, (i == 0 && k == 0) ? 0u : 1u);
         mma_commit(bar_q_empty + qst);
         if (i + 1 < n && !issue_dp(i + 1)) break;
+        if (i + 2 < n &&
+            !(mbar_wait(bar_s_free, (i + 1) & 1, limit, p.status) && issue_s(i + 2)))
+          break;
       }
       mma_commit(bar_done);
       mbar_wait(bar_done, 0, limit, p.status);  // every MMA done before TMEM is freed
@@ -430,59 +436,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4* lse4 = reinterpret_cast<const float4*>(vbuf);
       const float4* dd4 = reinterpret_cast<const float4*>(vbuf + kHalf);
       float pt[kHalf];
-#pragma unroll
-      for (int c = 0; c < kHalf / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + tl + cS + 32 * c, v);
+      {
+        uint32_t v[kHalf];
+        tmem_ld32(tmem + tl + cS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + tl + cS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
+        fence_before_sync();
+        mbar_arrive(bar_s_free);  // S^T(i) is in registers: S^T(i+1) may overwrite it
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = lse4[(32 * c + e) / 4];
-          pt[32 * c + e + 0] = ex2(fmaf(__uint_as_float(v[e + 0]), p.scale_log2, -l4.x));
-          pt[32 * c + e + 1] = ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -l4.y));
-          pt[32 * c + e + 2] = ex2(fmaf(__uint_as_float(v[e + 2]), p.scale_log2, -l4.z));
-          pt[32 * c + e + 3] = ex2(fmaf(__uint_as_float(v[e + 3]), p.scale_log2, -l4.w));
+        for (int e = 0; e < kHalf; e += 4) {
+          const float4 l4 = lse4[e / 4];
+          pt[e + 0] = ex2(fmaf(__uint_as_float(v[e + 0]), p.scale_log2, -l4.x));
+          pt[e + 1] = ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -l4.y));
+          pt[e + 2] = ex2(fmaf(__uint_as_float(v[e + 2]), p.scale_log2, -l4.z));
+          pt[e + 3] = ex2(fmaf(__uint_as_float(v[e + 3]), p.scale_log2, -l4.w));
         }
       }
       if (!full) {
 #pragma unroll
         for (int col = 0; col < kHalf; ++col) pt[col] = (col >= lo && col < hi) ? pt[col] : 0.f;
       }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(pt[2 * e], pt[2 * e + 1]);
-        tmem_st32(tmem + tl + cS, pk);
-        tmem_wait_st();
-      }
-      fence_before_sync();
-      mbar_arrive(bar_p_full);
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dp_full, i & 1, limit, p.status))) {
         ok = false;
         break;
       }
       fence_after_sync();
-      // dS^T over the 64 columns in two halves; each half's bf16 goes to the
-      // dP^T columns that have already been read
-#pragma unroll
-      for (int c = 0; c < kHalf / 32; ++c) {
-        uint32_t v[32], dsk[16];
-        tmem_ld32(tmem + tl + cdP + 32 * c, v);
+      {
+        uint32_t v[kHalf];
+        tmem_ld32(tmem + tl + cdP, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + tl + cdP + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
+        // P^T over the first 32 columns of this half (its dP^T is in registers)
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int col = 32 * c + e;
-          const float4 d4 = dd4[col / 4];
-          dsk[e / 2] = pack_bf16(pt[col] * (__uint_as_float(v[e]) - d4.x),
-                                 pt[col + 1] * (__uint_as_float(v[e + 1]) - d4.y));
-          dsk[e / 2 + 1] = pack_bf16(pt[col + 2] * (__uint_as_float(v[e + 2]) - d4.z),
-                                     pt[col + 3] * (__uint_as_float(v[e + 3]) - d4.w));
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(pt[2 * e], pt[2 * e + 1]);
+        tmem_st32(tmem + tl + cdP, pk);
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(bar_p_full);
+        // dS^T = P^T o (dP^T - D) over the last 32 columns
+#pragma unroll
+        for (int e = 0; e < kHalf; e += 4) {
+          const float4 d4 = dd4[e / 4];
+          pk[e / 2] = pack_bf16(pt[e] * (__uint_as_float(v[e]) - d4.x),
+                                pt[e + 1] * (__uint_as_float(v[e + 1]) - d4.y));
+          pk[e / 2 + 1] = pack_bf16(pt[e + 2] * (__uint_as_float(v[e + 2]) - d4.z),
+                                    pt[e + 3] * (__uint_as_float(v[e + 3]) - d4.w));
         }
-        tmem_st16(tmem + tl + cdP + 16 * c, dsk);
+        tmem_st32(tmem + tl + cdP + 32, pk);
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(bar_ds_full);
       }
-      tmem_wait_st();
-      fence_before_sync();
-      mbar_arrive(bar_ds_full);
     }
     // ---------------- epilogue: dK (warps 0-3), dV (warps 4-7); lane = key ----------------
     if (__all_sync(0xffffffffu, ok && mbar_wait(bar_done, 0, limit, p.status))) {
