@@ -38,6 +38,30 @@ struct LayoutMap {
     return n1 + n2;
   }
 
+  // The (rank r, tile t) at place c when all P * T tiles of `tile` local rows
+  // (T = ceil(L / tile)) are ordered by the global position of their rows:
+  // ascending, or descending with `descending`.  Under the causal rule this
+  // is the order of decreasing (key tiles, ascending) or decreasing (query
+  // tiles, descending) work, which launches the longest CTAs first.  Tiles
+  // of different ranks never interleave in position except under the
+  // striped layout, where tile t of every rank precedes tile t + 1.
+  __host__ __device__ __forceinline__ void ordered_tile(int T, int tile, int c, bool descending,
+                                                        int& r, int& t) const {
+    if (descending) c = P * T - 1 - c;
+    if (layout == RM_LAYOUT_STRIPED) {
+      t = c / P;
+      r = c - t * P;
+    } else if (layout == RM_LAYOUT_ZIGZAG && C % tile == 0) {
+      const int tc = (int)(C / tile);  // tiles per chunk; chunk q of the sequence is on rank
+      const int q = c / tc;            // q (first half) or 2P - 1 - q (second half)
+      r = q < P ? q : 2 * P - 1 - q;
+      t = (q < P ? 0 : tc) + (c - q * tc);
+    } else {  // contiguous, or zigzag chunks that do not hold whole tiles
+      r = c / T;
+      t = c - r * T;
+    }
+  }
+
   __host__ __device__ __forceinline__ static int64_t min64(int64_t a, int64_t b) {
     return a < b ? a : b;
   }

@@ -124,15 +124,14 @@ FwdWs fwd_ws(const rm_attn_desc* d) {
   return w;
 }
 struct BwdWs {
-  size_t delta, dq, total;
+  size_t delta, total;
 };
 BwdWs bwd_ws(const rm_attn_desc* d) {
   BwdWs w;
   const size_t rows_q = (size_t)d->B * d->N * d->Hq;
   w.delta = 0;
-  w.dq = align_up(rows_q * 4);
   // both backward paths write dQ / dK / dV themselves: delta is all they keep
-  w.total = w.dq;
+  w.total = align_up(rows_q * 4);
   return w;
 }
 
@@ -142,14 +141,6 @@ rm_tensor dense_bnhd(void* p, int64_t N, int H, int d) {
   t.stride_b = N * H * d;
   t.stride_n = (int64_t)H * d;
   t.stride_h = d;
-  return t;
-}
-rm_tensor dense_bhnd(void* p, int64_t N, int H, int d) {
-  rm_tensor t;
-  t.ptr = p;
-  t.stride_b = (int64_t)H * N * d;
-  t.stride_n = d;
-  t.stride_h = N * d;
   return t;
 }
 
@@ -511,7 +502,6 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
     return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
   cudaStream_t st = (cudaStream_t)stream;
   float* delta = (float*)((char*)ws + w.delta);
-  float* dq_acc = (float*)((char*)ws + w.dq);
   AttnArgs a = attn_args(desc, desc->N);
   a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse_in = lse; a.delta = delta;
   a.accumulate = 0;

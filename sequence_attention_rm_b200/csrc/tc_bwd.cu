@@ -241,9 +241,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   Walk W;
   W.lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  W.s = p.ring ? (int)(blockIdx.z % p.P) : p.kv_rank;
-  const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
-  W.g = blockIdx.y;
+  // grid: (KV head, key tile in order of decreasing work, batch)
+  const int b = blockIdx.z;
+  int xt;
+  {
+    const int T = (int)((L + BK - 1) / BK);
+    const int c = blockIdx.y;
+    if (!p.ring) {
+      W.s = p.kv_rank;
+      xt = c;
+    } else if (p.causal) {
+      W.lay.ordered_tile(T, BK, c, false, W.s, xt);
+    } else {
+      W.s = c / T;
+      xt = c - W.s * T;
+    }
+  }
+  W.g = blockIdx.x;
   W.group = p.Hq / p.Hkv;
   W.nranks = p.ring ? p.P : 1;
   W.qtiles = (int)((L + BQ - 1) / BQ);
@@ -251,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   W.q_rank = p.q_rank;
   W.P = p.P;
   W.causal = p.causal;
-  const int64_t i0 = (int64_t)blockIdx.x * BK;  // first key (local index in shard s)
+  const int64_t i0 = (int64_t)xt * BK;  // first key (local index in shard s)
   W.tk_first = W.lay.pos(W.s, i0);
   const int s = W.s, g = W.g;
   const long long limit = p.wait_limit;
@@ -603,10 +617,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const LayoutMap lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  const int r = p.ring ? (int)(blockIdx.z % p.P) : p.q_rank;
-  const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
-  const int64_t row0 = (int64_t)(gridDim.x - 1 - blockIdx.x) * BM;  // later rows see more keys: start them first
-  const int h = blockIdx.y;
+  // grid: (query head, query tile in order of decreasing work, batch)
+  const int b = blockIdx.z;
+  int r, u;
+  {
+    const int T = (int)((L + BM - 1) / BM);
+    const int c = blockIdx.y;
+    if (!p.ring) {
+      r = p.q_rank;
+      u = p.causal ? T - 1 - c : c;  // later rows see more keys: start them first
+    } else if (p.causal) {
+      lay.ordered_tile(T, BM, c, true, r, u);
+    } else {
+      r = c / T;
+      u = c - r * T;
+    }
+  }
+  const int64_t row0 = (int64_t)u * BM;
+  const int h = blockIdx.x;
   const int g = h / (p.Hq / p.Hkv);
   const int64_t last_row = LayoutMap::min64(row0 + BM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
@@ -874,6 +902,8 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.accumulate = a.accumulate;
   p.status = a.status;
   p.wait_limit = tc_wait_limit();
+  // grid.y holds (shard, tile) pairs, grid.z the batch
+  if (ceil_div(L, 128) * shards > 65535 || a.B > 65535) return RM_ERR_UNSUPPORTED;
   {  // dK, dV
     CUtensorMap mq, mk, mv, mdo;
     if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK ||
@@ -881,7 +911,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
         encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK)
       return RM_ERR_CUDA;
-    dim3 grid((unsigned)ceil_div(L, kv::BK), (unsigned)a.Hkv, (unsigned)(ring ? a.B * a.P : a.B));
+    dim3 grid((unsigned)a.Hkv, (unsigned)(ceil_div(L, kv::BK) * shards), (unsigned)a.B);
     if (cudaFuncSetAttribute(kv::tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kv::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;
@@ -896,7 +926,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
         encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK)
       return RM_ERR_CUDA;
-    dim3 grid((unsigned)ceil_div(L, dq::BM), (unsigned)a.Hq, (unsigned)(ring ? a.B * a.P : a.B));
+    dim3 grid((unsigned)a.Hq, (unsigned)(ceil_div(L, dq::BM) * shards), (unsigned)a.B);
     if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dq::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;

@@ -54,6 +54,7 @@ CASES = [
     (torch.bfloat16, 1, 4, 2, 1040, 128, 8, "striped", True),
     (torch.bfloat16, 2, 4, 2, 768, 128, 4, "contiguous", True),
     (torch.bfloat16, 1, 4, 2, 2048, 128, 8, "zigzag", False),
+    (torch.bfloat16, 1, 4, 2, 2048, 128, 4, "zigzag", True),
     (torch.bfloat16, 1, 3, 3, 600, 64, 2, "zigzag", True),
     (torch.bfloat16, 1, 2, 1, 520, 64, 4, "striped", True),
     (torch.bfloat16, 1, 4, 4, 800, 32, 2, "contiguous", True),
