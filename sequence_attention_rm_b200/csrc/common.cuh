@@ -70,6 +70,27 @@ struct LayoutMap {
   }
 };
 
+// Grid order of the tensor-core attention kernels: blockIdx.x = c * G + i
+// walks the tile places c (in order of decreasing work) of a block of G heads
+// (or head units), blockIdx.y is the head block; G is chosen so that the
+// operands streamed by G heads' CTAs stay in L2 together.  Returns false for
+// the padding CTAs of a ragged last block.
+__device__ __forceinline__ bool grid_place(int G, int heads, int& c, int& head) {
+  c = (int)(blockIdx.x / G);
+  head = (int)blockIdx.y * G + (int)(blockIdx.x - c * G);
+  return head < heads;
+}
+// G for heads whose CTAs each stream `bytes_per_head` bytes: about as many
+// heads as fit in 48 MB (well inside the 126 MB L2), at least 1, evened out
+// so that the last block is nearly full.
+inline int head_block(int64_t bytes_per_head, int heads) {
+  int64_t g = ((int64_t)48 << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
+  if (g < 1) g = 1;
+  if (g > heads) g = heads;
+  const int64_t blocks = (heads + g - 1) / g;  // then spread the heads evenly over the blocks
+  return (int)((heads + blocks - 1) / blocks);
+}
+
 __host__ __device__ inline LayoutMap make_layout(int layout, int64_t N, int P) {
   LayoutMap m;
   m.layout = layout;

@@ -53,6 +53,7 @@ struct BwdParams {
   void* dv;
   int64_t dv_sb, dv_sn, dv_sh;
   int accumulate;
+  int head_block;    // heads per grid block (see grid_place)
   unsigned int* status;
   long long wait_limit;
 };
@@ -241,12 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   Walk W;
   W.lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  // grid: (KV head, key tile in order of decreasing work, batch)
+  // grid: (key tile in order of decreasing work x KV head, KV head block, batch)
   const int b = blockIdx.z;
+  int c, gh;
+  if (!grid_place(p.head_block, p.Hkv, c, gh)) return;
   int xt;
   {
     const int T = (int)((L + BK - 1) / BK);
-    const int c = blockIdx.y;
     if (!p.ring) {
       W.s = p.kv_rank;
       xt = c;
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       xt = c - W.s * T;
     }
   }
-  W.g = blockIdx.x;
+  W.g = gh;
   W.group = p.Hq / p.Hkv;
   W.nranks = p.ring ? p.P : 1;
   W.qtiles = (int)((L + BQ - 1) / BQ);
@@ -617,12 +619,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const LayoutMap lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  // grid: (query head, query tile in order of decreasing work, batch)
+  // grid: (query tile in order of decreasing work x query head, head block, batch)
   const int b = blockIdx.z;
+  int c, h;
+  if (!grid_place(p.head_block, p.Hq, c, h)) return;
   int r, u;
   {
     const int T = (int)((L + BM - 1) / BM);
-    const int c = blockIdx.y;
     if (!p.ring) {
       r = p.q_rank;
       u = p.causal ? T - 1 - c : c;  // later rows see more keys: start them first
@@ -634,7 +637,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   const int64_t row0 = (int64_t)u * BM;
-  const int h = blockIdx.x;
   const int g = h / (p.Hq / p.Hkv);
   const int64_t last_row = LayoutMap::min64(row0 + BM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
@@ -902,8 +904,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.accumulate = a.accumulate;
   p.status = a.status;
   p.wait_limit = tc_wait_limit();
-  // grid.y holds (shard, tile) pairs, grid.z the batch
-  if (ceil_div(L, 128) * shards > 65535 || a.B > 65535) return RM_ERR_UNSUPPORTED;
+  if (a.B > 65535) return RM_ERR_UNSUPPORTED;  // grid.z
   {  // dK, dV
     CUtensorMap mq, mk, mv, mdo;
     if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK ||
@@ -911,7 +912,10 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
         encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK)
       return RM_ERR_CUDA;
-    dim3 grid((unsigned)a.Hkv, (unsigned)(ceil_div(L, kv::BK) * shards), (unsigned)a.B);
+    // a key-tile CTA streams Q and dO of every query head of its group
+    p.head_block = head_block((int64_t)(a.Hq / a.Hkv) * a.N * D * 2 * 2, a.Hkv);
+    dim3 grid((unsigned)(ceil_div(L, kv::BK) * shards * p.head_block),
+              (unsigned)ceil_div(a.Hkv, p.head_block), (unsigned)a.B);
     if (cudaFuncSetAttribute(kv::tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kv::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;
@@ -926,7 +930,11 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
         encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK)
       return RM_ERR_CUDA;
-    dim3 grid((unsigned)a.Hq, (unsigned)(ceil_div(L, dq::BM) * shards), (unsigned)a.B);
+    // a query-tile CTA streams K and V of its KV head (shared by the group)
+    const int group = a.Hq / a.Hkv;
+    p.head_block = head_block((int64_t)a.N * D * 2 * 2 / group, a.Hq);
+    dim3 grid((unsigned)(ceil_div(L, dq::BM) * shards * p.head_block),
+              (unsigned)ceil_div(a.Hq, p.head_block), (unsigned)a.B);
     if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dq::kSmem) != cudaSuccess)
       return RM_ERR_CUDA;

@@ -76,6 +76,7 @@ struct FwdParams {
   float scale_log2;  // softmax scale * log2(e)
   int ring, q_rank, kv_rank;
   int head_pairs;
+  int head_block;  // head units per grid block (see grid_place)
   void* o;
   int64_t o_sb, o_sn, o_sh;
   int o_f32;
@@ -128,17 +129,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const LayoutMap lay = make_layout(p.layout, p.N, p.P);
   const int64_t L = p.L;
-  const int r = p.ring ? (int)(blockIdx.z % p.P) : p.q_rank;
-  const int b = p.ring ? (int)(blockIdx.z / p.P) : (int)blockIdx.z;
-  const int unit = gridDim.x - 1 - blockIdx.x;  // later rows see more keys: start them first
+  // grid: (row unit in order of decreasing work x head unit, head block, batch);
+  // a head unit is a head pair (heads 2x, 2x+1) or one head
+  const int b = blockIdx.z;
+  const int urows = p.head_pairs ? kBM : 2 * kBM;  // query rows of one unit
+  int c, hu;
+  if (!grid_place(p.head_block, p.head_pairs ? p.Hq / 2 : p.Hq, c, hu)) return;
+  int r, unit;
+  {
+    const int T = (int)((L + urows - 1) / urows);
+    if (!p.ring) {
+      r = p.q_rank;
+      unit = p.causal ? T - 1 - c : c;  // later rows see more keys: start them first
+    } else if (p.causal) {
+      lay.ordered_tile(T, urows, c, true, r, unit);
+    } else {
+      r = c / T;
+      unit = c - r * T;
+    }
+  }
   int hA, hB;
   int64_t rowA, rowB;
   if (p.head_pairs) {
-    hA = 2 * blockIdx.y;
+    hA = 2 * hu;
     hB = hA + 1;
     rowA = rowB = (int64_t)unit * kBM;
   } else {
-    hA = hB = blockIdx.y;
+    hA = hB = hu;
     rowA = (int64_t)unit * 2 * kBM;
     rowB = rowA + kBM;
   }
@@ -327,9 +344,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c >= nvalid) sc[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max over 8 independent chains (a single chain is 128 dependent steps)
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, sc[c]);
+        for (int e = 0; e < 8; ++e) mx8[e] = sc[e];
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sc[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_tile = mx * p.scale_log2;
         // Lazy rescale: the reference max only moves when it grows by more
         // than 8 (a factor 256), so O is rescaled rarely; p <= 256 otherwise.
@@ -353,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums: independent chains
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t pk[16];
@@ -360,11 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) {
             const float p0 = ex2(fmaf(sc[c * 32 + 2 * i], p.scale_log2, -m_use));
             const float p1 = ex2(fmaf(sc[c * 32 + 2 * i + 1], p.scale_log2, -m_use));
-            l += p0 + p1;
+            l4[i & 3] += p0 + p1;
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + c * 16, pk);
         }
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         tmem_wait_st();
         fence_before_sync();
         mbar_arrive(p_full);
@@ -511,8 +535,12 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   p.status = a.status;
   p.wait_limit = tc_wait_limit();
   const int units = p.head_pairs ? ceil_div(L, kBM) : ceil_div(L, 2 * kBM);
-  dim3 grid((unsigned)units, (unsigned)(p.head_pairs ? a.Hq / 2 : a.Hq),
-            (unsigned)(ring ? a.B * a.P : a.B));
+  if (a.B > 65535) return RM_ERR_UNSUPPORTED;  // grid.z
+  const int hunits = p.head_pairs ? a.Hq / 2 : a.Hq;
+  // a CTA streams K and V of its KV head, shared by the query heads of the group
+  p.head_block = head_block((int64_t)a.N * a.d * 2 * 2 * a.Hkv / hunits, hunits);
+  dim3 grid((unsigned)(units * shards * p.head_block), (unsigned)ceil_div(hunits, p.head_block),
+            (unsigned)a.B);
   if (cudaFuncSetAttribute(tc_fwd_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmem) != cudaSuccess)
     return RM_ERR_CUDA;
