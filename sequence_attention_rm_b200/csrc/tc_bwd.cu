@@ -810,8 +810,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tmem + tl + cS + 32 * c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            pt[32 * c + e] = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -lse2));
+          for (int e = 0; e < 32; e += 2) {  // exponents two at a time (packed fp32 FMA)
+            const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                         make_float2(p.scale_log2, p.scale_log2),
+                                         make_float2(-lse2, -lse2));
+            pt[32 * c + e] = ex2(x2.x);
+            pt[32 * c + e + 1] = ex2(x2.y);
+          }
         }
         if (!full) {
 #pragma unroll
@@ -829,9 +834,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tmem + tl + cdP + 32 * c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            ds[e / 2] = pack_bf16(pt[32 * c + e] * (__uint_as_float(v[e]) - dd),
-                                  pt[32 * c + e + 1] * (__uint_as_float(v[e + 1]) - dd));
+          for (int e = 0; e < 32; e += 2) {  // packed fp32 subtract and multiply
+            const float2 s2 = __fmul2_rn(make_float2(pt[32 * c + e], pt[32 * c + e + 1]),
+                                         __fadd2_rn(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                                    make_float2(-dd, -dd)));
+            ds[e / 2] = pack_bf16(s2.x, s2.y);
+          }
           tmem_st16(tmem + tl + cS + 16 * c, ds);
         }
         tmem_wait_st();

@@ -106,6 +106,12 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile_addr, int k) {
   return smem_desc(tile_addr + k * 16 * C::kRowBytes, C::kBoxBytes, 8 * C::kRowBytes, C::kSwz);
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int DP>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -344,14 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c >= nvalid) sc[c] = -INFINITY;
         }
-        // row max over 8 independent chains (a single chain is 128 dependent steps)
+        // row max: 8 independent chains of three-input max (a single two-input
+        // chain is 128 dependent steps)
         float mx8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = sc[e];
+        for (int e = 0; e < 8; ++e) {
+          float a = max3f(sc[e], sc[e + 8], sc[e + 16]);
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sc[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int j = 3; j + 1 < kBN / 8; j += 2) a = max3f(a, sc[e + 8 * j], sc[e + 8 * j + 8]);
+          mx8[e] = (kBN / 8) % 2 == 0 ? fmaxf(a, sc[e + kBN - 8]) : a;
+        }
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float m_tile = mx * p.scale_log2;
         // Lazy rescale: the reference max only moves when it grows by more
         // than 8 (a factor 256), so O is rescaled rarely; p <= 256 otherwise.
@@ -375,20 +385,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
-        float l4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums: independent chains
+        // scores to exponents two at a time (packed fp32 FMA), partial row
+        // sums two at a time in two independent chains (packed fp32 add)
+        const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 neg_m2 = make_float2(-m_use, -m_use);
+        float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(sc[c * 32 + 2 * i], p.scale_log2, -m_use));
-            const float p1 = ex2(fmaf(sc[c * 32 + 2 * i + 1], p.scale_log2, -m_use));
-            l4[i & 3] += p0 + p1;
-            pk[i] = pack_bf16(p0, p1);
+            const float2 x2 = __ffma2_rn(make_float2(sc[c * 32 + 2 * i], sc[c * 32 + 2 * i + 1]),
+                                         scale2, neg_m2);
+            const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
+            l2[i & 1] = __fadd2_rn(l2[i & 1], p2);
+            pk[i] = pack_bf16(p2.x, p2.y);
           }
           tmem_st16(tS + c * 16, pk);
         }
-        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
         tmem_wait_st();
         fence_before_sync();
         mbar_arrive(p_full);
