@@ -5,13 +5,12 @@
 //    KV head and keeps its dK and dV in TMEM while it walks, for every query
 //    head of the GQA group and every rank in reverse-ring order (s, s+1, ...;
 //    ringmaster, "Status": the backward runs the ring in the opposite
-//    direction), the 64-query tiles that can see its keys:
+//    direction), the 128-query tiles that can see its keys:
 //      S^T = K Q^T, dP^T = V dO^T             (TMEM, keys on lanes)
 //      P^T = exp(S^T * scale - LSE),  dS^T = P^T o (dP^T - D)
-//      dV += P^T dO   (A = P^T from TMEM)     dK += dS^T Q   (A = dS^T from smem)
-//  tc_bwd_dq_kernel (query-stationary).  One CTA owns two 128-row query tiles
-//    on one KV head (like the forward) and walks the 64-key tiles they see in
-//    ring order:
+//      dV += P^T dO,  dK += dS^T Q            (A = P^T, dS^T from TMEM)
+//  tc_bwd_dq_kernel (query-stationary).  One CTA owns one 128-row query tile
+//    of one head and walks the 128-key tiles it sees in ring order:
 //      S = Q K^T, dP = dO V^T                 (TMEM, queries on lanes)
 //      dS = exp(S * scale - LSE) o (dP - D)   (written over S as bf16)
 //      dQ += dS K     (A = dS from TMEM)
@@ -19,6 +18,9 @@
 // S and dP are recomputed by both kernels (7 MMAs per pair instead of 5); in
 // exchange dQ is never reduced through L2, whose fp32 reduce-add throughput
 // (about 1.2 TB/s) bound the fused design, and the result is deterministic.
+// Every contraction is M=128, N=128: a tcgen05.mma costs its issuing thread
+// about 50 cycles, so the N=64 form (32 cycles of work) would leave the
+// tensor pipe a third idle.
 #include <cudaTypedefs.h>
 #include <stdlib.h>
 
