@@ -421,7 +421,53 @@ def extras(rm, peaks, peak_src, dev, flush):
     out["striped_128k_fwd"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 2),
                                "frac": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
                                "peak_source": f"{peak_src} bf16_tflops (burst: one kernel timed alone)"}
+    # layout permute of the striped 128k Q (global -> rank-major), 2 x 512 MiB
+    o2 = torch.empty_like(q)
+    fn = lambda: rm.layout_permute(q, "striped", 8, out=o2)
+    fn()
+    ms = _time(fn, 5, flush)
+    nbytes = 2 * q.numel() * 2
+    out["permute"] = {"shape": "striped P=8 [1, 131072, 16, 128] bf16", "ms": round(ms, 4),
+                      "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
+                      "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    del q, k, v, o, lse, o2
+    out["tabular_row_fwd"] = tabular_row(rm, flush)
     return out
+
+
+# exp2 rate of the SFU: 16 results per clock per SM on sm_100 (the documented
+# throughput of ex2.approx; a probe on this machine measured 16.0), times the SMs
+# and the maximum SM clock.
+EX2_PER_CLK_SM = 16
+
+
+def tabular_row(rm, flush):
+    """Row-axis attention of the tabular workload (20 sequences of 150000 rows,
+    d = 24 padded to 32, non-causal fused ring over 8 contiguous shards on
+    strided views): TFLOP/s of its 4*d flops per pair against the tensor peak,
+    and exponentials per second against the SFU rate (the d = 24 path does
+    only 96 MMA flops per exponential)."""
+    w = synthetic.TABULAR
+    q, k, v = (t.cuda() for t in synthetic.tabular_inputs(w))
+    R, F, E, H = w.rows, w.features, w.embed, w.heads
+    view = lambda x: x.view(w.batch, R, F * H, E // H)
+    o = torch.empty(w.batch, R, F * H, E // H, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(w.batch, F * H, R, device="cuda")
+    fn = lambda: rm.ring_attn_fwd(view(q), view(k), view(v), P=w.P, layout="contiguous",
+                                  causal=False, out=o, lse=lse)
+    fn()
+    ms = _time(fn, 3, flush)
+    seqs = w.batch * F * H
+    pairs = seqs * R * R
+    flops = 4 * (E // H) * pairs
+    props = torch.cuda.get_device_properties(0)
+    ex2_peak = EX2_PER_CLK_SM * props.multi_processor_count * 1965e6
+    ex2_rate = pairs / (ms * 1e-3)
+    return {"shape": f"{seqs} sequences x {R} rows, d={E // H}", "ms": round(ms, 3),
+            "TFLOP/s": round(flops / ms / 1e9, 2),
+            "exp_per_s": round(ex2_rate / 1e12, 3), "exp_unit": "T exp2/s",
+            "exp_frac": round(ex2_rate / ex2_peak, 4),
+            "exp_peak_source": f"derived: {EX2_PER_CLK_SM}/clk/SM x {props.multi_processor_count} SMs x 1965 MHz"}
 
 
 # ---------------------------------------------------------------------------

@@ -8,6 +8,14 @@
 
 namespace rm {
 
+// TMA path of the two transforms (tma_copy.cu); false when the shape is
+// outside it (odd row sizes, misaligned pointers), and the gather kernel runs.
+bool tma_seq_head_repack(int esize, int P, int64_t n_local, int H, int d, int head_to_seq,
+                         const void* in, void* out, cudaStream_t stream, cudaError_t* err);
+bool tma_layout_permute(int esize, int B, int64_t N, int H, int d, int layout, int P,
+                        int inverse, const void* in, void* out, cudaStream_t stream,
+                        cudaError_t* err);
+
 namespace {
 
 // Copies `rows` runs of `run_vecs` vectors.  Run i goes from src + so(i) to
@@ -131,6 +139,8 @@ cudaError_t launch_gather(const void* src, void* dst, int64_t rows, int64_t run_
 
 cudaError_t launch_layout_permute(int esize, int B, int64_t N, int H, int d, int layout, int P,
                                   int inverse, const void* in, void* out, cudaStream_t stream) {
+  cudaError_t err;
+  if (tma_layout_permute(esize, B, N, H, d, layout, P, inverse, in, out, stream, &err)) return err;
   PermuteMap m;
   m.lay = make_layout(layout, N, P);
   m.N = N;
@@ -142,6 +152,8 @@ cudaError_t launch_layout_permute(int esize, int B, int64_t N, int H, int d, int
 cudaError_t launch_seq_head_repack(int esize, int P, int64_t n_local, int H, int d,
                                    int head_to_seq, const void* in, void* out,
                                    cudaStream_t stream) {
+  cudaError_t err;
+  if (tma_seq_head_repack(esize, P, n_local, H, d, head_to_seq, in, out, stream, &err)) return err;
   RepackMap m;
   m.ntot = (int64_t)P * n_local;
   m.P = P;

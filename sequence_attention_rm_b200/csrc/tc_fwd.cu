@@ -501,6 +501,30 @@ rm_status encode_operand_map(CUtensorMap* map, const rm_tensor& t, int B, int sh
   return rc == CUDA_SUCCESS ? RM_OK : RM_ERR_CUDA;
 }
 
+// A plain (no swizzle) map for the TMA copies of tma_copy.cu: elements of
+// `esize` bytes moved as unsigned integers (bit copy), zero fill out of range.
+rm_status encode_copy_map(CUtensorMap* map, const void* ptr, int esize, const int64_t (&dims)[5],
+                          const int64_t (&strides)[4], const int (&box)[5]) {
+  auto fn = encode_fn();
+  if (!fn) return RM_ERR_CUDA;
+  CUtensorMapDataType type;
+  if (esize == 1) type = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  else if (esize == 2) type = CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  else if (esize == 4) type = CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  else return RM_ERR_UNSUPPORTED;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bx[5], estr[5] = {1, 1, 1, 1, 1};
+  for (int i = 0; i < 5; ++i) {
+    gdim[i] = (cuuint64_t)dims[i];
+    bx[i] = (cuuint32_t)box[i];
+  }
+  for (int i = 0; i < 4; ++i) gstr[i] = (cuuint64_t)strides[i];
+  CUresult rc = fn(map, type, 5, const_cast<void*>(ptr), gdim, gstr, bx, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? RM_OK : RM_ERR_CUDA;
+}
+
 bool tc_supported_head_dim(int d) { return d == 24 || d == 32 || d == 64 || d == 128; }
 
 int tc_padded_head_dim(int d) { return d <= 32 ? 32 : d; }
