@@ -5,9 +5,12 @@
 Workload (one "step"): the Llama-like causal ring -- B=1, 16 query heads / 8
 KV heads, d=128, N=16384 bf16 tokens, P=2 virtual ranks in the zigzag
 (load-balanced) layout, forward + backward:
-  layout permute of Q, K, V, dO to rank-major order -> fused ring forward ->
-  ring backward (delta preprocess, tcgen05 backward, dQ finalize) -> inverse
-  permute of O, LSE, dQ, dK, dV.
+  fused ring forward -> ring backward (delta preprocess, key-stationary dK/dV
+  kernel, query-stationary dQ kernel), on operands in their global token
+  order: each virtual rank's tiles are fetched through the zigzag layout by
+  the kernels' TMA coordinates and O, LSE, dQ, dK, dV are written back in
+  global order, so the step has no separate permute pass (the permute kernel
+  itself is timed in the extras).
 Inputs are seeded synthetic tensors already resident in HBM; L2 (126 MB) is
 flushed between timed steps.  ``value`` is algorithmic TFLOP/s summed over all
 ranks: forward 4*d and backward 10*d flops per visible (query, key) pair,
@@ -15,9 +18,10 @@ causal pairs only.  With --gpus N every rank runs an independent replica of
 the workload (the path has no data exchange on one GPU), so scaling is weak.
 
 Extra measurements on the same line: the LSE merge (8 partials per rank of the
-striped 128k shapes) and the Ulysses repack (Q and fused K|V of the 256k zigzag
-shapes) in GB/s against HBM, and the causal striped 128k forward against the
-bf16 tensor peak.
+striped 128k shapes), the Ulysses repack (the 256k zigzag Q shape) and the
+striped layout permute (the 128k Q shape) in GB/s against HBM, the causal
+striped 128k forward against the bf16 tensor peak, and the tabular row-axis
+attention (d = 24) against the tensor peak and the exp unit.
 
 ``--impl reference`` times the CPU fp64 oracle instead, on a bounded sample of
 the same workload (2048 queries of one query head, forward and backward against
@@ -170,47 +174,35 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 class Step:
-    """Pre-allocated buffers and the hot-path step of one workload."""
+    """Pre-allocated buffers and the hot-path step of one workload: the fused
+    ring forward and the ring backward on global-order operands."""
 
     def __init__(self, rm, w, q, k, v, do):
         self.rm, self.w = rm, w
         self.q, self.k, self.v, self.do = q, k, v, do
         e = lambda t: torch.empty_like(t)
-        self.qr, self.kr, self.vr, self.dor = e(q), e(k), e(v), e(do)
-        self.o, self.dq, self.dk, self.dv = e(q), e(q), e(k), e(v)
         self.o_g, self.dq_g, self.dk_g, self.dv_g = e(q), e(q), e(k), e(v)
-        self.lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
-        self.lse_g = torch.empty_like(self.lse)
-        dsc = rm.desc(w.dtype, w.B, w.Hq, w.Hkv, w.d, w.N, w.P, w.layout, w.causal)
+        self.lse_g = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
+        dsc = rm.desc(w.dtype, w.B, w.Hq, w.Hkv, w.d, w.N, w.P, w.layout, w.causal,
+                      order="global")
         self.ws = torch.empty(max(rm.ring_workspace_size(dsc, True), 256), dtype=torch.uint8,
                               device=q.device)
-        self.launches_per_step = 4 + 1 + 3 + 5
+        self.launches_per_step = 1 + 3  # forward; delta, dK/dV, dQ
 
     def run(self, ev=None):
         rm, w = self.rm, self.w
         lay, P = w.layout, w.P
         if ev:
             ev[0].record()
-        for src, dst in ((self.q, self.qr), (self.k, self.kr), (self.v, self.vr), (self.do, self.dor)):
-            rm.layout_permute(src, lay, P, out=dst)
+        rm.ring_attn_fwd(self.q, self.k, self.v, P=P, layout=lay, causal=w.causal,
+                         order="global", out=self.o_g, lse=self.lse_g)
         if ev:
             ev[1].record()
-        rm.ring_attn_fwd(self.qr, self.kr, self.vr, P=P, layout=lay, causal=w.causal,
-                         out=self.o, lse=self.lse)
+        rm.ring_attn_bwd(self.q, self.k, self.v, self.o_g, self.lse_g, self.do, P=P, layout=lay,
+                         causal=w.causal, order="global", dq=self.dq_g, dk=self.dk_g,
+                         dv=self.dv_g, ws=self.ws)
         if ev:
             ev[2].record()
-        rm.ring_attn_bwd(self.qr, self.kr, self.vr, self.o, self.lse, self.dor, P=P, layout=lay,
-                         causal=w.causal, dq=self.dq, dk=self.dk, dv=self.dv, ws=self.ws)
-        if ev:
-            ev[3].record()
-        for src, dst in ((self.o, self.o_g), (self.dq, self.dq_g), (self.dk, self.dk_g),
-                         (self.dv, self.dv_g)):
-            rm.layout_permute(src, lay, P, inverse=True, out=dst)
-        # LSE [B, H, N]: the token axis is the last one; view it as [B*H, N, 1, 1]
-        rm.layout_permute(self.lse.view(w.B * w.Hq, w.N, 1, 1), lay, P, inverse=True,
-                          out=self.lse_g.view(w.B * w.Hq, w.N, 1, 1))
-        if ev:
-            ev[4].record()
 
 
 # Algorithmic flops per launch of each attention kernel, per visible (query,
@@ -218,8 +210,7 @@ class Step:
 FLOPS_PER_PAIR = {"tc_fwd_kernel": 4, "tc_bwd_dkdv_kernel": 8, "tc_bwd_dq_kernel": 6}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from the committed
 # ncu captures of the current kernels (profiles/); None until captured.
-TRAFFIC = {"tc_fwd_kernel": 173_960_000, "tc_bwd_dkdv_kernel": 254_040_000,
-           "tc_bwd_dq_kernel": 251_990_000}
+TRAFFIC = {"tc_fwd_kernel": None, "tc_bwd_dkdv_kernel": None, "tc_bwd_dq_kernel": None}
 
 
 def kernel_table(records, steps, step_ms, w):
@@ -263,7 +254,7 @@ def bench_ours(args, world, rank, local):
         step.run()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     rm.profile_enable(True)  # per-launch CUDA events on the launching stream
@@ -275,12 +266,10 @@ def bench_ours(args, world, rank, local):
     barrier(world)
     records = rm.profile_records()
     rm.profile_enable(False)
-    per = [time_events([(e[0], e[4]), (e[1], e[2]), (e[2], e[3]), (e[0], e[1]), (e[3], e[4])])
-           for e in evs]
+    per = [time_events([(e[0], e[2]), (e[0], e[1]), (e[1], e[2])]) for e in evs]
     step_ms = sum(p[0] for p in per)
     fwd_ms = statistics.mean(p[1] for p in per)
     bwd_ms = statistics.mean(p[2] for p in per)
-    perm_ms = statistics.mean(p[3] + p[4] for p in per)
     step_ms_max = max_over_ranks(step_ms, world)
     total_flops = (flops_fwd(w) + flops_bwd(w)) * args.steps * world
     value = total_flops / (step_ms_max * 1e-3) / 1e12
@@ -347,8 +336,7 @@ def bench_ours(args, world, rank, local):
         "flops_per_launch": tk["flops"], "ms_per_launch": tk["ms"],
     }
     line["kernels"] = kernels
-    line["calls_ms"] = {"permute_in_out": round(perm_ms, 4), "ring_fwd": round(fwd_ms, 4),
-                        "ring_bwd": round(bwd_ms, 4)}
+    line["calls_ms"] = {"ring_fwd": round(fwd_ms, 4), "ring_bwd": round(bwd_ms, 4)}
     line["ring_fwd_tflops"] = round(fwd_tflops, 2)
     line["ring_bwd_tflops"] = round(bwd_tflops, 2)
     line["e2e"] = {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

@@ -95,6 +95,14 @@ typedef struct {
   int64_t stride_h;
 } rm_tensor;
 
+/* Token order of the ring entry points' operands.  RANK_MAJOR: rank 0's L
+ * tokens, then rank 1's ... (what rm_layout_permute produces).  GLOBAL: the
+ * tokens' own order; the kernels fetch every tile of a virtual rank straight
+ * from it through the layout map (no permute pass).  GLOBAL needs bf16, the
+ * fused mode, and for zigzag chunks of a multiple of 128 tokens
+ * (N % (256 P) == 0); otherwise RM_ERR_UNSUPPORTED. */
+typedef enum { RM_ORDER_RANK_MAJOR = 0, RM_ORDER_GLOBAL = 1 } rm_order;
+
 /* One attention problem: B sequences of N tokens split over P virtual ranks
  * (L = N / P tokens each) laid out by `layout`.  d is the true head
  * dimension.  bf16 supports d in {24, 32, 64, 128} (24 is zero-padded to 32
@@ -111,6 +119,8 @@ typedef struct {
   int causal;
   float scale;        /* <= 0: 1/sqrt(d) */
   rm_ring_mode mode;  /* rm_ring_attn_fwd only */
+  rm_order order;     /* rm_ring_attn_fwd / _bwd only: token order of every
+                         [B, N, H, d] operand and of lse / delta */
 } rm_attn_desc;
 
 /* ---- block level: one Q shard against one KV shard ---------------------- */

@@ -70,6 +70,32 @@ struct LayoutMap {
   }
 };
 
+// Where the ring kernels find local row j of virtual rank r.  Rank-major
+// operands: memory row r * L + j, TMA coordinates (row j, shard r) of the
+// [B, P, L, H, d] view.  Global-order operands: memory row pos(r, j); TMA
+// coordinates in a view that matches the layout -- striped: [B, P, L, H, d]
+// with the row and shard strides swapped (row j of shard r is global row
+// j * P + r), so the coordinates stay (j, r); zigzag: [B, 2P chunks, C, H, d],
+// coordinates (j mod C, chunk r or 2P - 1 - r), which needs tiles that do not
+// straddle a chunk (C a multiple of the tile).
+struct RingRows {
+  LayoutMap lay;
+  int global;
+  __host__ __device__ __forceinline__ int64_t row(int r, int64_t j) const {
+    return global ? lay.pos(r, j) : (int64_t)r * lay.L + j;
+  }
+  __host__ __device__ __forceinline__ void tma(int r, int64_t j, int& crow, int& cshard) const {
+    if (global && lay.layout == RM_LAYOUT_ZIGZAG) {
+      const bool second = j >= lay.C;
+      crow = (int)(second ? j - lay.C : j);
+      cshard = second ? 2 * lay.P - 1 - r : r;
+    } else {
+      crow = (int)j;
+      cshard = r;
+    }
+  }
+};
+
 // Grid order of the tensor-core attention kernels: blockIdx.x = c * G + i
 // walks the tile places c (in order of decreasing work) of a block of G heads
 // (or head units), blockIdx.y is the head block; G is chosen so that the

@@ -73,6 +73,7 @@ struct AttnArgs {
   const float* delta;    // bwd
   rm_tensor dq, dk, dv;  // bwd fp32 accumulators
   int accumulate;        // bwd: 1 = dq/dk/dv +=, 0 = written (=)
+  int global_order;      // ring: operands (and lse / delta) in global token order
   unsigned int* status;
 };
 // Forward.  q_rank < 0: all ranks (ring, rank-major operands, fused merge);

@@ -63,6 +63,8 @@ rm_status check_desc(const rm_attn_desc* d) {
     return fail(RM_ERR_INVALID_ARG, "zigzag needs N %% 2P == 0");
   if (d->mode != RM_RING_FUSED && d->mode != RM_RING_STEPWISE)
     return fail(RM_ERR_INVALID_ARG, "bad ring mode");
+  if (d->order != RM_ORDER_RANK_MAJOR && d->order != RM_ORDER_GLOBAL)
+    return fail(RM_ERR_INVALID_ARG, "bad token order");
   if (!(d->scale == d->scale) || isinf(d->scale)) return fail(RM_ERR_INVALID_ARG, "bad scale");
   if (d->dtype == RM_BF16) {
     if (!tc_supported_head_dim(d->d))
@@ -71,6 +73,20 @@ rm_status check_desc(const rm_attn_desc* d) {
     if (d->d < 4 || d->d > 128 || d->d % 4)
       return fail(RM_ERR_UNSUPPORTED, "fp32 head dim %d: need d %% 4 == 0, d <= 128", d->d);
   }
+  return RM_OK;
+}
+
+// The ring entry points with global-order operands: the tensor-core kernels
+// fetch rank tiles through the layout (contiguous: global = rank-major).
+rm_status check_order(const rm_attn_desc* d, int backward) {
+  if (d->order != RM_ORDER_GLOBAL || d->layout == RM_LAYOUT_CONTIGUOUS || d->P == 1) return RM_OK;
+  if (d->dtype != RM_BF16)
+    return fail(RM_ERR_UNSUPPORTED, "global token order needs bf16 (the tensor-core path)");
+  if (!backward && d->mode != RM_RING_FUSED)
+    return fail(RM_ERR_UNSUPPORTED, "global token order needs the fused ring mode");
+  if (d->layout == RM_LAYOUT_ZIGZAG && (d->N / (2 * (int64_t)d->P)) % 128)
+    return fail(RM_ERR_UNSUPPORTED,
+                "global token order with zigzag needs chunks of a multiple of 128 tokens");
   return RM_OK;
 }
 
@@ -339,6 +355,8 @@ static AttnArgs attn_args(const rm_attn_desc* desc, int64_t lse_ld) {
   a.causal = desc->causal ? 1 : 0;
   a.scale = eff_scale(desc);
   a.lse_ld = lse_ld;
+  a.global_order = (desc->order == RM_ORDER_GLOBAL && desc->layout != RM_LAYOUT_CONTIGUOUS &&
+                    desc->P > 1) ? 1 : 0;
   a.status = status_word();
   return a;
 }
@@ -408,6 +426,7 @@ rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank, r
 
 rm_status rm_ring_workspace_size(const rm_attn_desc* desc, int backward, size_t* bytes) {
   RM_TRY(check_desc(desc));
+  RM_TRY(check_order(desc, backward));
   if (!bytes) return fail(RM_ERR_INVALID_ARG, "bytes is NULL");
   *bytes = backward ? bwd_ws(desc).total : fwd_ws(desc).total;
   return RM_OK;
@@ -416,6 +435,7 @@ rm_status rm_ring_workspace_size(const rm_attn_desc* desc, int backward, size_t*
 rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, rm_tensor v,
                            rm_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   RM_TRY(check_desc(desc));
+  RM_TRY(check_order(desc, 0));
   if (desc->B == 0 || desc->N == 0) return RM_OK;
   RM_TRY(check_qkv(desc, desc->N, q, k, v));
   const int es = esize_of(desc->dtype);
@@ -485,6 +505,7 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
                            rm_tensor o, const float* lse, rm_tensor dout, rm_tensor dq,
                            rm_tensor dk, rm_tensor dv, void* ws, size_t ws_bytes, void* stream) {
   RM_TRY(check_desc(desc));
+  RM_TRY(check_order(desc, 1));
   if (desc->B == 0 || desc->N == 0) return RM_OK;
   RM_TRY(check_qkv(desc, desc->N, q, k, v));
   const int es = esize_of(desc->dtype);

@@ -30,7 +30,8 @@
 namespace rm {
 
 rm_status encode_operand_map(CUtensorMap* map, const rm_tensor& t, int B, int shards, int64_t L,
-                             int H, int d, int box_cols, int box_rows);
+                             int H, int d, int box_cols, int box_rows, int view);
+int operand_view(const AttnArgs& a, bool ring);
 long long tc_wait_limit();
 
 namespace {
@@ -56,9 +57,36 @@ struct BwdParams {
   int64_t dv_sb, dv_sn, dv_sh;
   int accumulate;
   int head_block;    // heads per grid block (see grid_place)
+  int global_order;  // ring operands, outputs, LSE and D in global token order
   unsigned int* status;
   long long wait_limit;
 };
+
+// Row addressing of a backward call: ring calls go through RingRows (rank-
+// major or global order); a single shard has memory row = local row and TMA
+// coordinates (row, 0).
+struct BwdRows {
+  RingRows rows;
+  int ring;
+  __device__ __forceinline__ void tma(int rank, int64_t j, int& crow, int& cshard) const {
+    if (ring) {
+      rows.tma(rank, j, crow, cshard);
+    } else {
+      crow = (int)j;
+      cshard = 0;
+    }
+  }
+  __device__ __forceinline__ int64_t row(int rank, int64_t j) const {
+    return ring ? rows.row(rank, j) : j;
+  }
+};
+__device__ __forceinline__ BwdRows bwd_rows(const BwdParams& p) {
+  BwdRows r;
+  r.rows.lay = make_layout(p.layout, p.N, p.P);
+  r.rows.global = p.global_order;
+  r.ring = p.ring;
+  return r;
+}
 
 // K-major SW128 operand with rows of 128 B, 64-column boxes box_bytes apart:
 // base descriptor, and the byte offset of K-step k (16 elements).
@@ -273,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   W.tk_first = W.lay.pos(W.s, i0);
   const int s = W.s, g = W.g;
   const long long limit = p.wait_limit;
+  const BwdRows R = bwd_rows(p);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -310,25 +339,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDO);
-      const int ks = p.ring ? s : 0;
+      int kr, ks;
+      R.tma(s, i0, kr, ks);
       mbar_arrive_expect_tx(bar_kv, 2 * kKTile);
       for (int x = 0; x < 2; ++x) {
-        tma_load_5d(smem + kOffK + x * kKBox, &tmK, bar_kv, x * 64, g, (int)i0, ks, b);
-        tma_load_5d(smem + kOffV + x * kKBox, &tmV, bar_kv, x * 64, g, (int)i0, ks, b);
+        tma_load_5d(smem + kOffK + x * kKBox, &tmK, bar_kv, x * 64, g, kr, ks, b);
+        tma_load_5d(smem + kOffV + x * kKBox, &tmV, bar_kv, x * 64, g, kr, ks, b);
       }
       int nq = 0, ndo = 0;  // Q / dO tiles issued
       Walk::Cursor cur = W.begin();
       for (int i = 0; i < n; ++i, W.next(cur)) {
         const int sq = i % kQStages, sd = i % kDOStages;
         const int h = W.head(cur), t = cur.t;
-        const int qs = p.ring ? cur.r : 0;
+        int qr, qs;
+        R.tma(cur.r, (int64_t)t * BQ, qr, qs);
         if (i >= kQStages &&
             !mbar_wait(bar_q_empty + sq, ((i / kQStages) - 1) & 1, limit, p.status))
           break;
         mbar_arrive_expect_tx(bar_q_full + sq, kQTile);
         for (int x = 0; x < 2; ++x)
           tma_load_5d(smem + kOffQ + sq * kQTile + x * kQBox, &tmQ, bar_q_full + sq, x * 64, h,
-                      t * BQ, qs, b);
+                      qr, qs, b);
         ++nq;
         if (i >= kDOStages &&
             !mbar_wait(bar_do_empty + sd, ((i / kDOStages) - 1) & 1, limit, p.status))
@@ -336,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar_do_full + sd, kQTile);
         for (int x = 0; x < 2; ++x)
           tma_load_5d(smem + kOffDO + sd * kQTile + x * kQBox, &tmDO, bar_do_full + sd, x * 64, h,
-                      t * BQ, qs, b);
+                      qr, qs, b);
         ++ndo;
       }
       // drain: every load issued has landed before the CTA exits
@@ -422,8 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx >= n) return 0.f;
       const int64_t j = (int64_t)c.t * BQ + kHalf * X + (tid & 63);
       if (j >= L) return 0.f;
-      const int64_t q0 = p.ring ? (int64_t)c.r * L : 0;
-      const int64_t off = ((int64_t)b * p.Hq + W.head(c)) * p.lse_ld + q0 + j;
+      const int64_t off = ((int64_t)b * p.Hq + W.head(c)) * p.lse_ld + R.row(c.r, j);
       return tid < 64 ? p.lse[off] * kLog2e : p.delta[off];
     };
     Walk::Cursor cur = W.begin();
@@ -513,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tcol = X == 0 ? kTdK : kTdV;
       const float f = X == 0 ? p.scale : 1.0f;
       const int es = p.accumulate ? 4 : 2;
-      const int64_t row = (p.ring ? (int64_t)s * L : 0) + key;
+      const int64_t row = R.row(s, key);
       char* base = X == 0 ? reinterpret_cast<char*>(p.dk) +
                                 (b * p.dk_sb + row * p.dk_sn + (int64_t)g * p.dk_sh) * es
                           : reinterpret_cast<char*>(p.dv) +
@@ -644,6 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t t_last = lay.pos(r, last_row);
   const int nsteps = p.ring ? p.P : 1;
   const long long limit = p.wait_limit;
+  const BwdRows R = bwd_rows(p);
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
   auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
   int n = 0;  // key tiles of the whole walk
@@ -682,20 +713,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDO);
-      const int qs = p.ring ? r : 0;
+      int qr, qs;
+      R.tma(r, row0, qr, qs);
       mbar_arrive_expect_tx(bar_q, 2 * kQTile);
       for (int x = 0; x < 2; ++x) {
-        tma_load_5d(smem + kOffQ + x * kQBox, &tmQ, bar_q, x * 64, h, (int)row0, qs, b);
-        tma_load_5d(smem + kOffDO + x * kQBox, &tmDO, bar_q, x * 64, h, (int)row0, qs, b);
+        tma_load_5d(smem + kOffQ + x * kQBox, &tmQ, bar_q, x * 64, h, qr, qs, b);
+        tma_load_5d(smem + kOffDO + x * kQBox, &tmDO, bar_q, x * 64, h, qr, qs, b);
       }
       int nk = 0, nv = 0;  // K / V tiles issued
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int s = shard_of(step);
         const int nt = (int)((cta_keys(s) + BN - 1) / BN);
-        const int ks = p.ring ? s : 0;
         for (int t = 0; t < nt; ++t) {
           const int sk = nk % kKStages, sv = nv % kVStages;
+          int kr, ks;
+          R.tma(s, (int64_t)t * BN, kr, ks);
           if (nk >= kKStages &&
               !mbar_wait(bar_k_empty + sk, ((nk / kKStages) - 1) & 1, limit, p.status)) {
             ok = false;
@@ -704,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar_k_full + sk, kKTile);
           for (int x = 0; x < 2; ++x)
             tma_load_5d(smem + kOffK + sk * kKTile + x * kKBox, &tmK, bar_k_full + sk, x * 64, g,
-                        t * BN, ks, b);
+                        kr, ks, b);
           ++nk;
           if (nv >= kVStages &&
               !mbar_wait(bar_v_empty + sv, ((nv / kVStages) - 1) & 1, limit, p.status)) {
@@ -714,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar_v_full + sv, kKTile);
           for (int x = 0; x < 2; ++x)
             tma_load_5d(smem + kOffV + sv * kKTile + x * kKBox, &tmV, bar_v_full + sv, x * 64, g,
-                        t * BN, ks, b);
+                        kr, ks, b);
           ++nv;
         }
       }
@@ -782,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t row = row0 + lane_base + lane;
     const bool live = row < L;
     const int64_t tq = live ? lay.pos(r, row) : -1;
-    const int64_t qrow = (p.ring ? (int64_t)r * L : 0) + row;
+    const int64_t qrow = R.row(r, row);
     float lse2 = 0.f, dd = 0.f;
     if (live) {
       const int64_t off = ((int64_t)b * p.Hq + h) * p.lse_ld + qrow;
@@ -912,15 +945,17 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.dv_sn = a.dv.stride_n;
   p.dv_sh = a.dv.stride_h;
   p.accumulate = a.accumulate;
+  p.global_order = ring ? a.global_order : 0;
+  const int view = operand_view(a, ring);
   p.status = a.status;
   p.wait_limit = tc_wait_limit();
   if (a.B > 65535) return RM_ERR_UNSUPPORTED;  // grid.z
   {  // dK, dV
     CUtensorMap mq, mk, mv, mdo;
-    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK ||
-        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
-        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK) != RM_OK ||
-        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ) != RM_OK)
+    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ, view) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
+        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ, view) != RM_OK)
       return RM_ERR_CUDA;
     // a key-tile CTA streams Q and dO of every query head of its group
     p.head_block = head_block((int64_t)(a.Hq / a.Hkv) * a.N * D * 2 * 2, a.Hkv);
@@ -935,10 +970,10 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   }
   {  // dQ
     CUtensorMap mq, mk, mv, mdo;
-    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK ||
-        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
-        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN) != RM_OK ||
-        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM) != RM_OK)
+    if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, dq::BM, view) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
+        encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM, view) != RM_OK)
       return RM_ERR_CUDA;
     // a query-tile CTA streams K and V of its KV head (shared by the group)
     const int group = a.Hq / a.Hkv;

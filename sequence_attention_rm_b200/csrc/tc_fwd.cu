@@ -77,6 +77,7 @@ struct FwdParams {
   int ring, q_rank, kv_rank;
   int head_pairs;
   int head_block;  // head units per grid block (see grid_place)
+  int global_order;  // ring operands, O and LSE in global token order
   void* o;
   int64_t o_sb, o_sn, o_sh;
   int o_f32;
@@ -166,6 +167,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     rowB = rowA + kBM;
   }
   const int g = hA / (p.Hq / p.Hkv);
+  RingRows rows;
+  rows.lay = lay;
+  rows.global = p.global_order;
+  // TMA (row, shard) coordinates of local row j of rank `rank` (a single
+  // shard: row j of the one shard)
+  auto tma_rs = [&](int rank, int64_t j, int& crow, int& cshard) {
+    if (p.ring) {
+      rows.tma(rank, j, crow, cshard);
+    } else {
+      crow = (int)j;
+      cshard = 0;
+    }
+  };
   const int64_t last_row = min((p.head_pairs ? rowA : rowB) + kBM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
   const int nsteps = p.ring ? p.P : 1;
@@ -206,23 +220,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int qs = p.ring ? r : 0;
+      int qrA, qsA, qrB, qsB;  // TMA (row, shard) coordinates of the two query tiles
+      tma_rs(r, rowA, qrA, qsA);
+      tma_rs(r, rowB, qrB, qsB);
       mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
 #pragma unroll
       for (int x = 0; x < C::kBoxes; ++x) {
-        tma_load_5d(smem + C::kQ0 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hA, (int)rowA,
-                    qs, b);
-        tma_load_5d(smem + C::kQ1 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hB, (int)rowB,
-                    qs, b);
+        tma_load_5d(smem + C::kQ0 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hA, qrA, qsA, b);
+        tma_load_5d(smem + C::kQ1 + x * C::kBoxBytes, &tmQ, bar_q, x * C::kBoxCols, hB, qrB, qsB, b);
       }
       int j = 0;
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int s = shard_of(step);
         const int nt = (int)((cta_keys(s) + kBN - 1) / kBN);
-        const int ks = p.ring ? s : 0;
         for (int t = 0; t < nt; ++t, ++j) {
           const int st = j & 1;
+          int kr, ks;
+          tma_rs(s, (int64_t)t * kBN, kr, ks);
           if (j >= kStages && !mbar_wait(bar_kv_empty + st, ((j >> 1) - 1) & 1, limit, p.status)) {
             ok = false;
             break;
@@ -231,12 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < C::kBoxes; ++x)
             tma_load_5d(smem + C::kK + st * C::kTileBytes + x * C::kBoxBytes, &tmK,
-                        bar_k_full + st, x * C::kBoxCols, g, t * kBN, ks, b);
+                        bar_k_full + st, x * C::kBoxCols, g, kr, ks, b);
           mbar_arrive_expect_tx(bar_v_full + st, C::kTileBytes);
 #pragma unroll
           for (int x = 0; x < C::kBoxes; ++x)
             tma_load_5d(smem + C::kV + st * C::kTileBytes + x * C::kBoxBytes, &tmV,
-                        bar_v_full + st, x * C::kBoxCols, g, t * kBN, ks, b);
+                        bar_v_full + st, x * C::kBoxCols, g, kr, ks, b);
         }
       }
       // drain: the last load issued into each stage has landed before exit
@@ -414,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       const float lse = l > 0.f ? (((m == -INFINITY) ? 0.f : m) + __log2f(l)) * kLn2 : -INFINITY;
-      const int64_t orow = (p.ring ? (int64_t)r * L : 0) + row;
+      const int64_t orow = p.ring ? rows.row(r, row) : row;
       char* obase = reinterpret_cast<char*>(p.o) +
                     (b * p.o_sb + orow * p.o_sn + (int64_t)h * p.o_sh) * (p.o_f32 ? 4 : 2);
 #pragma unroll
@@ -476,21 +491,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// A [B, P', L, H, d] view (P' = P in ring mode, 1 for a single shard) of a
-// bf16 operand, read in boxes of (box_cols, 1 head, 128 rows); columns past d
-// (head-dim padding) and rows past L are zero-filled by the TMA unit.
+// A TMA view of a [B, N or L, H, d] bf16 operand with 5 coordinates
+// (col, head, row, shard, batch).  view 0: [B, P', L, H, d] (P' = shards, 1
+// for a single shard), row j of shard r at memory row r * L + j -- rank-major
+// ring operands or one shard.  view 1 (global striped): the same dimensions
+// with the row / shard strides swapped, row j of shard r at j * P + r.  view 2
+// (global zigzag): [B, 2P, C, H, d], row j of chunk q at q * C + j.  Boxes of
+// box_rows rows and box_cols columns; columns past d (head-dim padding) and
+// rows past the row dimension are zero-filled by the TMA unit.
 rm_status encode_operand_map(CUtensorMap* map, const rm_tensor& t, int B, int shards, int64_t L,
-                             int H, int d, int box_cols, int box_rows) {
+                             int H, int d, int box_cols, int box_rows, int view) {
   auto fn = encode_fn();
   if (!fn) return RM_ERR_CUDA;
   const int64_t sn = t.stride_n * 2;
   const int64_t sh = (H > 1 ? t.stride_h : d) * 2;
-  const int64_t sp = L * t.stride_n * 2;
   const int64_t sb = (B > 1 ? t.stride_b : (int64_t)shards * L * t.stride_n) * 2;
-  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)shards,
+  int64_t rows = L, nshard = shards, s_row = sn, s_shard = L * sn;
+  if (view == 1) {  // striped: row j of shard r is global row j * P + r
+    s_row = (int64_t)shards * sn;
+    s_shard = sn;
+  } else if (view == 2) {  // zigzag: 2P chunks of C = L / 2 rows
+    rows = L / 2;
+    nshard = 2 * (int64_t)shards;
+    s_shard = rows * sn;
+  }
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)nshard,
                         (cuuint64_t)B};
-  cuuint64_t strides[4] = {(cuuint64_t)sh, (cuuint64_t)sn, (cuuint64_t)(sp > 0 ? sp : 16),
-                           (cuuint64_t)(sb > 0 ? sb : 16)};
+  cuuint64_t strides[4] = {(cuuint64_t)sh, (cuuint64_t)s_row,
+                           (cuuint64_t)(s_shard > 0 ? s_shard : 16), (cuuint64_t)(sb > 0 ? sb : 16)};
   cuuint32_t box[5] = {(cuuint32_t)box_cols, 1, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle swz =
@@ -501,8 +529,12 @@ rm_status encode_operand_map(CUtensorMap* map, const rm_tensor& t, int B, int sh
   return rc == CUDA_SUCCESS ? RM_OK : RM_ERR_CUDA;
 }
 
-// A plain (no swizzle) map for the TMA copies of tma_copy.cu: elements of
-// `esize` bytes moved as unsigned integers (bit copy), zero fill out of range.
+// The operand view (see encode_operand_map) of a ring or single-shard call.
+int operand_view(const AttnArgs& a, bool ring) {
+  if (!ring || !a.global_order) return 0;
+  return a.layout == RM_LAYOUT_STRIPED ? 1 : a.layout == RM_LAYOUT_ZIGZAG ? 2 : 0;
+}
+
 rm_status encode_copy_map(CUtensorMap* map, const void* ptr, int esize, const int64_t (&dims)[5],
                           const int64_t (&strides)[4], const int (&box)[5]) {
   auto fn = encode_fn();
@@ -545,9 +577,10 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   const int64_t L = a.N / a.P;
   const int shards = ring ? a.P : 1;
   CUtensorMap mq, mk, mv;
-  if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, C::kBoxCols, kBM) != RM_OK ||
-      encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN) != RM_OK ||
-      encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN) != RM_OK)
+  const int view = operand_view(a, ring);
+  if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, C::kBoxCols, kBM, view) != RM_OK ||
+      encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK ||
+      encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK)
     return RM_ERR_CUDA;
   FwdParams p;
   p.B = a.B;
@@ -564,6 +597,7 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   p.q_rank = q_rank;
   p.kv_rank = kv_rank;
   p.head_pairs = ((a.Hq / a.Hkv) % 2 == 0) ? 1 : 0;
+  p.global_order = ring ? a.global_order : 0;
   p.o = a.o.ptr;
   p.o_sb = a.o.stride_b;
   p.o_sn = a.o.stride_n;

@@ -23,6 +23,7 @@ RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_WORKSPACE, RM_ERR_CUDA, RM
 RM_F32, RM_BF16 = 0, 1
 LAYOUTS = {"contiguous": 0, "zigzag": 1, "striped": 2}
 MODES = {"fused": 0, "stepwise": 1}
+ORDERS = {"rank": 0, "global": 1}
 
 EXPORTED = (
     "rm_attn_block_fwd", "rm_attn_block_bwd", "rm_attn_bwd_preprocess", "rm_lse_merge",
@@ -42,7 +43,7 @@ class RmAttnDesc(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("Hq", ctypes.c_int),
                 ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("N", ctypes.c_int64),
                 ("P", ctypes.c_int), ("layout", ctypes.c_int), ("causal", ctypes.c_int),
-                ("scale", ctypes.c_float), ("mode", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("mode", ctypes.c_int), ("order", ctypes.c_int)]
 
 
 class RmError(RuntimeError):
@@ -124,9 +125,10 @@ def _bnhd(t: torch.Tensor) -> RmTensor:
 
 
 def desc(dtype: torch.dtype, B: int, Hq: int, Hkv: int, d: int, N: int, P: int, layout: str,
-         causal: bool, scale: float | None = None, mode: str = "fused") -> RmAttnDesc:
+         causal: bool, scale: float | None = None, mode: str = "fused",
+         order: str = "rank") -> RmAttnDesc:
     return RmAttnDesc(_dtype_code(dtype), B, Hq, Hkv, d, N, P, LAYOUTS[layout], int(bool(causal)),
-                      0.0 if scale is None else float(scale), MODES[mode])
+                      0.0 if scale is None else float(scale), MODES[mode], ORDERS[order])
 
 
 # ---- entry points -----------------------------------------------------------
@@ -225,10 +227,13 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None):
 
 
 def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | None = None,
-                  mode: str = "fused", out=None, lse=None, ws=None, stream=None):
-    """Ring forward over P virtual ranks; q/k/v rank-major [B, N, H, d] -> (O, LSE [B, Hq, N])."""
+                  mode: str = "fused", order: str = "rank", out=None, lse=None, ws=None,
+                  stream=None):
+    """Ring forward over P virtual ranks; q/k/v [B, N, H, d] in `order` ("rank":
+    rank-major, "global": the tokens' own order) -> (O, LSE [B, Hq, N]) in the
+    same order."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
     wp, wn = _workspace(ring_workspace_size(dsc, False), q.device, ws)
@@ -238,10 +243,11 @@ def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | 
 
 
 def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
-                  scale: float | None = None, dq=None, dk=None, dv=None, ws=None, stream=None):
-    """Ring backward; returns (dq, dk, dv) in the input dtype, rank-major."""
+                  scale: float | None = None, order: str = "rank", dq=None, dk=None, dv=None,
+                  ws=None, stream=None):
+    """Ring backward; returns (dq, dk, dv) in the input dtype and in `order`."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order)
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
@@ -253,11 +259,12 @@ def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
 
 
 def ring_attn_bwd_noalloc(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
-                          scale: float | None = None, dq=None, dk=None, dv=None, stream=None):
+                          scale: float | None = None, order: str = "rank", dq=None, dk=None,
+                          dv=None, stream=None):
     """rm_ring_attn_bwd without a workspace: the library's fixed device scratch
     (at most 64 MiB of workspace) is used instead."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order)
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv

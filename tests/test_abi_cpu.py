@@ -60,12 +60,26 @@ def _desc(rm, **kw):
     (dict(dtype=9), 1),
     (dict(dtype=0, d=130), 2),  # fp32 d > 128
     (dict(mode=3), 1),
+    (dict(order=5), 1),                      # bad token order
+    (dict(order=1, N=2000, P=2), 2),         # global zigzag: chunk of 500 tokens
+    (dict(order=1, dtype=0), 2),             # global order needs bf16
+    (dict(order=1, mode=1), 2),              # global order needs the fused forward
 ])
 def test_desc_validation(rm, bad, status):
     n = ctypes.c_size_t(0)
     d = _desc(rm, **bad)
     assert rm.raw().rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == status
     assert rm.raw().rm_last_error()
+
+
+def test_global_order_accepted(rm):
+    n = ctypes.c_size_t(0)
+    lib = rm.raw()
+    for kw in (dict(order=1), dict(order=1, layout=2, P=8), dict(order=1, layout=0, dtype=0, mode=1),
+               dict(order=1, P=1, dtype=0, mode=1, N=1000)):
+        d = _desc(rm, **kw)
+        assert lib.rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0, kw
+        assert lib.rm_ring_workspace_size(ctypes.byref(d), 1, ctypes.byref(n)) == 0, kw
 
 
 def test_workspace_sizes(rm):

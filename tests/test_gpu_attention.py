@@ -200,3 +200,59 @@ def test_bf16_backward_other_head_dims_are_rejected(rm):
     with pytest.raises(rm.RmError) as e:
         rm.ring_attn_bwd(qg, kg, vg, o, l, dog, P=2, layout="contiguous", causal=True)
     assert e.value.status == rm.RM_ERR_UNSUPPORTED
+
+
+def _global_ok(case):
+    dtype, B, Hq, Hkv, N, d, P, layout, causal = case
+    return layout != "zigzag" or (N // (2 * P)) % 128 == 0
+
+
+GLOBAL_CASES = [c for c in CASES if c[0] == torch.bfloat16 and _global_ok(c)] + [
+    (torch.bfloat16, 1, 4, 2, 1024, 64, 2, "zigzag", True),
+    (torch.bfloat16, 1, 4, 2, 1024, 32, 8, "striped", True),
+]
+
+
+def _lse_unpermute(rm, lse, layout, P):
+    B, H, N = lse.shape
+    flat = lse.reshape(B * H, N, 1, 1).contiguous()
+    return rm.layout_permute(flat, layout, P, inverse=True).reshape(B, H, N)
+
+
+@pytest.mark.parametrize("case", GLOBAL_CASES, ids=lambda c: f"B{c[1]}H{c[2]}/{c[3]}-N{c[4]}-d{c[5]}-P{c[6]}-{c[7]}-{'c' if c[8] else 'nc'}")
+def test_ring_global_order_matches_rank_major(rm, case):
+    """Global-order operands (the kernels fetch each rank's tiles through the
+    layout) give bit-for-bit the results of permute -> rank-major ring ->
+    un-permute, forward and (d = 128) backward."""
+    dtype, B, Hq, Hkv, N, d, P, layout, causal = case
+    q, k, v, do = (t.cuda() for t in _inputs(dtype, B, Hq, Hkv, N, d, 330 + N))
+    perm = lambda x: rm.layout_permute(x, layout, P)
+    unperm = lambda x: rm.layout_permute(x, layout, P, inverse=True)
+    qr, kr, vr, dor = perm(q), perm(k), perm(v), perm(do)
+    o_r, l_r = rm.ring_attn_fwd(qr, kr, vr, P=P, layout=layout, causal=causal)
+    o_g, l_g = rm.ring_attn_fwd(q, k, v, P=P, layout=layout, causal=causal, order="global")
+    assert torch.equal(o_g, unperm(o_r))
+    assert torch.equal(l_g, _lse_unpermute(rm, l_r, layout, P))
+    if d != 128:
+        return
+    grads_r = rm.ring_attn_bwd(qr, kr, vr, o_r, l_r, dor, P=P, layout=layout, causal=causal)
+    grads_g = rm.ring_attn_bwd(q, k, v, o_g, l_g, do, P=P, layout=layout, causal=causal,
+                               order="global")
+    for name, gr, gg in zip(("dq", "dk", "dv"), grads_r, grads_g):
+        assert torch.equal(gg, unperm(gr)), name
+
+
+def test_ring_global_order_against_oracle(rm):
+    """One global-order case straight against the oracle (no permutes at all)."""
+    case = (torch.bfloat16, 1, 4, 2, 2048, 128, 4, "zigzag", True)
+    dtype, B, Hq, Hkv, N, d, P, layout, causal = case
+    q, k, v, do = _inputs(dtype, B, Hq, Hkv, N, d, 777)
+    o_ref, l_ref = oatt.attention_forward(np64(q), np64(k), np64(v), causal=True)
+    g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=True)
+    qg, kg, vg, dog = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, l = rm.ring_attn_fwd(qg, kg, vg, P=P, layout=layout, causal=True, order="global")
+    assert_max_abs(np64(o), o_ref, BF16_O_TOL, "O")
+    assert_max_abs(np64(l), l_ref, BF16_LSE_TOL, "LSE")
+    grads = rm.ring_attn_bwd(qg, kg, vg, o, l, dog, P=P, layout=layout, causal=True, order="global")
+    for name, g, ref in zip(("dq", "dk", "dv"), grads, g_ref):
+        assert_grad_close(np64(g), ref, what=name)
