@@ -1,6 +1,8 @@
 """Full-size parity of the ring forward + backward at the three bf16 causal
-workloads (16k zigzag P=2, 128k striped P=8, 256k zigzag P=8), in the launch
-configuration bench.py times (fused ring forward, ring backward).
+workloads (16k zigzag P=2, 128k striped P=8, 256k zigzag P=8): the
+rank-major ring (after a layout permute) is checked against the oracle, and
+the launch configuration bench.py times (fused ring forward and ring
+backward on global-order operands) must reproduce its results bit for bit.
 
 The oracle cannot materialise these problems, so it checks what it can
 compute exactly one by one:
@@ -61,6 +63,17 @@ def test_full_size_ring_fwd_bwd(rm, w):
     lse_g = rm.layout_permute(lse.view(w.Hq, w.N, 1, 1), w.layout, w.P, inverse=True).view(
         w.B, w.Hq, w.N).cpu()
     del qr, kr, vr, dor, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+    # the launch configuration bench.py times: the same ring on global-order
+    # operands (no permute pass) must give the same bits
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    og, lg = rm.ring_attn_fwd(qd, kd, vd, P=w.P, layout=w.layout, causal=True, order="global")
+    grads = rm.ring_attn_bwd(qd, kd, vd, og, lg, dod, P=w.P, layout=w.layout, causal=True,
+                             order="global")
+    assert torch.equal(og.cpu(), o_g) and torch.equal(lg.cpu(), lse_g), "global-order forward"
+    for name, a, ref in zip(("dq", "dk", "dv"), grads, (dq_g, dk_g, dv_g)):
+        assert torch.equal(a.cpu(), ref), f"global-order {name}"
+    del qd, kd, vd, dod, og, lg, grads
     torch.cuda.empty_cache()
     assert rm.get_device_status() == rm.RM_OK
 
