@@ -379,23 +379,38 @@ def extras(rm, peaks, peak_src, dev, flush):
     lse_out = torch.empty(1, H, P * Lr, device=dev)
     fn = lambda: rm.lse_merge(o_parts, lse_parts, torch.bfloat16, out=o_out, lse_out=lse_out)
     fn()
-    ms = _time(fn, 5, flush)
+    ms = _time(fn, 10, flush)
     nbytes = P * (P * Lr * H * d * 4 + H * P * Lr * 4) + P * Lr * H * d * 2 + H * P * Lr * 4
     out["lse_merge"] = {"shape": "8 partials x [1, 131072, 16, 128] fp32 -> bf16", "ms": round(ms, 4),
                         "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
                         "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
-    del o_parts, lse_parts, o_out, lse_out
-    # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and fused K|V [8 x 32768, 16, 128]
-    x = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
-    y = torch.empty(8, 8 * 32768, 2, 128, dtype=torch.bfloat16, device=dev)
-    fn = lambda: rm.seq_head_repack(x, 8, out=y)
+    # pairwise merge (the running-state form): fp32 O_acc <- merge(O_acc, O_new), in place
+    acc, lacc = o_parts[0], lse_parts[0]
+    fn = lambda: rm.lse_merge([acc, o_parts[1]], [lacc, lse_parts[1]], torch.float32, out=acc,
+                              lse_out=lacc)
     fn()
-    ms = _time(fn, 5, flush)
-    nbytes = 2 * x.numel() * 2
-    out["repack"] = {"shape": "seq->head [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16", "ms": round(ms, 4),
-                     "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
-                     "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
-    del x, y
+    ms = _time(fn, 10, flush)
+    nbytes = 3 * P * Lr * H * d * 4 + 3 * H * P * Lr * 4
+    out["lse_merge_pairwise"] = {"shape": "2 partials x [1, 131072, 16, 128] fp32 -> fp32 in place",
+                                 "ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1),
+                                 "frac": round(nbytes / ms / 1e6 / hbm, 4), "peak": hbm,
+                                 "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    del o_parts, lse_parts, o_out, lse_out
+    # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and the fused K|V (8 K heads
+    # then 8 V heads) of the same shape, seq -> head, one call each
+    x = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
+    kv = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
+    y = torch.empty(8, 8 * 32768, 2, 128, dtype=torch.bfloat16, device=dev)
+    y2 = torch.empty_like(y)
+    fn = lambda: (rm.seq_head_repack(x, 8, out=y), rm.seq_head_repack(kv, 8, out=y2))
+    fn()
+    ms = _time(fn, 10, flush)
+    nbytes = 2 * (x.numel() + kv.numel()) * 2
+    out["repack"] = {"shape": "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16",
+                     "ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1),
+                     "frac": round(nbytes / ms / 1e6 / hbm, 4), "peak": hbm,
+                     "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    del x, kv, y, y2
     # the causal striped 128k forward (fused ring over 8 virtual ranks)
     w3 = synthetic.STRIPED_128K
     q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
@@ -414,13 +429,13 @@ def extras(rm, peaks, peak_src, dev, flush):
     o2 = torch.empty_like(q)
     fn = lambda: rm.layout_permute(q, "striped", 8, out=o2)
     fn()
-    ms = _time(fn, 5, flush)
+    ms = _time(fn, 10, flush)
     nbytes = 2 * q.numel() * 2
     out["permute"] = {"shape": "striped P=8 [1, 131072, 16, 128] bf16", "ms": round(ms, 4),
                       "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
                       "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
     del q, k, v, o, lse, o2
-    out["tabular_row_fwd"] = tabular_row(rm, flush)
+    out["tabular_row_fwd"], out["tabular_feature_fwd"] = tabular(rm, flush, hbm, peak_src)
     return out
 
 
@@ -430,12 +445,14 @@ def extras(rm, peaks, peak_src, dev, flush):
 EX2_PER_CLK_SM = 16
 
 
-def tabular_row(rm, flush):
-    """Row-axis attention of the tabular workload (20 sequences of 150000 rows,
-    d = 24 padded to 32, non-causal fused ring over 8 contiguous shards on
-    strided views): TFLOP/s of its 4*d flops per pair against the tensor peak,
-    and exponentials per second against the SFU rate (the d = 24 path does
-    only 96 MMA flops per exponential)."""
+def tabular(rm, flush, hbm, peak_src):
+    """The tabular workload.  Row axis (20 sequences of 150000 rows, d = 24
+    padded to 32, non-causal fused ring over 8 contiguous shards on strided
+    views): TFLOP/s of its 4*d flops per pair against the tensor peak, and
+    exponentials per second against the SFU rate (the d = 24 path does only
+    96 MMA flops per exponential).  Feature axis (600000 sequences of 5
+    tokens): GB/s of its algorithmic traffic (read Q, K, V, write O, LSE)
+    against HBM."""
     w = synthetic.TABULAR
     q, k, v = (t.cuda() for t in synthetic.tabular_inputs(w))
     R, F, E, H = w.rows, w.features, w.embed, w.heads
@@ -452,11 +469,24 @@ def tabular_row(rm, flush):
     props = torch.cuda.get_device_properties(0)
     ex2_peak = EX2_PER_CLK_SM * props.multi_processor_count * 1965e6
     ex2_rate = pairs / (ms * 1e-3)
-    return {"shape": f"{seqs} sequences x {R} rows, d={E // H}", "ms": round(ms, 3),
-            "TFLOP/s": round(flops / ms / 1e9, 2),
-            "exp_per_s": round(ex2_rate / 1e12, 3), "exp_unit": "T exp2/s",
-            "exp_frac": round(ex2_rate / ex2_peak, 4),
-            "exp_peak_source": f"derived: {EX2_PER_CLK_SM}/clk/SM x {props.multi_processor_count} SMs x 1965 MHz"}
+    row = {"shape": f"{seqs} sequences x {R} rows, d={E // H}", "ms": round(ms, 3),
+           "TFLOP/s": round(flops / ms / 1e9, 2),
+           "exp_per_s": round(ex2_rate / 1e12, 3), "exp_unit": "T exp2/s",
+           "exp_frac": round(ex2_rate / ex2_peak, 4),
+           "exp_peak_source": f"derived: {EX2_PER_CLK_SM}/clk/SM x {props.multi_processor_count} SMs x 1965 MHz"}
+    del o, lse
+    fview = lambda x: x.view(w.batch * R, F, H, E // H)
+    fo = torch.empty(w.batch * R, F, H, E // H, dtype=torch.bfloat16, device="cuda")
+    flse = torch.empty(w.batch * R, H, F, device="cuda")
+    fn = lambda: rm.attn_block_fwd(fview(q), fview(k), fview(v), N=F, P=1, layout="contiguous",
+                                   causal=False, q_rank=0, kv_rank=0, out=fo, lse=flse)
+    fn()
+    ms = _time(fn, 10, flush)
+    nbytes = 4 * q.numel() * 2 + flse.numel() * 4
+    feat = {"shape": f"{w.batch * R * H} sequences x {F} tokens, d={E // H}", "ms": round(ms, 4),
+            "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
+            "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    return row, feat
 
 
 # ---------------------------------------------------------------------------
@@ -514,10 +544,21 @@ def _cores():
         return os.cpu_count()
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(heads: int):
     secs, flops = oracle_sample(heads)
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
-            "kind": "oracle",
+            "cpu_model": _cpu_model(), "kind": "oracle",
             "sample": f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions "
                       f"12288-14335, virtual rank 0) of {heads} of 16 query heads, N=16384 zigzag "
                       f"P=2; {secs:.1f} s"}
