@@ -59,16 +59,22 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
     const int h = (int)(bh % a.H);
     const int b = (int)(bh / a.H);
     const int64_t lidx = bh * a.lse_ld + t;
+    const bool active = col < a.d;
+    // every load of the row is issued before any of them is used (the O loads
+    // do not wait for the LSE values), so one row costs one memory latency
+    float4 x[kMaxMergeParts];
     float l[kMaxMergeParts];
-    float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kMaxMergeParts; ++i) {
       if (i < nparts) {
+        if (active) x[i] = load4(a.o_ptr[i] + b * a.o_sb[i] + t * a.o_sn[i] + h * a.o_sh[i] + col);
         l[i] = a.lse_ptr[i][lidx];
-        m = fmaxf(m, l[i]);
       }
     }
-    const bool active = col < a.d;
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxMergeParts; ++i)
+      if (i < nparts) m = fmaxf(m, l[i]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lse;
     if (m == -INFINITY) {
@@ -86,11 +92,6 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
       const float inv = 1.0f / sum;
       lse = m + logf(sum);
       if (active) {
-        float4 x[kMaxMergeParts];
-#pragma unroll
-        for (int i = 0; i < kMaxMergeParts; ++i)
-          if (i < nparts)
-            x[i] = load4(a.o_ptr[i] + b * a.o_sb[i] + t * a.o_sn[i] + h * a.o_sh[i] + col);
 #pragma unroll
         for (int i = 0; i < kMaxMergeParts; ++i) {
           if (i < nparts && w[i] != 0.f) {
@@ -121,30 +122,30 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(int B, int64_t N, i
   const int lane = threadIdx.x & 31;
   const int sub = lane / lanes;
   const int col = (lane % lanes) * 4;
-  const int64_t rows = (int64_t)B * H * N;
   const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t base = warp0 * rows_per_warp; base < rows; base += nwarps * rows_per_warp) {
-    const int64_t row = base + sub;
-    const bool valid = row < rows;
-    float s = 0.f;
-    int64_t t = 0, bh = 0;
-    if (valid) {
-      t = row % N;
-      bh = row / N;
-      const int h = (int)(bh % H);
-      const int b = (int)(bh / H);
-      if (col < d) {
-        float4 x = load4(reinterpret_cast<const InT*>(o.ptr) + b * o.stride_b + t * o.stride_n +
-                         h * o.stride_h + col);
-        float4 y = load4(reinterpret_cast<const InT*>(dout.ptr) + b * dout.stride_b +
-                         t * dout.stride_n + h * dout.stride_h + col);
-        s = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
-        if (zero_fill) store4(zero_fill + row * d + col, make_float4(0.f, 0.f, 0.f, 0.f));
+  // a warp takes whole tokens (b, t): its lane groups read the H head rows of
+  // the token, which are contiguous in memory, so the tensor is read in order;
+  // delta is written at its [B, H, N] index
+  const int64_t tokens = (int64_t)B * N;
+  for (int64_t bt = warp0; bt < tokens; bt += nwarps) {
+    const int64_t t = bt % N;
+    const int64_t b = bt / N;
+    const InT* orow = reinterpret_cast<const InT*>(o.ptr) + b * o.stride_b + t * o.stride_n;
+    const InT* drow = reinterpret_cast<const InT*>(dout.ptr) + b * dout.stride_b + t * dout.stride_n;
+    for (int h0 = 0; h0 < H; h0 += rows_per_warp) {
+      const int h = h0 + sub;
+      float v = 0.f;
+      if (h < H && col < d) {
+        const float4 x = load4(orow + (int64_t)h * o.stride_h + col);
+        const float4 y = load4(drow + (int64_t)h * dout.stride_h + col);
+        v = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+        if (zero_fill)
+          store4(zero_fill + ((b * H + h) * N + t) * d + col, make_float4(0.f, 0.f, 0.f, 0.f));
       }
+      for (int off = lanes >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (h < H && (lane % lanes) == 0) delta[(b * H + h) * N + t] = v;
     }
-    for (int off = lanes >> 1; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (valid && (lane % lanes) == 0) delta[row] = s;
   }
 }
 
@@ -211,7 +212,7 @@ cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, r
   const int64_t rows = (int64_t)B * H * N;
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(d);
-  int grid = grid_for_rows(rows, g.rows_per_warp);
+  int grid = grid_for_rows((int64_t)B * N, 1);  // one token per warp pass
   ProfScope ps("bwd_preprocess", stream);
   if (in_bf16)
     bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
