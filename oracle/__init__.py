@@ -30,10 +30,11 @@ Modules:
 - ``ring``       the ring over P ranks (forward and backward)
 - ``repack``     Ulysses sequence<->head repack as explicit index loops
 - ``multiaxis``  row-axis / feature-axis routing of a tabular tensor
+- ``usp``        Ulysses x ring composition (USP) and its degree selection
 
 Parity status: every function above is pinned by ``tests/test_oracle_*.py``
 (closed forms, brute force, invariants, finite differences, a library
 cross-check); none is "parity unpinned".
 """
 
-from . import attention, layouts, merge, multiaxis, repack, ring  # noqa: F401
+from . import attention, layouts, merge, multiaxis, repack, ring, usp  # noqa: F401
