@@ -224,6 +224,43 @@ rm_status rm_ring_attn_bwd_noalloc(const rm_attn_desc* desc, rm_tensor q, rm_ten
                                    rm_tensor dout, rm_tensor dq, rm_tensor dk,
                                    rm_tensor dv, void* stream);
 
+/* ---- USP: the Ulysses head all-to-all composed with the ring ------------- */
+
+/* The split of `world` virtual devices into ulysses x ring [ringmaster,
+ * "Why": USP on a 2-D mesh, with an auto-selector driven by the KV-head count
+ * and the world size]: the largest Ulysses degree that divides `world` and
+ * Hkv (the Ulysses cap) and is at most `node_size`; ring = world / ulysses.
+ * Host only.  RM_ERR_INVALID_ARG for non-positive sizes or Hq % Hkv != 0. */
+rm_status rm_usp_auto_select(int Hq, int Hkv, int world, int node_size, int* ulysses,
+                             int* ring);
+
+/* Workspace bytes of rm_usp_attn_fwd (backward = 0) or rm_usp_attn_bwd (1). */
+rm_status rm_usp_workspace_size(const rm_attn_desc* desc, int ulysses, int backward,
+                                size_t* bytes);
+
+/* USP forward on one GPU: desc->P is the ring degree (the layout's rank
+ * count) and `ulysses` the Ulysses degree, so P * ulysses virtual devices.
+ * Each ring shard is cut into `ulysses` contiguous sub-shards; inside every
+ * ring group the seq->head repack (rm_seq_head_repack) gives each Ulysses rank
+ * the whole ring shard for Hq/ulysses query heads (and Hkv/ulysses KV heads);
+ * the ring (rm_ring_attn_fwd, desc->mode / order) then runs for every head
+ * group over the P ring ranks, and the head->seq repack returns O.
+ * q/o [B, N, Hq, d], k/v [B, N, Hkv, d]: DENSE tensors in desc->order for the
+ * P ring ranks; lse fp32 [B, Hq, N].  Needs Hq % ulysses == Hkv % ulysses ==
+ * (N/P) % ulysses == 0.  ws: rm_usp_workspace_size(desc, ulysses, 0) bytes,
+ * 256-byte aligned (the repacked operands and the ring's own workspace). */
+rm_status rm_usp_attn_fwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm_tensor k,
+                          rm_tensor v, rm_tensor o, float* lse, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* USP backward: repack q, k, v, o, dout; rm_ring_attn_bwd per head group;
+ * repack dq, dk, dv back.  Same layouts and requirements as the forward;
+ * ws: rm_usp_workspace_size(desc, ulysses, 1) bytes. */
+rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm_tensor k,
+                          rm_tensor v, rm_tensor o, const float* lse, rm_tensor dout,
+                          rm_tensor dq, rm_tensor dk, rm_tensor dv, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* ---- bit-exact layout transforms ---------------------------------------- */
 
 /* Global token order <-> rank-major order (see pos(r, j) above) of a dense

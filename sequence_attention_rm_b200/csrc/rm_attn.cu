@@ -543,4 +543,164 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
   return tc_bwd(a, -1, -1, st);
 }
 
+// ---- USP ------------------------------------------------------------------
+
+rm_status rm_usp_auto_select(int Hq, int Hkv, int world, int node_size, int* ulysses,
+                             int* ring) {
+  if (Hq < 1 || Hkv < 1 || world < 1 || node_size < 1 || !ulysses || !ring)
+    return fail(RM_ERR_INVALID_ARG, "bad USP selector arguments");
+  if (Hq % Hkv) return fail(RM_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  int best = 1;
+  for (int u = 1; u <= world; ++u)
+    if (world % u == 0 && Hkv % u == 0 && u <= node_size) best = u;
+  *ulysses = best;
+  *ring = world / best;
+  return RM_OK;
+}
+
+namespace {
+
+// The ring problem of one USP call: every (batch, head group) is a sequence
+// of its own, with Hq/u query and Hkv/u KV heads.
+rm_status usp_desc(const rm_attn_desc* desc, int u, rm_attn_desc* out) {
+  RM_TRY(check_desc(desc));
+  if (u < 1) return fail(RM_ERR_INVALID_ARG, "ulysses degree must be >= 1");
+  if (desc->Hq % u || desc->Hkv % u)
+    return fail(RM_ERR_INVALID_ARG, "ulysses degree %d must divide Hq (%d) and Hkv (%d)", u,
+                desc->Hq, desc->Hkv);
+  if ((desc->N / desc->P) % u)
+    return fail(RM_ERR_INVALID_ARG, "ulysses degree %d must divide the ring shard (%lld tokens)",
+                u, (long long)(desc->N / desc->P));
+  *out = *desc;
+  out->B = desc->B * u;
+  out->Hq = desc->Hq / u;
+  out->Hkv = desc->Hkv / u;
+  return RM_OK;
+}
+
+struct UspWs {
+  size_t q, kv, ring_off, ring_bytes, total;  // q / kv: bytes of one repacked operand
+};
+
+rm_status usp_ws(const rm_attn_desc* desc, int u, int backward, UspWs* w) {
+  rm_attn_desc d2;
+  RM_TRY(usp_desc(desc, u, &d2));
+  const size_t es = esize_of(desc->dtype);
+  w->q = align_up((size_t)desc->B * desc->N * desc->Hq * desc->d * es);
+  w->kv = align_up((size_t)desc->B * desc->N * desc->Hkv * desc->d * es);
+  // forward: q, o, k, v; backward: q, o, dout, dq and k, v, dk, dv
+  w->ring_off = backward ? 4 * w->q + 4 * w->kv : 2 * w->q + 2 * w->kv;
+  size_t rb = 0;
+  RM_TRY(rm_ring_workspace_size(&d2, backward, &rb));
+  w->ring_bytes = rb;
+  w->total = w->ring_off + align_up(rb);
+  return RM_OK;
+}
+
+bool dense(const rm_tensor& t, int64_t N, int H, int d) {
+  return t.stride_h == d && t.stride_n == (int64_t)H * d && t.stride_b == N * H * d;
+}
+
+// seq->head (or back) of every batch entry of a dense [B, N, H, d] tensor:
+// batch b viewed as [u, N/u, H, d] <-> [u, N, H/u, d] at the same offset.
+rm_status usp_repack(const rm_attn_desc* desc, int u, int H, int head_to_seq, const void* in,
+                     void* out, cudaStream_t st) {
+  const int es = esize_of(desc->dtype);
+  const int64_t per = desc->N * H * desc->d * es;
+  for (int b = 0; b < desc->B; ++b)
+    RM_CUDA(launch_seq_head_repack(es, u, desc->N / u, H, desc->d, head_to_seq,
+                                   (const char*)in + b * per, (char*)out + b * per, st),
+            "usp repack launch");
+  return RM_OK;
+}
+
+rm_tensor dense_t(void* p, const rm_attn_desc& d2, int H) {
+  rm_tensor t;
+  t.ptr = p;
+  t.stride_h = d2.d;
+  t.stride_n = (int64_t)H * d2.d;
+  t.stride_b = d2.N * H * d2.d;
+  return t;
+}
+
+}  // namespace
+
+rm_status rm_usp_workspace_size(const rm_attn_desc* desc, int ulysses, int backward,
+                                size_t* bytes) {
+  if (!bytes) return fail(RM_ERR_INVALID_ARG, "bytes is NULL");
+  UspWs w;
+  RM_TRY(usp_ws(desc, ulysses, backward, &w));
+  *bytes = w.total;
+  return RM_OK;
+}
+
+rm_status rm_usp_attn_fwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm_tensor k,
+                          rm_tensor v, rm_tensor o, float* lse, void* ws, size_t ws_bytes,
+                          void* stream) {
+  rm_attn_desc d2;
+  RM_TRY(usp_desc(desc, ulysses, &d2));
+  if (desc->B == 0 || desc->N == 0) return RM_OK;
+  const int64_t N = desc->N;
+  if (!dense(q, N, desc->Hq, desc->d) || !dense(o, N, desc->Hq, desc->d) ||
+      !dense(k, N, desc->Hkv, desc->d) || !dense(v, N, desc->Hkv, desc->d))
+    return fail(RM_ERR_INVALID_ARG, "USP operands must be dense [B, N, H, d]");
+  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse) return fail(RM_ERR_INVALID_ARG, "NULL pointer");
+  UspWs w;
+  RM_TRY(usp_ws(desc, ulysses, 0, &w));
+  if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = (char*)ws;
+  void *yq = base, *yo = base + w.q, *yk = base + 2 * w.q, *yv = base + 2 * w.q + w.kv;
+  const int u = ulysses;
+  RM_TRY(usp_repack(desc, u, desc->Hq, 0, q.ptr, yq, st));
+  RM_TRY(usp_repack(desc, u, desc->Hkv, 0, k.ptr, yk, st));
+  RM_TRY(usp_repack(desc, u, desc->Hkv, 0, v.ptr, yv, st));
+  // lse [B, Hq, N] is [B*u, Hq/u, N]: the ring writes it in place
+  RM_TRY(rm_ring_attn_fwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
+                          dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
+                          base + w.ring_off, w.ring_bytes, stream));
+  return usp_repack(desc, u, desc->Hq, 1, yo, o.ptr, st);
+}
+
+rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm_tensor k,
+                          rm_tensor v, rm_tensor o, const float* lse, rm_tensor dout,
+                          rm_tensor dq, rm_tensor dk, rm_tensor dv, void* ws, size_t ws_bytes,
+                          void* stream) {
+  rm_attn_desc d2;
+  RM_TRY(usp_desc(desc, ulysses, &d2));
+  if (desc->B == 0 || desc->N == 0) return RM_OK;
+  const int64_t N = desc->N;
+  const int hq = desc->Hq, hkv = desc->Hkv, d = desc->d;
+  if (!dense(q, N, hq, d) || !dense(o, N, hq, d) || !dense(dout, N, hq, d) ||
+      !dense(dq, N, hq, d) || !dense(k, N, hkv, d) || !dense(v, N, hkv, d) ||
+      !dense(dk, N, hkv, d) || !dense(dv, N, hkv, d))
+    return fail(RM_ERR_INVALID_ARG, "USP operands must be dense [B, N, H, d]");
+  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !dout.ptr || !dq.ptr || !dk.ptr || !dv.ptr || !lse)
+    return fail(RM_ERR_INVALID_ARG, "NULL pointer");
+  UspWs w;
+  RM_TRY(usp_ws(desc, ulysses, 1, &w));
+  if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = (char*)ws;
+  void *yq = base, *yo = base + w.q, *ydo = base + 2 * w.q, *ydq = base + 3 * w.q;
+  char* kvb = base + 4 * w.q;
+  void *yk = kvb, *yv = kvb + w.kv, *ydk = kvb + 2 * w.kv, *ydv = kvb + 3 * w.kv;
+  const int u = ulysses;
+  RM_TRY(usp_repack(desc, u, hq, 0, q.ptr, yq, st));
+  RM_TRY(usp_repack(desc, u, hkv, 0, k.ptr, yk, st));
+  RM_TRY(usp_repack(desc, u, hkv, 0, v.ptr, yv, st));
+  RM_TRY(usp_repack(desc, u, hq, 0, o.ptr, yo, st));
+  RM_TRY(usp_repack(desc, u, hq, 0, dout.ptr, ydo, st));
+  RM_TRY(rm_ring_attn_bwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
+                          dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
+                          dense_t(ydo, d2, d2.Hq), dense_t(ydq, d2, d2.Hq),
+                          dense_t(ydk, d2, d2.Hkv), dense_t(ydv, d2, d2.Hkv), base + w.ring_off,
+                          w.ring_bytes, stream));
+  RM_TRY(usp_repack(desc, u, hq, 1, ydq, dq.ptr, st));
+  RM_TRY(usp_repack(desc, u, hkv, 1, ydk, dk.ptr, st));
+  return usp_repack(desc, u, hkv, 1, ydv, dv.ptr, st);
+}
+
 }  // extern "C"

@@ -30,7 +30,8 @@ EXPORTED = (
     "rm_ring_workspace_size", "rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_layout_permute",
     "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
     "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
-    "rm_profile_get",
+    "rm_profile_get", "rm_usp_auto_select", "rm_usp_workspace_size", "rm_usp_attn_fwd",
+    "rm_usp_attn_bwd",
 )
 
 
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_profile_enable": [i],
         "rm_profile_count": [],
         "rm_profile_get": [i, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)],
+        "rm_usp_auto_select": [i, i, i, i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)],
+        "rm_usp_workspace_size": [D, i, i, ctypes.POINTER(sz)],
+        "rm_usp_attn_fwd": [D, i, T, T, T, T, vp, vp, sz, vp],
+        "rm_usp_attn_bwd": [D, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -271,6 +276,50 @@ def ring_attn_bwd_noalloc(q, k, v, o, lse, dout, *, P: int, layout: str, causal:
     _check(_lib.rm_ring_attn_bwd_noalloc(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
                                          _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv),
                                          _stream(stream)))
+    return dq, dk, dv
+
+
+def usp_auto_select(Hq: int, Hkv: int, world: int, node_size: int = 8) -> tuple[int, int]:
+    """(ulysses, ring) split of `world` virtual devices for USP."""
+    u, r = ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.rm_usp_auto_select(Hq, Hkv, world, node_size, ctypes.byref(u), ctypes.byref(r)))
+    return u.value, r.value
+
+
+def usp_workspace_size(dsc: RmAttnDesc, ulysses: int, backward: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.rm_usp_workspace_size(ctypes.byref(dsc), ulysses, int(backward), ctypes.byref(n)))
+    return n.value
+
+
+def usp_attn_fwd(q, k, v, *, P: int, ulysses: int, layout: str, causal: bool,
+                 scale: float | None = None, mode: str = "fused", order: str = "rank", out=None,
+                 lse=None, ws=None, stream=None):
+    """USP forward: Ulysses degree `ulysses` x ring degree P; dense q/k/v
+    [B, N, H, d] in `order` for the P ring ranks -> (O, LSE [B, Hq, N])."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order)
+    out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    wp, wn = _workspace(usp_workspace_size(dsc, ulysses, False), q.device, ws)
+    _check(_lib.rm_usp_attn_fwd(ctypes.byref(dsc), ulysses, _bnhd(q), _bnhd(k), _bnhd(v),
+                                _bnhd(out), _ptr(lse), wp, wn, _stream(stream)))
+    return out, lse
+
+
+def usp_attn_bwd(q, k, v, o, lse, dout, *, P: int, ulysses: int, layout: str, causal: bool,
+                 scale: float | None = None, order: str = "rank", dq=None, dk=None, dv=None,
+                 ws=None, stream=None):
+    """USP backward -> (dq, dk, dv) in the input dtype and order."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order)
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    wp, wn = _workspace(usp_workspace_size(dsc, ulysses, True), q.device, ws)
+    _check(_lib.rm_usp_attn_bwd(ctypes.byref(dsc), ulysses, _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
+                                _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
+                                _stream(stream)))
     return dq, dk, dv
 
 

@@ -129,3 +129,32 @@ def test_entry_points_reject_bad_arguments_before_launch(rm):
                                 nul) == 3
     # block forward: rank out of range
     assert lib.rm_attn_block_fwd(ctypes.byref(d), 2, 0, ok, kv, kv, ok, 0, p, nul) == 1
+
+
+def test_usp_auto_select_matches_the_rule(rm):
+    from oracle import usp as ousp
+    for hkv in (1, 2, 3, 4, 8, 16):
+        for group in (1, 2, 4):
+            for world in (1, 2, 4, 6, 8, 12, 16, 32):
+                assert rm.usp_auto_select(hkv * group, hkv, world) == ousp.auto_select(
+                    hkv * group, hkv, world)
+    assert rm.usp_auto_select(64, 16, 32, node_size=8) == (8, 4)
+
+
+@pytest.mark.parametrize("kw,u", [(dict(), 3), (dict(), 16), (dict(N=16386, P=2), 4),
+                                  (dict(Hq=12, Hkv=6), 4)])
+def test_usp_validation(rm, kw, u):
+    n = ctypes.c_size_t(0)
+    d = _desc(rm, **kw)
+    assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), u, 0, ctypes.byref(n)) != 0
+
+
+def test_usp_workspace_sizes(rm):
+    n = ctypes.c_size_t(0)
+    d = _desc(rm)  # bf16 B=1 Hq=16 Hkv=8 d=128 N=16384 P=2
+    q_bytes = 16384 * 16 * 128 * 2
+    kv_bytes = 16384 * 8 * 128 * 2
+    assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), 2, 0, ctypes.byref(n)) == 0
+    assert n.value == 2 * q_bytes + 2 * kv_bytes
+    assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), 2, 1, ctypes.byref(n)) == 0
+    assert n.value == 4 * q_bytes + 4 * kv_bytes + 16 * 16384 * 4
