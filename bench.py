@@ -436,7 +436,37 @@ def extras(rm, peaks, peak_src, dev, flush):
                       "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
     del q, k, v, o, lse, o2
     out["tabular_row_fwd"], out["tabular_feature_fwd"] = tabular(rm, flush, hbm, peak_src)
+    out["usp_16k_fwd_bwd"] = usp_line(rm, flush, peaks, peak_src)
     return out
+
+
+def usp_line(rm, flush, peaks, peak_src):
+    """USP fwd+bwd on the Llama-like 16k workload for a world of 16 virtual
+    devices: the selector gives Ulysses 8 x ring 2 (zigzag), global order."""
+    w = synthetic.LLAMA_ZIGZAG
+    u, p_ring = rm.usp_auto_select(w.Hq, w.Hkv, 16)
+    q, k, v, do = (t.cuda() for t in synthetic.attention_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.N, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsc = rm.desc(w.dtype, w.B, w.Hq, w.Hkv, w.d, w.N, p_ring, w.layout, True, order="global")
+    wsf = torch.empty(max(rm.usp_workspace_size(dsc, u, False), 256), dtype=torch.uint8,
+                      device="cuda")
+    wsb = torch.empty(max(rm.usp_workspace_size(dsc, u, True), 256), dtype=torch.uint8,
+                      device="cuda")
+
+    def fn():
+        rm.usp_attn_fwd(q, k, v, P=p_ring, ulysses=u, layout=w.layout, causal=True,
+                        order="global", out=o, lse=lse, ws=wsf)
+        rm.usp_attn_bwd(q, k, v, o, lse, do, P=p_ring, ulysses=u, layout=w.layout, causal=True,
+                        order="global", dq=dq, dk=dk, dv=dv, ws=wsb)
+    fn()
+    ms = _time(fn, 5, flush)
+    tf = (flops_fwd(w) + flops_bwd(w)) / (ms * 1e-3) / 1e12
+    return {"split": f"ulysses {u} x ring {p_ring} ({w.layout})", "ms": round(ms, 4),
+            "TFLOP/s": round(tf, 2), "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "note": "includes the 8 repack launches of Q/K/V/O/dO and dQ/dK/dV"}
 
 
 # exp2 rate of the SFU: 16 results per clock per SM on sm_100 (the documented
