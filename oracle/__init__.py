@@ -24,7 +24,8 @@ sequence does not need a 137 GB matrix); there is no online softmax and no
 tiling of the key axis anywhere in this package.
 
 Modules:
-- ``attention``  exact attention forward / backward on one (Q, KV) pair
+- ``attention``  exact attention forward / backward on one (Q, KV) pair,
+                 optionally packed or right-padded (segment ids)
 - ``merge``      LSE merge of partial (O, LSE) results
 - ``layouts``    contiguous / zigzag / striped global-position maps, permutes
 - ``ring``       the ring over P ranks (forward and backward)

@@ -21,7 +21,13 @@ Readings of points the pages leave open:
   function serves any shard pair of any layout;
 - grouped-query attention: query head h reads KV head h // (Hq // Hkv)
   (contiguous groups; ringmaster "Quickstart" only names num_kv_heads);
-- a query row with no visible key has o = 0 and lse = -inf.
+- a query row with no visible key has o = 0 and lse = -inf;
+- packed and right-padded batches (ringmaster "Status": attention takes dense
+  causal sequences or globally right-padded batches; packed attention uses
+  global position boundaries): ``seg`` gives every global position of every
+  batch entry a segment id, -1 for padding.  A key is visible to a query only
+  inside the query's segment (and, if causal, not after it); padding tokens
+  see nothing and are seen by nothing.
 
 The full score row of each query is materialised; queries are processed in
 row blocks only to bound host memory.  No online softmax is used.
@@ -48,11 +54,45 @@ def kv_head_of(h: int, hq: int, hkv: int) -> int:
     return h // (hq // hkv)
 
 
-def visible(q_pos: np.ndarray, k_pos: np.ndarray, causal: bool) -> np.ndarray:
-    """Boolean [Nq, Nk]: may query at global position q_pos[i] see key k_pos[j]."""
+def visible(q_pos: np.ndarray, k_pos: np.ndarray, causal: bool, q_seg=None,
+            k_seg=None) -> np.ndarray:
+    """Boolean [Nq, Nk]: may query at global position q_pos[i] see key k_pos[j].
+    q_seg / k_seg: segment ids of those positions (-1 = padding), or None."""
     if not causal:
-        return np.ones((len(q_pos), len(k_pos)), dtype=bool)
-    return k_pos[None, :] <= q_pos[:, None]
+        vis = np.ones((len(q_pos), len(k_pos)), dtype=bool)
+    else:
+        vis = k_pos[None, :] <= q_pos[:, None]
+    if q_seg is not None:
+        vis = vis & (k_seg[None, :] == q_seg[:, None]) & (k_seg[None, :] >= 0)
+    return vis
+
+
+def segments_from_boundaries(cu, n: int) -> np.ndarray:
+    """Segment id of each of n global positions from boundaries
+    0 = cu[0] < cu[1] < ... < cu[S] <= n (packing); positions >= cu[S] are
+    padding (-1).  Shape [n]."""
+    cu = np.asarray(cu, dtype=np.int64)
+    seg = np.full(n, -1, dtype=np.int64)
+    for i in range(len(cu) - 1):
+        seg[cu[i]:cu[i + 1]] = i
+    return seg
+
+
+def segments_from_lengths(lengths, n: int) -> np.ndarray:
+    """Right padding: batch entry b holds lengths[b] valid tokens, then
+    padding.  Shape [B, n]."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    seg = np.full((len(lengths), n), -1, dtype=np.int64)
+    for b, length in enumerate(lengths):
+        seg[b, :length] = 0
+    return seg
+
+
+def _segs(seg, b, q_pos, k_pos):
+    if seg is None:
+        return None, None
+    row = np.asarray(seg)[b] if np.ndim(seg) == 2 else np.asarray(seg)
+    return row[q_pos], row[k_pos]
 
 
 def _prepare(q, k, v, scale, q_pos, k_pos):
@@ -99,10 +139,12 @@ def _softmax_rows(s: np.ndarray, vis: np.ndarray):
     return probs, lse
 
 
-def attention_forward(q, k, v, scale=None, causal=False, q_pos=None, k_pos=None):
+def attention_forward(q, k, v, scale=None, causal=False, q_pos=None, k_pos=None, seg=None):
     """(o, lse) of softmax(q k^T * scale) v with optional causal mask.
 
-    Returns o [B, Nq, Hq, dv] float64 and lse [B, Hq, Nq] float64.
+    seg: segment ids [B, N] or [N] by global position (see the module
+    docstring), or None.  Returns o [B, Nq, Hq, dv] float64 and lse
+    [B, Hq, Nq] float64.
     """
     q, k, v, scale, q_pos, k_pos = _prepare(q, k, v, scale, q_pos, k_pos)
     B, nq, hq, _ = q.shape
@@ -110,12 +152,15 @@ def attention_forward(q, k, v, scale=None, causal=False, q_pos=None, k_pos=None)
     o = np.zeros((B, nq, hq, dv))
     lse = np.full((B, hq, nq), -np.inf)
     for b in range(B):
+        qs, ks = _segs(seg, b, q_pos, k_pos)
         for h in range(hq):
             g = kv_head_of(h, hq, hkv)
             kk, vv = k[b, :, g, :], v[b, :, g, :]
             for r0, r1 in _row_blocks(nq, nk):
                 s = (q[b, r0:r1, h, :] @ kk.T) * scale
-                probs, row_lse = _softmax_rows(s, visible(q_pos[r0:r1], k_pos, causal))
+                vis = visible(q_pos[r0:r1], k_pos, causal,
+                              None if qs is None else qs[r0:r1], ks)
+                probs, row_lse = _softmax_rows(s, vis)
                 o[b, r0:r1, h, :] = probs @ vv
                 lse[b, h, r0:r1] = row_lse
     return o, lse
@@ -148,7 +193,7 @@ def delta_from_output(dout, o):
 
 
 def attention_backward_block(q, k, v, dout, lse, delta, scale=None, causal=False,
-                             q_pos=None, k_pos=None):
+                             q_pos=None, k_pos=None, seg=None):
     """Gradient contributions of one (query set, key set) pair.
 
     The probabilities are rebuilt from the given row LSE (the LSE of the whole
@@ -176,6 +221,7 @@ def attention_backward_block(q, k, v, dout, lse, delta, scale=None, causal=False
     dk = np.zeros(k.shape)
     dv = np.zeros(v.shape)
     for b in range(B):
+        qs, ks = _segs(seg, b, q_pos, k_pos)
         for h in range(hq):
             g = kv_head_of(h, hq, hkv)
             kk, vv = k[b, :, g, :], v[b, :, g, :]
@@ -183,7 +229,8 @@ def attention_backward_block(q, k, v, dout, lse, delta, scale=None, causal=False
                 qq = q[b, r0:r1, h, :]
                 do = dout[b, r0:r1, h, :]
                 s = (qq @ kk.T) * scale
-                vis = visible(q_pos[r0:r1], k_pos, causal)
+                vis = visible(q_pos[r0:r1], k_pos, causal,
+                              None if qs is None else qs[r0:r1], ks)
                 with np.errstate(over="ignore", invalid="ignore"):
                     probs = np.where(vis, np.exp(s - lse[b, h, r0:r1, None]), 0.0)
                 dv[b, :, g, :] += probs.T @ do
@@ -194,7 +241,8 @@ def attention_backward_block(q, k, v, dout, lse, delta, scale=None, causal=False
     return dq, dk, dv
 
 
-def attention_backward(q, k, v, dout, scale=None, causal=False, q_pos=None, k_pos=None):
+def attention_backward(q, k, v, dout, scale=None, causal=False, q_pos=None, k_pos=None,
+                       seg=None):
     """(dq, dk, dv) of sum(dout * attention_forward(q, k, v)[0]).
 
     D_t is taken straight from the definition, D_t = sum_u P_tu dP_tu, with the
@@ -204,14 +252,17 @@ def attention_backward(q, k, v, dout, scale=None, causal=False, q_pos=None, k_po
     dout = np.asarray(dout, dtype=np.float64)
     B, nq, hq, _ = q.shape
     nk, hkv = k.shape[1], k.shape[2]
-    _, lse = attention_forward(q, k, v, scale, causal, q_pos, k_pos)
+    _, lse = attention_forward(q, k, v, scale, causal, q_pos, k_pos, seg)
     delta = np.zeros((B, hq, nq))
     for b in range(B):
+        qs, ks = _segs(seg, b, q_pos, k_pos)
         for h in range(hq):
             g = kv_head_of(h, hq, hkv)
             for r0, r1 in _row_blocks(nq, nk):
                 s = (q[b, r0:r1, h, :] @ k[b, :, g, :].T) * scale
-                probs, _ = _softmax_rows(s, visible(q_pos[r0:r1], k_pos, causal))
+                vis = visible(q_pos[r0:r1], k_pos, causal,
+                              None if qs is None else qs[r0:r1], ks)
+                probs, _ = _softmax_rows(s, vis)
                 dp = dout[b, r0:r1, h, :] @ v[b, :, g, :].T
                 delta[b, h, r0:r1] = (probs * dp).sum(axis=1)
-    return attention_backward_block(q, k, v, dout, lse, delta, scale, causal, q_pos, k_pos)
+    return attention_backward_block(q, k, v, dout, lse, delta, scale, causal, q_pos, k_pos, seg)

@@ -16,6 +16,9 @@ its query rows and uses the row term D_t = dO_t . O_t of the final O; dQ of a
 rank sums over its steps, dK / dV of a shard sum over all ranks that used it
 (on real hardware they travel back round the ring; here it is a sum).
 
+``seg`` (segment ids by global position, see ``attention``) restricts every
+pair to same-segment keys: packed and right-padded batches.
+
 Tensors are in rank-major order along the token axis (see ``layouts``):
 q, dout [B, N, Hq, d]; k, v [B, N, Hkv, d]; lse [B, Hq, N].
 """
@@ -36,7 +39,8 @@ def _shard(x, r, local):
     return x[:, r * local:(r + 1) * local]
 
 
-def ring_forward(q, k, v, layout: str, p: int, causal: bool, scale=None, return_partials=False):
+def ring_forward(q, k, v, layout: str, p: int, causal: bool, scale=None, return_partials=False,
+                 seg=None):
     """(o, lse) for all ranks; o [B, N, Hq, dv], lse [B, Hq, N], rank-major order.
 
     With return_partials, also returns partials[r][k] = (o, lse) of rank r at
@@ -55,7 +59,7 @@ def ring_forward(q, k, v, layout: str, p: int, causal: bool, scale=None, return_
             s = table[r][step]
             parts.append(attention.attention_forward(
                 _shard(q, r, local), _shard(k, s, local), _shard(v, s, local),
-                scale=scale, causal=causal, q_pos=pos[r], k_pos=pos[s]))
+                scale=scale, causal=causal, q_pos=pos[r], k_pos=pos[s], seg=seg))
         o_r, lse_r = merge.lse_merge([a for a, _ in parts], [b for _, b in parts])
         o_out.append(o_r)
         lse_out.append(lse_r)
@@ -67,7 +71,8 @@ def ring_forward(q, k, v, layout: str, p: int, causal: bool, scale=None, return_
     return o, lse
 
 
-def ring_backward(q, k, v, o, lse, dout, layout: str, p: int, causal: bool, scale=None):
+def ring_backward(q, k, v, o, lse, dout, layout: str, p: int, causal: bool, scale=None,
+                  seg=None):
     """(dq, dk, dv) in rank-major order, from the final o and lse of the forward."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -89,7 +94,7 @@ def ring_backward(q, k, v, o, lse, dout, layout: str, p: int, causal: bool, scal
             gq, gk, gv = attention.attention_backward_block(
                 q[:, rows], k[:, cols], v[:, cols], np.asarray(dout, dtype=np.float64)[:, rows],
                 np.asarray(lse)[:, :, rows], delta[:, :, rows],
-                scale=scale, causal=causal, q_pos=pos[r], k_pos=pos[s])
+                scale=scale, causal=causal, q_pos=pos[r], k_pos=pos[s], seg=seg)
             dq[:, rows] += gq
             dk[:, cols] += gk
             dv[:, cols] += gv
