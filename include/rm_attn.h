@@ -104,8 +104,8 @@ typedef struct {
 typedef enum { RM_ORDER_RANK_MAJOR = 0, RM_ORDER_GLOBAL = 1 } rm_order;
 
 /* One attention problem: B sequences of N tokens split over P virtual ranks
- * (L = N / P tokens each) laid out by `layout`.  d is the true head
- * dimension.  bf16 supports d in {24, 32, 64, 128} (24 is zero-padded to 32
+ * (L = N / P tokens each) laid out by `layout`; N < 2^31 (token positions
+ * are 32-bit on the device).  d is the true head dimension.  bf16 supports d in {24, 32, 64, 128} (24 is zero-padded to 32
  * on chip); fp32 supports d % 4 == 0, d <= 128. */
 typedef struct {
   rm_dtype dtype;
@@ -121,6 +121,23 @@ typedef struct {
   rm_ring_mode mode;  /* rm_ring_attn_fwd only */
   rm_order order;     /* rm_ring_attn_fwd / _bwd only: token order of every
                          [B, N, H, d] operand and of lse / delta */
+  /* Packed or right-padded batches [ringmaster, "Status": dense causal
+   * sequences or globally right-padded batches; packing by global position
+   * boundaries].  A key is visible only inside its query's segment (and not
+   * after it when causal); padding tokens see nothing and are seen by
+   * nothing (their O is 0, their LSE -inf, their gradients 0).  At most one:
+   *   cu_seqlens: device int32[num_segments + 1], global positions
+   *               0 = cu[0] < cu[1] < ... < cu[num_segments] <= N; positions
+   *               from cu[num_segments] on are padding; needs B == 1;
+   *   seq_lens:   device int32[B], valid tokens of each batch entry (right
+   *               padding).
+   * NULL / 0: dense.  Supported on the bf16 tensor-core path (fwd: d in
+   * {24, 32, 64, 128}; bwd: d = 128); fp32 and the <= 16-token path return
+   * RM_ERR_UNSUPPORTED.  The values are read on the device: malformed
+   * boundaries give wrong results but no out-of-range access. */
+  const int32_t* cu_seqlens;
+  int num_segments;
+  const int32_t* seq_lens;
 } rm_attn_desc;
 
 /* ---- block level: one Q shard against one KV shard ---------------------- */

@@ -70,6 +70,63 @@ struct LayoutMap {
   }
 };
 
+// Segments of packed / right-padded batches (see rm_attn_desc).  range():
+// the [start, end) global positions of the segment holding position t of
+// batch entry b; a padding token gets the empty range start = t + 1, end = t.
+// query_span / key_span: the first and last global position a query may see /
+// that may see a key (last < first when there is none).  Every bound is
+// non-decreasing in t, so the bounds of a run of consecutive local rows are
+// those of its first and last row.
+struct Segs {
+  const int* cu;    // packing boundaries, or null
+  int nseg;
+  const int* lens;  // right padding lengths, or null
+  int64_t N;
+  __device__ __forceinline__ void range(int b, int64_t t, int64_t& start, int64_t& end) const {
+    if (cu) {
+      if (t >= cu[nseg]) {
+        start = t + 1;
+        end = t;
+        return;
+      }
+      int lo = 0, hi = nseg;  // cu[lo] <= t < cu[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cu[mid] <= t) lo = mid;
+        else hi = mid;
+      }
+      start = cu[lo];
+      end = cu[hi];
+    } else if (lens) {
+      const int64_t len = lens[b];
+      if (t < len) {
+        start = 0;
+        end = len;
+      } else {
+        start = t + 1;
+        end = t;
+      }
+    } else {
+      start = 0;
+      end = N;
+    }
+  }
+  __device__ __forceinline__ void query_span(int b, int64_t t, bool causal, int64_t& first,
+                                             int64_t& last) const {
+    int64_t a, e;
+    range(b, t, a, e);
+    first = a;
+    last = causal ? (t < e - 1 ? t : e - 1) : e - 1;
+  }
+  __device__ __forceinline__ void key_span(int b, int64_t u, bool causal, int64_t& first,
+                                           int64_t& last) const {
+    int64_t a, e;
+    range(b, u, a, e);
+    first = causal ? (u > a ? u : a) : a;
+    last = e - 1;
+  }
+};
+
 // Where the ring kernels find local row j of virtual rank r.  Rank-major
 // operands: memory row r * L + j, TMA coordinates (row j, shard r) of the
 // [B, P, L, H, d] view.  Global-order operands: memory row pos(r, j); TMA

@@ -74,6 +74,9 @@ struct AttnArgs {
   rm_tensor dq, dk, dv;  // bwd fp32 accumulators
   int accumulate;        // bwd: 1 = dq/dk/dv +=, 0 = written (=)
   int global_order;      // ring: operands (and lse / delta) in global token order
+  const int* cu_seqlens; // packing boundaries (device) or null
+  int num_segments;
+  const int* seq_lens;   // right-padding lengths (device) or null
   unsigned int* status;
 };
 // Forward.  q_rank < 0: all ranks (ring, rank-major operands, fused merge);

@@ -2,6 +2,7 @@
 // dispatch.  Every entry point validates on the host and returns before any
 // launch on a bad argument; no entry point allocates device memory.
 #include <math.h>
+#include <stdint.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -54,6 +55,7 @@ rm_status check_desc(const rm_attn_desc* d) {
   if (d->B < 0 || d->N < 0 || d->P < 1 || d->Hq < 1 || d->Hkv < 1)
     return fail(RM_ERR_INVALID_ARG, "bad sizes (B=%d N=%lld P=%d Hq=%d Hkv=%d)", d->B,
                 (long long)d->N, d->P, d->Hq, d->Hkv);
+  if (d->N > INT32_MAX) return fail(RM_ERR_INVALID_ARG, "N must be < 2^31");
   if (d->Hq % d->Hkv) return fail(RM_ERR_INVALID_ARG, "Hq %% Hkv != 0");
   if (d->layout != RM_LAYOUT_CONTIGUOUS && d->layout != RM_LAYOUT_ZIGZAG &&
       d->layout != RM_LAYOUT_STRIPED)
@@ -65,6 +67,12 @@ rm_status check_desc(const rm_attn_desc* d) {
     return fail(RM_ERR_INVALID_ARG, "bad ring mode");
   if (d->order != RM_ORDER_RANK_MAJOR && d->order != RM_ORDER_GLOBAL)
     return fail(RM_ERR_INVALID_ARG, "bad token order");
+  if (d->cu_seqlens && d->seq_lens)
+    return fail(RM_ERR_INVALID_ARG, "cu_seqlens and seq_lens are exclusive");
+  if (d->cu_seqlens && (d->num_segments < 1 || d->B != 1))
+    return fail(RM_ERR_INVALID_ARG, "packing needs num_segments >= 1 and B == 1");
+  if ((d->cu_seqlens || d->seq_lens) && d->dtype != RM_BF16)
+    return fail(RM_ERR_UNSUPPORTED, "packed / right-padded batches need bf16 (tensor-core path)");
   if (!(d->scale == d->scale) || isinf(d->scale)) return fail(RM_ERR_INVALID_ARG, "bad scale");
   if (d->dtype == RM_BF16) {
     if (!tc_supported_head_dim(d->d))
@@ -357,6 +365,9 @@ static AttnArgs attn_args(const rm_attn_desc* desc, int64_t lse_ld) {
   a.lse_ld = lse_ld;
   a.global_order = (desc->order == RM_ORDER_GLOBAL && desc->layout != RM_LAYOUT_CONTIGUOUS &&
                     desc->P > 1) ? 1 : 0;
+  a.cu_seqlens = desc->cu_seqlens;
+  a.num_segments = desc->cu_seqlens ? desc->num_segments : 0;
+  a.seq_lens = desc->seq_lens;
   a.status = status_word();
   return a;
 }
@@ -367,7 +378,7 @@ static rm_status block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm
                            int64_t lse_ld, cudaStream_t st) {
   AttnArgs a = attn_args(desc, lse_ld);
   a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = o_f32; a.lse = lse;
-  if (small_seq_supported(desc->N / desc->P, desc->d)) {
+  if (small_seq_supported(desc->N / desc->P, desc->d) && !desc->cu_seqlens && !desc->seq_lens) {
     RM_CUDA(launch_small_seq_fwd(a, q_rank, kv_rank, desc->dtype == RM_BF16, st),
             "short-sequence fwd launch");
     return RM_OK;
@@ -448,7 +459,8 @@ rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
     return fail(RM_ERR_UNSUPPORTED, "stepwise mode supports P <= %d", kMaxMergeParts);
   cudaStream_t st = (cudaStream_t)stream;
   const int64_t L = desc->N / desc->P;
-  if (desc->mode == RM_RING_FUSED && desc->P == 1 && small_seq_supported(desc->N, desc->d))
+  if (desc->mode == RM_RING_FUSED && desc->P == 1 && small_seq_supported(desc->N, desc->d) &&
+      !desc->cu_seqlens && !desc->seq_lens)
     return block_fwd(desc, 0, 0, q, k, v, o, desc->dtype == RM_F32, lse, desc->N, st);
   if (desc->mode == RM_RING_FUSED) {
     AttnArgs a = attn_args(desc, desc->N);
@@ -565,6 +577,8 @@ namespace {
 rm_status usp_desc(const rm_attn_desc* desc, int u, rm_attn_desc* out) {
   RM_TRY(check_desc(desc));
   if (u < 1) return fail(RM_ERR_INVALID_ARG, "ulysses degree must be >= 1");
+  if (desc->cu_seqlens || desc->seq_lens)
+    return fail(RM_ERR_UNSUPPORTED, "USP with packed / right-padded batches is not supported");
   if (desc->Hq % u || desc->Hkv % u)
     return fail(RM_ERR_INVALID_ARG, "ulysses degree %d must divide Hq (%d) and Hkv (%d)", u,
                 desc->Hq, desc->Hkv);

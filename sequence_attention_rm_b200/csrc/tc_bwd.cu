@@ -58,6 +58,9 @@ struct BwdParams {
   int accumulate;
   int head_block;    // heads per grid block (see grid_place)
   int global_order;  // ring operands, outputs, LSE and D in global token order
+  const int* cu_seqlens;  // packing boundaries (device) or null
+  int num_segments;
+  const int* seq_lens;    // right-padding lengths (device) or null
   unsigned int* status;
   long long wait_limit;
 };
@@ -182,36 +185,44 @@ __device__ __forceinline__ uint32_t p_col(int k) { return kHalf * (k >> 2) + 8 *
 __device__ __forceinline__ uint32_t ds_col(int k) { return p_col(k) + 32; }
 
 // The CTA's walk: for every query head of the group, every rank in
-// reverse-ring order, the query tiles that can see key i0.
+// reverse-ring order, the query tiles that can see a key of the CTA: the
+// queries at global positions [span_first, span_last].
 struct Walk {
   LayoutMap lay;
   int s, g, group, nranks, qtiles, ring, q_rank, P, causal;
-  int64_t tk_first;
+  int64_t span_first, span_last;
   __device__ __forceinline__ int rank_of(int step) const {
     return ring ? (s + step) % P : q_rank;
   }
-  // first query tile of rank r that can see key i0 (later tiles all can)
+  // query tiles [first_tile(r), end_tile(r)) of rank r
   __device__ __forceinline__ int first_tile(int r) const {
-    if (!causal) return 0;
-    return (int)(lay.visible_count(r, tk_first - 1) / BQ);  // queries with pos < tk_first
+    return (int)(lay.visible_count(r, span_first - 1) / BQ);
+  }
+  __device__ __forceinline__ int end_tile(int r) const {
+    return (int)((lay.visible_count(r, span_last) + BQ - 1) / BQ);
   }
   __device__ __forceinline__ int count() const {
     int n = 0;
-    for (int step = 0; step < nranks; ++step) n += qtiles - first_tile(rank_of(step));
+    for (int step = 0; step < nranks; ++step) {
+      const int r = rank_of(step);
+      n += max(0, end_tile(r) - first_tile(r));
+    }
     return n * group;
   }
-  // A position in the walk, advanced one tile at a time (no rescans).
+  // A position in the walk, advanced one tile at a time (no rescans); end is
+  // end_tile(r) of the current rank, computed when the rank changes.
   struct Cursor {
-    int hh, step, r, t;
+    int hh, step, r, t, end;
   };
   __device__ __forceinline__ void settle(Cursor& c) const {
-    while (c.t >= qtiles && c.hh < group) {
+    while (c.t >= c.end && c.hh < group) {
       if (++c.step == nranks) {
         c.step = 0;
         ++c.hh;
       }
       c.r = rank_of(c.step);
       c.t = first_tile(c.r);
+      c.end = end_tile(c.r);
     }
   }
   __device__ __forceinline__ Cursor begin() const {
@@ -220,6 +231,7 @@ struct Walk {
     c.step = 0;
     c.r = rank_of(0);
     c.t = first_tile(c.r);
+    c.end = end_tile(c.r);
     settle(c);
     return c;
   }
@@ -298,7 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   W.P = p.P;
   W.causal = p.causal;
   const int64_t i0 = (int64_t)xt * BK;  // first key (local index in shard s)
-  W.tk_first = W.lay.pos(W.s, i0);
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  {  // queries that may see a key of the CTA (the bounds are monotone in the key)
+    int64_t f, l;
+    sg.key_span(b, W.lay.pos(W.s, i0), p.causal, W.span_first, l);
+    sg.key_span(b, W.lay.pos(W.s, LayoutMap::min64(i0 + BK - 1, L - 1)), p.causal, f, W.span_last);
+  }
   const int s = W.s, g = W.g;
   const long long limit = p.wait_limit;
   const BwdRows R = bwd_rows(p);
@@ -443,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int krow = lane_base + lane;       // key row of the tile (TMEM lane)
     const int64_t key = i0 + krow;
     const bool key_live = key < L;
-    const int64_t tk = key_live ? W.lay.pos(s, key) : 0;
-    // queries of rank r with position < tk cannot see this key
+    // local queries [span_lo, span_hi) of rank span_rank see this key
+    int span_rank = -1, span_lo = 0, span_hi = 0;
     const int tid = threadIdx.x & 127;
     const uint32_t cS = kTS + kHalf * X, cdP = kTdP + kHalf * X;
     bool ok = true;
@@ -467,11 +484,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar_vec + X * 2 + y);
       next = fetch(ahead, i + 1);  // in flight during this tile
       const int r = cur.r, t = cur.t;
-      const int64_t j0 = (int64_t)t * BQ + kHalf * X;
+      if (r != span_rank) {  // recomputed per rank rather than held across the walk
+        span_rank = r;
+        span_lo = span_hi = 0;
+        if (key_live) {
+          int64_t f, l;  // global positions of the queries that see this key
+          sg.key_span(b, W.lay.pos(s, key), p.causal, f, l);
+          span_lo = (int)W.lay.visible_count(r, f - 1);
+          span_hi = (int)W.lay.visible_count(r, l);
+        }
+      }
       // visible query columns [lo, hi) of this key in this warpgroup's half
-      const int64_t hidden = !p.causal ? 0 : (key_live ? W.lay.visible_count(r, tk - 1) : L);
-      const int lo = (int)LayoutMap::clamp64(hidden - j0, 0, kHalf);
-      const int hi = key_live ? (int)LayoutMap::clamp64(L - j0, 0, kHalf) : 0;
+      const int j0 = t * BQ + kHalf * X;
+      const int lo = min(max(span_lo - j0, 0), kHalf);
+      const int hi = min(max(span_hi - j0, 0), kHalf);
       const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kHalf);
       W.next(cur);
       W.next(ahead);
@@ -672,13 +698,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = h / (p.Hq / p.Hkv);
   const int64_t last_row = LayoutMap::min64(row0 + BM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  // global span of the keys any row of the CTA may see (the bounds are
+  // monotone in the row, so its first and last rows give them)
+  int64_t span_first, span_last;
+  {
+    int64_t f, l;
+    sg.query_span(b, lay.pos(r, LayoutMap::min64(row0, L - 1)), p.causal, span_first, l);
+    sg.query_span(b, t_last, p.causal, f, span_last);
+  }
   const int nsteps = p.ring ? p.P : 1;
   const long long limit = p.wait_limit;
   const BwdRows R = bwd_rows(p);
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
-  auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
+  // key tiles [tile_begin(s), tile_end(s)) of shard s hold every key the CTA may see
+  auto tile_begin = [&](int s) -> int { return (int)(lay.visible_count(s, span_first - 1) / BN); };
+  auto tile_end = [&](int s) -> int {
+    return (int)((lay.visible_count(s, span_last) + BN - 1) / BN);
+  };
   int n = 0;  // key tiles of the whole walk
-  for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + BN - 1) / BN);
+  for (int step = 0; step < nsteps; ++step) {
+    const int s = shard_of(step);
+    n += max(0, tile_end(s) - tile_begin(s));
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -724,8 +766,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int s = shard_of(step);
-        const int nt = (int)((cta_keys(s) + BN - 1) / BN);
-        for (int t = 0; t < nt; ++t) {
+        const int te = tile_end(s);
+        for (int t = tile_begin(s); t < te; ++t) {
           const int sk = nk % kKStages, sv = nv % kVStages;
           int kr, ks;
           R.tma(s, (int64_t)t * BN, kr, ks);
@@ -826,13 +868,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int step = 0; step < nsteps && ok; ++step) {
       const int s = shard_of(step);
-      const int nt = (int)((cta_keys(s) + BN - 1) / BN);
-      const int64_t row_keys = !live ? 0 : (p.causal ? lay.visible_count(s, tq) : L);
-      for (int t = 0; t < nt; ++t, ++j) {
+      const int te = tile_end(s);
+      // keys [row_lo, row_hi) of shard s are visible to this row
+      int64_t row_lo = 0, row_hi = 0;
+      if (live) {
+        int64_t f, l;
+        sg.query_span(b, tq, p.causal, f, l);
+        row_lo = lay.visible_count(s, f - 1);
+        row_hi = lay.visible_count(s, l);
+      }
+      for (int t = tile_begin(s); t < te; ++t, ++j) {
         const uint32_t cS = kTS + (j & 1) * BN + kHalf * X, cdP = kTdP + kHalf * X;
-        // visible keys of this warpgroup's half: [0, nvalid)
-        const int64_t nvalid = row_keys - (int64_t)t * BN - kHalf * X;
-        const bool full = __all_sync(0xffffffffu, nvalid >= kHalf);
+        // visible keys of this warpgroup's half: [c_lo, c_hi)
+        const int64_t c0 = (int64_t)t * BN + kHalf * X;
+        const int64_t c_lo = row_lo - c0, c_hi = row_hi - c0;
+        const bool full = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kHalf);
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, limit, p.status))) {
           ok = false;
           break;
@@ -855,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!full) {
 #pragma unroll
-          for (int col = 0; col < kHalf; ++col) pt[col] = col < nvalid ? pt[col] : 0.f;
+          for (int col = 0; col < kHalf; ++col) pt[col] = (col >= c_lo && col < c_hi) ? pt[col] : 0.f;
         }
         if (!__all_sync(0xffffffffu, mbar_wait(bar_dp_full, j & 1, limit, p.status))) {
           ok = false;
@@ -946,6 +996,9 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.dv_sh = a.dv.stride_h;
   p.accumulate = a.accumulate;
   p.global_order = ring ? a.global_order : 0;
+  p.cu_seqlens = a.cu_seqlens;
+  p.num_segments = a.num_segments;
+  p.seq_lens = a.seq_lens;
   const int view = operand_view(a, ring);
   p.status = a.status;
   p.wait_limit = tc_wait_limit();

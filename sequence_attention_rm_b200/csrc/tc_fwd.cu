@@ -78,6 +78,9 @@ struct FwdParams {
   int head_pairs;
   int head_block;  // head units per grid block (see grid_place)
   int global_order;  // ring operands, O and LSE in global token order
+  const int* cu_seqlens;  // packing boundaries (device) or null
+  int num_segments;
+  const int* seq_lens;    // right-padding lengths (device) or null
   void* o;
   int64_t o_sb, o_sn, o_sh;
   int o_f32;
@@ -182,6 +185,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   const int64_t last_row = min((p.head_pairs ? rowA : rowB) + kBM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  // global span of the keys any row of the CTA may see (bounds are monotone
+  // in the row, so its first and last rows give them)
+  int64_t span_first, span_last;
+  {
+    int64_t f, l;
+    sg.query_span(b, lay.pos(r, min(rowA, L - 1)), p.causal, span_first, l);
+    sg.query_span(b, t_last, p.causal, f, span_last);
+  }
   const int nsteps = p.ring ? p.P : 1;
   const long long limit = p.wait_limit;
 
@@ -211,7 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // KV shard of ring step `step`, and how many of its keys the CTA may see.
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
-  auto cta_keys = [&](int s) -> int64_t { return p.causal ? lay.visible_count(s, t_last) : L; };
+  // key tiles [tile_begin(s), tile_end(s)) of shard s hold every key the CTA may see
+  auto tile_begin = [&](int s) -> int { return (int)(lay.visible_count(s, span_first - 1) / kBN); };
+  auto tile_end = [&](int s) -> int {
+    return (int)((lay.visible_count(s, span_last) + kBN - 1) / kBN);
+  };
 
   if (warp >= 8) {
     regs_dec<kRegsOther>();
@@ -233,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int s = shard_of(step);
-        const int nt = (int)((cta_keys(s) + kBN - 1) / kBN);
-        for (int t = 0; t < nt; ++t, ++j) {
+        const int te = tile_end(s);
+        for (int t = tile_begin(s); t < te; ++t, ++j) {
           const int st = j & 1;
           int kr, ks;
           tma_rs(s, (int64_t)t * kBN, kr, ks);
@@ -268,7 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q0 = smem_u32(smem + C::kQ0), q1 = smem_u32(smem + C::kQ1);
       const uint32_t kbase = smem_u32(smem + C::kK), vbase = smem_u32(smem + C::kV);
       int n = 0;
-      for (int step = 0; step < nsteps; ++step) n += (int)((cta_keys(shard_of(step)) + kBN - 1) / kBN);
+      for (int step = 0; step < nsteps; ++step) {
+        const int s = shard_of(step);
+        n += max(0, tile_end(s) - tile_begin(s));
+      }
       auto issue_s = [&](uint32_t qaddr, uint32_t scol, int st) {
         const uint32_t kaddr = kbase + st * C::kTileBytes;
 #pragma unroll
@@ -340,9 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int step = 0; step < nsteps && ok; ++step) {
       const int s = shard_of(step);
-      const int nt = (int)((cta_keys(s) + kBN - 1) / kBN);
-      const int64_t row_keys = !live ? 0 : (p.causal ? lay.visible_count(s, tq) : L);
-      for (int t = 0; t < nt; ++t, ++j) {
+      const int te = tile_end(s);
+      // keys [row_lo, row_hi) of shard s are visible to this row
+      int64_t row_lo = 0, row_hi = 0;
+      if (live) {
+        int64_t f, l;
+        sg.query_span(b, tq, p.causal, f, l);
+        row_lo = lay.visible_count(s, f - 1);
+        row_hi = lay.visible_count(s, l);
+      }
+      for (int t = tile_begin(s); t < te; ++t, ++j) {
         // all lanes leave together, so the warp-collective tcgen05.ld / st
         // below always run converged
         if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, limit, p.status))) {
@@ -359,11 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) sc[c * 32 + i] = __uint_as_float(v[i]);
         }
         tmem_wait_ld();
-        const int64_t nvalid = row_keys - (int64_t)t * kBN;
-        if (nvalid < kBN) {
+        const int64_t c_lo = row_lo - (int64_t)t * kBN, c_hi = row_hi - (int64_t)t * kBN;
+        if (c_lo > 0 || c_hi < kBN) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if (c >= nvalid) sc[c] = -INFINITY;
+            if (c < c_lo || c >= c_hi) sc[c] = -INFINITY;
         }
         // row max: 8 independent chains of three-input max (a single two-input
         // chain is 128 dependent steps)
@@ -598,6 +624,9 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   p.kv_rank = kv_rank;
   p.head_pairs = ((a.Hq / a.Hkv) % 2 == 0) ? 1 : 0;
   p.global_order = ring ? a.global_order : 0;
+  p.cu_seqlens = a.cu_seqlens;
+  p.num_segments = a.num_segments;
+  p.seq_lens = a.seq_lens;
   p.o = a.o.ptr;
   p.o_sb = a.o.stride_b;
   p.o_sn = a.o.stride_n;

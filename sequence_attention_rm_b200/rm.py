@@ -44,7 +44,9 @@ class RmAttnDesc(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("Hq", ctypes.c_int),
                 ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("N", ctypes.c_int64),
                 ("P", ctypes.c_int), ("layout", ctypes.c_int), ("causal", ctypes.c_int),
-                ("scale", ctypes.c_float), ("mode", ctypes.c_int), ("order", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("mode", ctypes.c_int), ("order", ctypes.c_int),
+                ("cu_seqlens", ctypes.c_void_p), ("num_segments", ctypes.c_int),
+                ("seq_lens", ctypes.c_void_p)]
 
 
 class RmError(RuntimeError):
@@ -129,11 +131,25 @@ def _bnhd(t: torch.Tensor) -> RmTensor:
     return RmTensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
 
 
+def _segs(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("cu_seqlens / seq_lens must be contiguous CUDA int32 tensors")
+    return t.data_ptr()
+
+
 def desc(dtype: torch.dtype, B: int, Hq: int, Hkv: int, d: int, N: int, P: int, layout: str,
-         causal: bool, scale: float | None = None, mode: str = "fused",
-         order: str = "rank") -> RmAttnDesc:
+         causal: bool, scale: float | None = None, mode: str = "fused", order: str = "rank",
+         cu_seqlens: torch.Tensor | None = None, seq_lens: torch.Tensor | None = None
+         ) -> RmAttnDesc:
+    """cu_seqlens: packing boundaries (global positions, int32 on the device,
+    B == 1); seq_lens: right-padding lengths per batch entry (int32 on the
+    device).  The tensors must outlive the asynchronous calls that use them."""
     return RmAttnDesc(_dtype_code(dtype), B, Hq, Hkv, d, N, P, LAYOUTS[layout], int(bool(causal)),
-                      0.0 if scale is None else float(scale), MODES[mode], ORDERS[order])
+                      0.0 if scale is None else float(scale), MODES[mode], ORDERS[order],
+                      _segs(cu_seqlens), 0 if cu_seqlens is None else cu_seqlens.numel() - 1,
+                      _segs(seq_lens))
 
 
 # ---- entry points -----------------------------------------------------------
@@ -232,13 +248,14 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None):
 
 
 def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | None = None,
-                  mode: str = "fused", order: str = "rank", out=None, lse=None, ws=None,
-                  stream=None):
+                  mode: str = "fused", order: str = "rank", cu_seqlens=None, seq_lens=None,
+                  out=None, lse=None, ws=None, stream=None):
     """Ring forward over P virtual ranks; q/k/v [B, N, H, d] in `order` ("rank":
     rank-major, "global": the tokens' own order) -> (O, LSE [B, Hq, N]) in the
     same order."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order,
+               cu_seqlens, seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
     wp, wn = _workspace(ring_workspace_size(dsc, False), q.device, ws)
@@ -248,11 +265,12 @@ def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | 
 
 
 def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
-                  scale: float | None = None, order: str = "rank", dq=None, dk=None, dv=None,
-                  ws=None, stream=None):
+                  scale: float | None = None, order: str = "rank", cu_seqlens=None,
+                  seq_lens=None, dq=None, dk=None, dv=None, ws=None, stream=None):
     """Ring backward; returns (dq, dk, dv) in the input dtype and in `order`."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv

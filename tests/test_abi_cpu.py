@@ -64,6 +64,12 @@ def _desc(rm, **kw):
     (dict(order=1, N=2000, P=2), 2),         # global zigzag: chunk of 500 tokens
     (dict(order=1, dtype=0), 2),             # global order needs bf16
     (dict(order=1, mode=1), 2),              # global order needs the fused forward
+    (dict(N=1 << 31), 1),                    # positions are 32-bit on the device
+    # segments (the pointers are never read by the validation)
+    (dict(cu_seqlens=16, num_segments=2, seq_lens=16), 1),  # exclusive
+    (dict(cu_seqlens=16, num_segments=2, B=2), 1),          # packing needs B == 1
+    (dict(cu_seqlens=16, num_segments=0), 1),
+    (dict(seq_lens=16, dtype=0), 2),                        # fp32: no segments
 ])
 def test_desc_validation(rm, bad, status):
     n = ctypes.c_size_t(0)
@@ -142,7 +148,8 @@ def test_usp_auto_select_matches_the_rule(rm):
 
 
 @pytest.mark.parametrize("kw,u", [(dict(), 3), (dict(), 16), (dict(N=16386, P=2), 4),
-                                  (dict(Hq=12, Hkv=6), 4)])
+                                  (dict(Hq=12, Hkv=6), 4),
+                                  (dict(seq_lens=16), 2)])  # no segments under USP
 def test_usp_validation(rm, kw, u):
     n = ctypes.c_size_t(0)
     d = _desc(rm, **kw)
