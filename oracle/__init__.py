@@ -11,7 +11,7 @@ arithmetic.
 Everything here is written to be checked by eye against the pages it cites:
 - "Mosaic: Sharding Attention Across GPUs When Your Sequence Doesn't Fit"
   (dev.to, P. Sateesh), sections "The Problem", "How Ring Attention Works",
-  "The Implementation";
+  "The Implementation", "Beyond 1D: Mesh2D Attention";
 - "ringmaster" (PyPI page of axolotl-ringmaster 0.2.0), sections "Why",
   "Status", "Layout";
 - "Ring Attention & Friends" (slide deck), slides "Vanilla Transformer",
@@ -32,10 +32,11 @@ Modules:
 - ``repack``     Ulysses sequence<->head repack as explicit index loops
 - ``multiaxis``  row-axis / feature-axis routing of a tabular tensor
 - ``usp``        Ulysses x ring composition (USP) and its degree selection
+- ``mesh2d``     Mesh2D: tiles of a (query chunk x key chunk) grid, merged
 
 Parity status: every function above is pinned by ``tests/test_oracle_*.py``
 (closed forms, brute force, invariants, finite differences, a library
 cross-check); none is "parity unpinned".
 """
 
-from . import attention, layouts, merge, multiaxis, repack, ring, usp  # noqa: F401
+from . import attention, layouts, merge, mesh2d, multiaxis, repack, ring, usp  # noqa: F401
