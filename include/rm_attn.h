@@ -278,6 +278,38 @@ rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
                           rm_tensor dq, rm_tensor dk, rm_tensor dv, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* ---- Mesh2D ---------------------------------------------------------------
+ * [Mosaic, "Beyond 1D: Mesh2D Attention": both Q and K are sharded; on a
+ * grid of devices, device (i, j) computes the tile of QK^T between query
+ * chunk i and key chunk j.]  Here the grid_q x grid_k tiles run in turn on
+ * one GPU.  Query chunk i = global positions [i*N/grid_q, (i+1)*N/grid_q),
+ * key / value chunk j = [j*N/grid_k, (j+1)*N/grid_k) (contiguous; the grid
+ * may be rectangular).  Tile (i, j) is the block forward of that pair
+ * (rm_attn_block_fwd with its own chunk lengths): an fp32 partial O and its
+ * LSE.  The forward merges the partials of each query chunk with the LSE
+ * merge (rm_lse_merge); the backward adds every tile's contributions, from
+ * the final LSE and D = rowsum(dO o O), into dQ of chunk i and dK / dV of
+ * chunk j (fp32 accumulators, then the output dtype, RNE for bf16).  Tiles
+ * without a visible pair under the causal rule are skipped.
+ *
+ * desc: dtype, B, Hq, Hkv, d, N, causal, scale as for the ring; P, layout,
+ * mode and order are ignored (operands in global token order); no segments
+ * (RM_ERR_UNSUPPORTED).  grid_q, grid_k >= 1 must divide N; grid_k <= 16
+ * (RM_ERR_UNSUPPORTED above).  The bf16 backward needs d = 128.
+ * q/o/dout/dq [B, N, Hq, d], k/v/dk/dv [B, N, Hkv, d] strided as rm_tensor;
+ * lse fp32 [B, Hq, N].  Workspace (caller-owned, 256-byte aligned):
+ * forward grid_k fp32 partial O [B, N, Hq, d] and LSE [B, Hq, N] slots;
+ * backward delta [B, Hq, N] and fp32 dQ / dK / dV accumulators. */
+rm_status rm_mesh2d_workspace_size(const rm_attn_desc* desc, int grid_q, int grid_k,
+                                   int backward, size_t* bytes);
+rm_status rm_mesh2d_attn_fwd(const rm_attn_desc* desc, int grid_q, int grid_k, rm_tensor q,
+                             rm_tensor k, rm_tensor v, rm_tensor o, float* lse, void* ws,
+                             size_t ws_bytes, void* stream);
+rm_status rm_mesh2d_attn_bwd(const rm_attn_desc* desc, int grid_q, int grid_k, rm_tensor q,
+                             rm_tensor k, rm_tensor v, rm_tensor o, const float* lse,
+                             rm_tensor dout, rm_tensor dq, rm_tensor dk, rm_tensor dv, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* ---- bit-exact layout transforms ---------------------------------------- */
 
 /* Global token order <-> rank-major order (see pos(r, j) above) of a dense

@@ -183,6 +183,28 @@ __host__ __device__ inline LayoutMap make_layout(int layout, int64_t N, int P) {
   return m;
 }
 
+// Key side of a (query shard, KV shard) call: the layout's own shards, or,
+// for one tile of a rectangular grid (Pk != P, contiguous layout), contiguous
+// chunks of N / Pk keys.
+struct KeyShards {
+  LayoutMap lay;  // equal shards
+  int chunked;    // 1: chunks of L keys
+  int64_t L;      // keys per shard
+  __host__ __device__ __forceinline__ int64_t pos(int s, int64_t i) const {
+    return chunked ? (int64_t)s * L + i : lay.pos(s, i);
+  }
+  __host__ __device__ __forceinline__ int64_t visible_count(int s, int64_t t) const {
+    return chunked ? LayoutMap::clamp64(t - (int64_t)s * L + 1, 0, L) : lay.visible_count(s, t);
+  }
+};
+__host__ __device__ inline KeyShards key_shards(const LayoutMap& lay, int64_t N, int Pk) {
+  KeyShards k;
+  k.lay = lay;
+  k.chunked = Pk != lay.P;
+  k.L = N / Pk;
+  return k;
+}
+
 // ---- device status word (bounded-wait expiry) ------------------------------
 enum : uint32_t { kStatusTimeout = 1u, kStatusSmemAlign = 2u };
 

@@ -62,6 +62,7 @@ struct AttnArgs {
   int B, Hq, Hkv, d;
   int64_t N;
   int P, layout, causal;
+  int Pk;                // block calls: KV chunks of a rectangular grid (0: P)
   float scale;
   rm_tensor q, k, v;     // bases of the q / kv operands (see launchers)
   rm_tensor o;           // fwd output
@@ -79,6 +80,8 @@ struct AttnArgs {
   const int* seq_lens;   // right-padding lengths (device) or null
   unsigned int* status;
 };
+__host__ __device__ inline int kv_shards(const AttnArgs& a) { return a.Pk > 0 ? a.Pk : a.P; }
+
 // Forward.  q_rank < 0: all ranks (ring, rank-major operands, fused merge);
 // else one (q_rank, kv_rank) pair with shard-local operands.
 cudaError_t launch_simt_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);

@@ -373,12 +373,15 @@ static AttnArgs attn_args(const rm_attn_desc* desc, int64_t lse_ld) {
 }
 
 // One (q_rank, kv_rank) forward with shard-local operands; LSE rows lse_ld apart.
+// Pk > 0: the KV side has Pk contiguous chunks (a tile of a rectangular grid).
 static rm_status block_fwd(const rm_attn_desc* desc, int q_rank, int kv_rank, rm_tensor q,
                            rm_tensor k, rm_tensor v, rm_tensor o, int o_f32, float* lse,
-                           int64_t lse_ld, cudaStream_t st) {
+                           int64_t lse_ld, cudaStream_t st, int Pk = 0) {
   AttnArgs a = attn_args(desc, lse_ld);
   a.q = q; a.k = k; a.v = v; a.o = o; a.o_f32 = o_f32; a.lse = lse;
-  if (small_seq_supported(desc->N / desc->P, desc->d) && !desc->cu_seqlens && !desc->seq_lens) {
+  a.Pk = Pk;
+  if (small_seq_supported(desc->N / desc->P, desc->d) && !desc->cu_seqlens && !desc->seq_lens &&
+      kv_shards(a) == desc->P) {
     RM_CUDA(launch_small_seq_fwd(a, q_rank, kv_rank, desc->dtype == RM_BF16, st),
             "short-sequence fwd launch");
     return RM_OK;
@@ -715,6 +718,186 @@ rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
   RM_TRY(usp_repack(desc, u, hq, 1, ydq, dq.ptr, st));
   RM_TRY(usp_repack(desc, u, hkv, 1, ydk, dk.ptr, st));
   return usp_repack(desc, u, hkv, 1, ydv, dv.ptr, st);
+}
+
+// ---- Mesh2D ---------------------------------------------------------------
+
+namespace {
+
+// The tile problem of a Mesh2D call: query chunks are the P = grid_q
+// contiguous shards of the block API, KV chunks its Pk = grid_k ones.
+rm_status mesh2d_desc(const rm_attn_desc* desc, int grid_q, int grid_k, rm_attn_desc* out) {
+  if (!desc) return fail(RM_ERR_INVALID_ARG, "desc is NULL");
+  if (grid_q < 1 || grid_k < 1) return fail(RM_ERR_INVALID_ARG, "grid sizes must be >= 1");
+  if (grid_k > kMaxMergeParts)
+    return fail(RM_ERR_UNSUPPORTED, "grid_k must be <= %d (merge parts)", kMaxMergeParts);
+  if (desc->N % grid_q) return fail(RM_ERR_INVALID_ARG, "grid_q must divide N");
+  *out = *desc;
+  out->P = grid_q;
+  out->layout = RM_LAYOUT_CONTIGUOUS;
+  out->mode = RM_RING_STEPWISE;
+  out->order = RM_ORDER_RANK_MAJOR;
+  RM_TRY(check_desc(out));
+  if (desc->N % grid_k) return fail(RM_ERR_INVALID_ARG, "grid_k must divide N");
+  if (desc->cu_seqlens || desc->seq_lens)
+    return fail(RM_ERR_UNSUPPORTED, "Mesh2D with packed / right-padded batches is not supported");
+  return RM_OK;
+}
+
+struct MeshWs {
+  size_t o_parts, lse_parts;    // forward: grid_k fp32 partial O and LSE slots
+  size_t delta, dq, dk, dv;     // backward: delta and fp32 accumulators
+  size_t total;
+};
+MeshWs mesh2d_ws(const rm_attn_desc* d, int grid_k, int backward) {
+  MeshWs w;
+  memset(&w, 0, sizeof(w));
+  const size_t rows_q = (size_t)d->B * d->N * d->Hq, rows_kv = (size_t)d->B * d->N * d->Hkv;
+  if (!backward) {
+    w.lse_parts = align_up(rows_q * d->d * 4 * (size_t)grid_k);
+    w.total = w.lse_parts + align_up(rows_q * 4 * (size_t)grid_k);
+  } else {
+    w.dq = align_up(rows_q * 4);
+    w.dk = w.dq + align_up(rows_q * d->d * 4);
+    w.dv = w.dk + align_up(rows_kv * d->d * 4);
+    w.total = w.dv + align_up(rows_kv * d->d * 4);
+  }
+  return w;
+}
+
+// Whether tile (i, j) holds a visible pair: under the causal rule the first
+// key of chunk j must not lie after the last query of chunk i.
+bool mesh2d_tile_live(const rm_attn_desc* d, int grid_q, int grid_k, int i, int j) {
+  if (!d->causal) return true;
+  return (int64_t)j * (d->N / grid_k) <= (int64_t)(i + 1) * (d->N / grid_q) - 1;
+}
+
+}  // namespace
+
+rm_status rm_mesh2d_workspace_size(const rm_attn_desc* desc, int grid_q, int grid_k,
+                                   int backward, size_t* bytes) {
+  rm_attn_desc d2;
+  RM_TRY(mesh2d_desc(desc, grid_q, grid_k, &d2));
+  if (!bytes) return fail(RM_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = mesh2d_ws(&d2, grid_k, backward).total;
+  return RM_OK;
+}
+
+rm_status rm_mesh2d_attn_fwd(const rm_attn_desc* desc, int grid_q, int grid_k, rm_tensor q,
+                             rm_tensor k, rm_tensor v, rm_tensor o, float* lse, void* ws,
+                             size_t ws_bytes, void* stream) {
+  rm_attn_desc d2;
+  RM_TRY(mesh2d_desc(desc, grid_q, grid_k, &d2));
+  if (d2.B == 0 || d2.N == 0) return RM_OK;
+  RM_TRY(check_qkv(&d2, d2.N, q, k, v));
+  const int es = esize_of(d2.dtype);
+  RM_TRY(check_tensor("o", o, es, (int64_t)d2.B * d2.N, d2.Hq, d2.d));
+  if (!lse || ((uintptr_t)lse & 3)) return fail(RM_ERR_INVALID_ARG, "lse NULL/misaligned");
+  const MeshWs w = mesh2d_ws(&d2, grid_k, 0);
+  if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t Lq = d2.N / grid_q, Lk = d2.N / grid_k;
+  const size_t rows_q = (size_t)d2.B * d2.N * d2.Hq;
+  float* o_slots = (float*)((char*)ws + w.o_parts);
+  float* lse_slots = (float*)((char*)ws + w.lse_parts);
+  for (int i = 0; i < grid_q; ++i) {
+    // tile (i, j): partial O into rows of chunk i of slot j, its LSE likewise
+    int parts = 0;
+    for (int j = 0; j < grid_k && mesh2d_tile_live(&d2, grid_q, grid_k, i, j); ++j, ++parts) {
+      rm_tensor o_j = dense_bnhd(o_slots + (size_t)j * rows_q * d2.d, d2.N, d2.Hq, d2.d);
+      RM_TRY(block_fwd(&d2, i, j, offset_rows(q, i * Lq, es), offset_rows(k, j * Lk, es),
+                       offset_rows(v, j * Lk, es), offset_rows(o_j, i * Lq, 4), 1,
+                       lse_slots + (size_t)j * rows_q + i * Lq, d2.N, st, grid_k));
+    }
+    // the live tiles of a row are a prefix j < parts (parts >= 1: key 0 sees every query)
+    MergeArgs m;
+    memset(&m, 0, sizeof(m));
+    m.B = d2.B;
+    m.H = d2.Hq;
+    m.d = d2.d;
+    m.Nq = Lq;
+    m.n_parts = parts;
+    m.lse_ld = d2.N;
+    for (int j = 0; j < parts; ++j) {
+      m.o_ptr[j] = o_slots + (size_t)j * rows_q * d2.d + (size_t)i * Lq * d2.Hq * d2.d;
+      m.o_sb[j] = d2.N * d2.Hq * d2.d;
+      m.o_sn[j] = (int64_t)d2.Hq * d2.d;
+      m.o_sh[j] = d2.d;
+      m.lse_ptr[j] = lse_slots + (size_t)j * rows_q + i * Lq;
+    }
+    const rm_tensor o_i = offset_rows(o, i * Lq, es);
+    m.out = o_i.ptr;
+    m.out_sb = o.stride_b;
+    m.out_sn = o.stride_n;
+    m.out_sh = o.stride_h;
+    m.lse_out = lse + i * Lq;
+    RM_CUDA(launch_lse_merge(m, d2.dtype == RM_BF16, st), "Mesh2D merge launch");
+  }
+  return RM_OK;
+}
+
+rm_status rm_mesh2d_attn_bwd(const rm_attn_desc* desc, int grid_q, int grid_k, rm_tensor q,
+                             rm_tensor k, rm_tensor v, rm_tensor o, const float* lse,
+                             rm_tensor dout, rm_tensor dq, rm_tensor dk, rm_tensor dv, void* ws,
+                             size_t ws_bytes, void* stream) {
+  rm_attn_desc d2;
+  RM_TRY(mesh2d_desc(desc, grid_q, grid_k, &d2));
+  if (d2.B == 0 || d2.N == 0) return RM_OK;
+  RM_TRY(check_qkv(&d2, d2.N, q, k, v));
+  const int es = esize_of(d2.dtype);
+  const int64_t rows = (int64_t)d2.B * d2.N;
+  RM_TRY(check_tensor("o", o, es, rows, d2.Hq, d2.d));
+  RM_TRY(check_tensor("dout", dout, es, rows, d2.Hq, d2.d));
+  RM_TRY(check_tensor("dq", dq, es, rows, d2.Hq, d2.d));
+  RM_TRY(check_tensor("dk", dk, es, rows, d2.Hkv, d2.d));
+  RM_TRY(check_tensor("dv", dv, es, rows, d2.Hkv, d2.d));
+  if (!lse) return fail(RM_ERR_INVALID_ARG, "lse NULL");
+  if (d2.dtype == RM_BF16 && d2.d != 128)
+    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", d2.d);
+  const MeshWs w = mesh2d_ws(&d2, grid_k, 1);
+  if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
+    return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = (char*)ws;
+  float* delta = (float*)(base + w.delta);
+  const rm_tensor dq_acc = dense_bnhd(base + w.dq, d2.N, d2.Hq, d2.d);
+  const rm_tensor dk_acc = dense_bnhd(base + w.dk, d2.N, d2.Hkv, d2.d);
+  const rm_tensor dv_acc = dense_bnhd(base + w.dv, d2.N, d2.Hkv, d2.d);
+  const size_t kv_bytes = (size_t)rows * d2.Hkv * d2.d * 4;
+  // delta from the final O (and the dQ accumulator zeroed in the same pass)
+  RM_CUDA(launch_bwd_preprocess(d2.dtype == RM_BF16, d2.B, d2.N, d2.Hq, d2.d, o, dout, delta,
+                                (float*)dq_acc.ptr, st),
+          "bwd preprocess launch");
+  RM_CUDA(cudaMemsetAsync(dk_acc.ptr, 0, kv_bytes, st), "dK accumulator clear");
+  RM_CUDA(cudaMemsetAsync(dv_acc.ptr, 0, kv_bytes, st), "dV accumulator clear");
+  const int64_t Lq = d2.N / grid_q, Lk = d2.N / grid_k;
+  for (int i = 0; i < grid_q; ++i) {
+    for (int j = 0; j < grid_k && mesh2d_tile_live(&d2, grid_q, grid_k, i, j); ++j) {
+      AttnArgs a = attn_args(&d2, d2.N);
+      a.Pk = grid_k;
+      a.q = offset_rows(q, i * Lq, es);
+      a.dout = offset_rows(dout, i * Lq, es);
+      a.k = offset_rows(k, j * Lk, es);
+      a.v = offset_rows(v, j * Lk, es);
+      a.lse_in = lse + i * Lq;
+      a.delta = delta + i * Lq;
+      a.dq = offset_rows(dq_acc, i * Lq, 4);
+      a.dk = offset_rows(dk_acc, j * Lk, 4);
+      a.dv = offset_rows(dv_acc, j * Lk, 4);
+      a.accumulate = 1;
+      if (d2.dtype == RM_F32) {
+        RM_CUDA(launch_simt_bwd(a, i, j, st), "simt Mesh2D tile bwd launch");
+      } else {
+        RM_TRY(tc_bwd(a, i, j, st));
+      }
+    }
+  }
+  const int out_bf16 = d2.dtype == RM_BF16;
+  RM_CUDA(launch_convert_f32(out_bf16, d2.B, d2.N, d2.Hq, d2.d, dq_acc, dq, st), "dQ convert");
+  RM_CUDA(launch_convert_f32(out_bf16, d2.B, d2.N, d2.Hkv, d2.d, dk_acc, dk, st), "dK convert");
+  RM_CUDA(launch_convert_f32(out_bf16, d2.B, d2.N, d2.Hkv, d2.d, dv_acc, dv, st), "dV convert");
+  return RM_OK;
 }
 
 }  // extern "C"

@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
   const LayoutMap lay = make_layout(a.layout, a.N, a.P);
   const int64_t L = lay.L;
   const bool ring = q_rank < 0;
+  const KeyShards kmap = key_shards(lay, a.N, ring ? a.P : kv_shards(a));
   const int r = ring ? (int)(blockIdx.z % a.P) : q_rank;
   const int b = ring ? (int)(blockIdx.z / a.P) : (int)blockIdx.z;
   const int h = blockIdx.y;
@@ -92,8 +93,8 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
   for (int step = 0; step < nsteps; ++step) {
     const int s = ring ? ((r - step) % a.P + a.P) % a.P : kv_rank;
     // keys of shard s this row (and this CTA) may see
-    const int64_t row_lim = !live ? 0 : (a.causal ? lay.visible_count(s, tq) : L);
-    const int64_t cta_lim = a.causal ? lay.visible_count(s, t_last) : L;
+    const int64_t row_lim = !live ? 0 : (a.causal ? kmap.visible_count(s, tq) : kmap.L);
+    const int64_t cta_lim = a.causal ? kmap.visible_count(s, t_last) : kmap.L;
     const int64_t kv0 = ring ? (int64_t)s * L : 0;
     const float* kb = reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
                       kv0 * a.k.stride_n;
@@ -101,8 +102,8 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
                       kv0 * a.v.stride_n;
     for (int64_t i0 = 0; i0 < cta_lim; i0 += kTile) {
       __syncthreads();
-      stage<DMAX>(ks, kb, a.k.stride_n, i0, L, a.d);
-      stage<DMAX>(vs, vb, a.v.stride_n, i0, L, a.d);
+      stage<DMAX>(ks, kb, a.k.stride_n, i0, kmap.L, a.d);
+      stage<DMAX>(vs, vb, a.v.stride_n, i0, kmap.L, a.d);
       __syncthreads();
       float sc[kTile];
       float tmax = -INFINITY;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
   const LayoutMap lay = make_layout(a.layout, a.N, a.P);
   const int64_t L = lay.L;
   const bool ring = q_rank < 0;
+  const KeyShards kmap = key_shards(lay, a.N, ring ? a.P : kv_shards(a));
   const int r = ring ? (int)(blockIdx.z % a.P) : q_rank;
   const int b = ring ? (int)(blockIdx.z / a.P) : (int)blockIdx.z;
   const int h = blockIdx.y;
@@ -180,8 +182,8 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
   const int nsteps = ring ? a.P : 1;
   for (int step = 0; step < nsteps; ++step) {
     const int s = ring ? ((r - step) % a.P + a.P) % a.P : kv_rank;
-    const int64_t row_lim = !live ? 0 : (a.causal ? lay.visible_count(s, tq) : L);
-    const int64_t cta_lim = a.causal ? lay.visible_count(s, t_last) : L;
+    const int64_t row_lim = !live ? 0 : (a.causal ? kmap.visible_count(s, tq) : kmap.L);
+    const int64_t cta_lim = a.causal ? kmap.visible_count(s, t_last) : kmap.L;
     const int64_t kv0 = ring ? (int64_t)s * L : 0;
     const float* kb = reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
                       kv0 * a.k.stride_n;
@@ -189,8 +191,8 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
                       kv0 * a.v.stride_n;
     for (int64_t i0 = 0; i0 < cta_lim; i0 += kTile) {
       __syncthreads();
-      stage<DMAX>(ks, kb, a.k.stride_n, i0, L, a.d);
-      stage<DMAX>(vs, vb, a.v.stride_n, i0, L, a.d);
+      stage<DMAX>(ks, kb, a.k.stride_n, i0, kmap.L, a.d);
+      stage<DMAX>(vs, vb, a.v.stride_n, i0, kmap.L, a.d);
       __syncthreads();
 #pragma unroll 2
       for (int kk = 0; kk < kTile; ++kk) {
@@ -230,17 +232,18 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int
   const LayoutMap lay = make_layout(a.layout, a.N, a.P);
   const int64_t L = lay.L;
   const bool ring = q_rank < 0;
+  const KeyShards kmap = key_shards(lay, a.N, ring ? a.P : kv_shards(a));
   const int s = ring ? (int)(blockIdx.z % a.P) : kv_rank;
   const int b = ring ? (int)(blockIdx.z / a.P) : (int)blockIdx.z;
   const int g = blockIdx.y;
   const int group = a.Hq / a.Hkv;
   const int row_in_cta = threadIdx.x >> 2, sub = threadIdx.x & 3;
   const int64_t i = (int64_t)blockIdx.x * kRows + row_in_cta;  // local key index
-  const bool live = i < L;
+  const bool live = i < kmap.L;
   const int64_t krow = (ring ? (int64_t)s * L : 0) + i;
-  const int64_t tk = live ? lay.pos(s, i) : 0;
+  const int64_t tk = live ? kmap.pos(s, i) : 0;
   const int64_t i_first = (int64_t)blockIdx.x * kRows;
-  const int64_t t_first = lay.pos(s, i_first);
+  const int64_t t_first = kmap.pos(s, i_first);
 
   Slice<DMAX> k, v, dk, dv;
 #pragma unroll
@@ -335,7 +338,7 @@ cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   if (L == 0 || a.B == 0 || a.Hq == 0) return cudaSuccess;
   const unsigned z = (unsigned)(q_rank < 0 ? a.B * a.P : a.B);
   dim3 gq((unsigned)ceil_div(L, kRows), (unsigned)a.Hq, z);
-  dim3 gk((unsigned)ceil_div(L, kRows), (unsigned)a.Hkv, z);
+  dim3 gk((unsigned)ceil_div(q_rank < 0 ? L : a.N / kv_shards(a), kRows), (unsigned)a.Hkv, z);
   ProfScope ps("simt_bwd", stream);
   if (a.d <= 32) {
     simt_bwd_dq_kernel<32><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);

@@ -43,6 +43,8 @@ constexpr int D = 128;  // head dim
 struct BwdParams {
   int B, Hq, Hkv, P, layout, causal;
   int64_t N, L;
+  int Pk;      // KV shards: P, except for one (query chunk, KV chunk) tile of a rectangular grid
+  int64_t Lk;  // N / Pk
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int ring, q_rank, kv_rank;
@@ -253,6 +255,8 @@ struct Walk {
 //   dV(i) [needs P^T(i)], dK(i) [needs dS^T(i)], dP^T(i+1), S^T(i+2)
 // and the exponentials of tile i+1 overlap all four; the in-order pipe makes
 // the single dP^T buffer safe (dP^T(i+1) is issued after dK(i) read dS^T(i)).
+// kChunkedKeys: the KV side is one contiguous chunk of a rectangular grid (Pk != P).
+template <bool kChunkedKeys>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -283,14 +287,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   Walk W;
   W.lay = make_layout(p.layout, p.N, p.P);
-  const int64_t L = p.L;
+  const int64_t L = p.L;                   // queries per shard
+  const int64_t Lk = kChunkedKeys ? p.Lk : L;  // keys per shard
+  // global position of key i of shard s (a tile of a rectangular grid:
+  // contiguous chunks of Lk keys)
+  auto kpos = [&](int s, int64_t i) -> int64_t {
+    return kChunkedKeys ? (int64_t)s * Lk + i : W.lay.pos(s, i);
+  };
   // grid: (key tile in order of decreasing work x KV head, KV head block, batch)
   const int b = blockIdx.z;
   int c, gh;
   if (!grid_place(p.head_block, p.Hkv, c, gh)) return;
   int xt;
   {
-    const int T = (int)((L + BK - 1) / BK);
+    const int T = (int)((Lk + BK - 1) / BK);
     if (!p.ring) {
       W.s = p.kv_rank;
       xt = c;
@@ -313,8 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
   {  // queries that may see a key of the CTA (the bounds are monotone in the key)
     int64_t f, l;
-    sg.key_span(b, W.lay.pos(W.s, i0), p.causal, W.span_first, l);
-    sg.key_span(b, W.lay.pos(W.s, LayoutMap::min64(i0 + BK - 1, L - 1)), p.causal, f, W.span_last);
+    sg.key_span(b, kpos(W.s, i0), p.causal, W.span_first, l);
+    sg.key_span(b, kpos(W.s, LayoutMap::min64(i0 + BK - 1, Lk - 1)), p.causal, f, W.span_last);
   }
   const int s = W.s, g = W.g;
   const long long limit = p.wait_limit;
@@ -459,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = (uint32_t)lane_base << 16;
     const int krow = lane_base + lane;       // key row of the tile (TMEM lane)
     const int64_t key = i0 + krow;
-    const bool key_live = key < L;
+    const bool key_live = key < Lk;
     // local queries [span_lo, span_hi) of rank span_rank see this key
     int span_rank = -1, span_lo = 0, span_hi = 0;
     const int tid = threadIdx.x & 127;
@@ -489,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         span_lo = span_hi = 0;
         if (key_live) {
           int64_t f, l;  // global positions of the queries that see this key
-          sg.key_span(b, W.lay.pos(s, key), p.causal, f, l);
+          sg.key_span(b, kpos(s, key), p.causal, f, l);
           span_lo = (int)W.lay.visible_count(r, f - 1);
           span_hi = (int)W.lay.visible_count(r, l);
         }
@@ -651,6 +661,8 @@ __device__ __forceinline__ uint32_t a_col(int k) { return kHalf * (k >> 2) + 8 *
 // tensor pipe runs, per tile j,
 //   dQ(j) [needs dS(j)], dP(j+1), S(j+2)
 // so the exponentials of tile j+1 overlap dQ(j) and dP(j+1).
+// kChunkedKeys: the KV side is one contiguous chunk of a rectangular grid (Pk != P).
+template <bool kChunkedKeys>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -711,11 +723,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long limit = p.wait_limit;
   const BwdRows R = bwd_rows(p);
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
-  // key tiles [tile_begin(s), tile_end(s)) of shard s hold every key the CTA may see
-  auto tile_begin = [&](int s) -> int { return (int)(lay.visible_count(s, span_first - 1) / BN); };
-  auto tile_end = [&](int s) -> int {
-    return (int)((lay.visible_count(s, span_last) + BN - 1) / BN);
+  // keys of shard s at global positions <= t: the layout's count, or for a
+  // tile of a rectangular grid (contiguous chunks of Lk keys) the chunk's
+  auto kvis = [&](int s, int64_t t) -> int64_t {
+    return !kChunkedKeys ? lay.visible_count(s, t)
+                       : LayoutMap::clamp64(t - (int64_t)s * p.Lk + 1, 0, p.Lk);
   };
+  // key tiles [tile_begin(s), tile_end(s)) of shard s hold every key the CTA may see
+  auto tile_begin = [&](int s) -> int { return (int)(kvis(s, span_first - 1) / BN); };
+  auto tile_end = [&](int s) -> int { return (int)((kvis(s, span_last) + BN - 1) / BN); };
   int n = 0;  // key tiles of the whole walk
   for (int step = 0; step < nsteps; ++step) {
     const int s = shard_of(step);
@@ -874,8 +890,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (live) {
         int64_t f, l;
         sg.query_span(b, tq, p.causal, f, l);
-        row_lo = lay.visible_count(s, f - 1);
-        row_hi = lay.visible_count(s, l);
+        row_lo = kvis(s, f - 1);
+        row_hi = kvis(s, l);
       }
       for (int t = tile_begin(s); t < te; ++t, ++j) {
         const uint32_t cS = kTS + (j & 1) * BN + kHalf * X, cdP = kTdP + kHalf * X;
@@ -964,6 +980,8 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   if (a.d != D) return RM_ERR_UNSUPPORTED;
   const bool ring = q_rank < 0;
   const int64_t L = a.N / a.P;
+  const int Pk = ring ? a.P : kv_shards(a);
+  const int64_t Lk = a.N / Pk;
   const int shards = ring ? a.P : 1;
   BwdParams p;
   p.B = a.B;
@@ -974,6 +992,8 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.causal = a.causal;
   p.N = a.N;
   p.L = L;
+  p.Pk = Pk;
+  p.Lk = Lk;
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   p.ring = ring ? 1 : 0;
@@ -1006,26 +1026,27 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   {  // dK, dV
     CUtensorMap mq, mk, mv, mdo;
     if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, kv::BQ, view) != RM_OK ||
-        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
-        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, Lk, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, Lk, a.Hkv, a.d, 64, kv::BK, view) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, kv::BQ, view) != RM_OK)
       return RM_ERR_CUDA;
     // a key-tile CTA streams Q and dO of every query head of its group
     p.head_block = head_block((int64_t)(a.Hq / a.Hkv) * a.N * D * 2 * 2, a.Hkv);
-    dim3 grid((unsigned)(ceil_div(L, kv::BK) * shards * p.head_block),
+    dim3 grid((unsigned)(ceil_div(Lk, kv::BK) * shards * p.head_block),
               (unsigned)ceil_div(a.Hkv, p.head_block), (unsigned)a.B);
-    if (cudaFuncSetAttribute(kv::tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kv::kSmem) != cudaSuccess)
+    auto kernel = Pk != a.P ? kv::tc_bwd_dkdv_kernel<true> : kv::tc_bwd_dkdv_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem) !=
+        cudaSuccess)
       return RM_ERR_CUDA;
     ProfScope ps("tc_bwd_dkdv_kernel", stream);
-    kv::tc_bwd_dkdv_kernel<<<grid, kv::kThreads, kv::kSmem, stream>>>(mq, mk, mv, mdo, p);
+    kernel<<<grid, kv::kThreads, kv::kSmem, stream>>>(mq, mk, mv, mdo, p);
     if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
   }
   {  // dQ
     CUtensorMap mq, mk, mv, mdo;
     if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, 64, dq::BM, view) != RM_OK ||
-        encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
-        encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
+        encode_operand_map(&mk, a.k, a.B, shards, Lk, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
+        encode_operand_map(&mv, a.v, a.B, shards, Lk, a.Hkv, a.d, 64, dq::BN, view) != RM_OK ||
         encode_operand_map(&mdo, a.dout, a.B, shards, L, a.Hq, a.d, 64, dq::BM, view) != RM_OK)
       return RM_ERR_CUDA;
     // a query-tile CTA streams K and V of its KV head (shared by the group)
@@ -1033,11 +1054,12 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
     p.head_block = head_block((int64_t)a.N * D * 2 * 2 / group, a.Hq);
     dim3 grid((unsigned)(ceil_div(L, dq::BM) * shards * p.head_block),
               (unsigned)ceil_div(a.Hq, p.head_block), (unsigned)a.B);
-    if (cudaFuncSetAttribute(dq::tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             dq::kSmem) != cudaSuccess)
+    auto kernel = Pk != a.P ? dq::tc_bwd_dq_kernel<true> : dq::tc_bwd_dq_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem) !=
+        cudaSuccess)
       return RM_ERR_CUDA;
     ProfScope ps("tc_bwd_dq_kernel", stream);
-    dq::tc_bwd_dq_kernel<<<grid, dq::kThreads, dq::kSmem, stream>>>(mq, mk, mv, mdo, p);
+    kernel<<<grid, dq::kThreads, dq::kSmem, stream>>>(mq, mk, mv, mdo, p);
     if (cudaGetLastError() != cudaSuccess) return RM_ERR_CUDA;
   }
   return RM_OK;

@@ -72,6 +72,8 @@ struct FwdCfg {
 
 struct FwdParams {
   int B, Hq, Hkv, d, P, layout, causal;
+  int Pk;     // KV shards: P, except for one (query chunk, KV chunk) tile of a rectangular grid
+  int64_t Lk;  // N / Pk
   int64_t N, L;
   float scale_log2;  // softmax scale * log2(e)
   int ring, q_rank, kv_rank;
@@ -138,6 +140,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const LayoutMap lay = make_layout(p.layout, p.N, p.P);
+  // keys of shard s at global positions <= t: the layout's count, or for a
+  // tile of a rectangular grid (contiguous chunks of Lk keys) the chunk's
+  auto kvis = [&](int s, int64_t t) -> int64_t {
+    return p.Pk == p.P ? lay.visible_count(s, t)
+                       : LayoutMap::clamp64(t - (int64_t)s * p.Lk + 1, 0, p.Lk);
+  };
   const int64_t L = p.L;
   // grid: (row unit in order of decreasing work x head unit, head block, batch);
   // a head unit is a head pair (heads 2x, 2x+1) or one head
@@ -224,9 +232,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // KV shard of ring step `step`, and how many of its keys the CTA may see.
   auto shard_of = [&](int step) { return p.ring ? ((r - step) % p.P + p.P) % p.P : p.kv_rank; };
   // key tiles [tile_begin(s), tile_end(s)) of shard s hold every key the CTA may see
-  auto tile_begin = [&](int s) -> int { return (int)(lay.visible_count(s, span_first - 1) / kBN); };
+  auto tile_begin = [&](int s) -> int {
+    return (int)(kvis(s, span_first - 1) / kBN);
+  };
   auto tile_end = [&](int s) -> int {
-    return (int)((lay.visible_count(s, span_last) + kBN - 1) / kBN);
+    return (int)((kvis(s, span_last) + kBN - 1) / kBN);
   };
 
   if (warp >= 8) {
@@ -365,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (live) {
         int64_t f, l;
         sg.query_span(b, tq, p.causal, f, l);
-        row_lo = lay.visible_count(s, f - 1);
-        row_hi = lay.visible_count(s, l);
+        row_lo = kvis(s, f - 1);
+        row_hi = kvis(s, l);
       }
       for (int t = tile_begin(s); t < te; ++t, ++j) {
         // all lanes leave together, so the warp-collective tcgen05.ld / st
@@ -601,12 +611,14 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   using C = FwdCfg<DP>;
   const bool ring = q_rank < 0;
   const int64_t L = a.N / a.P;
+  const int Pk = ring ? a.P : kv_shards(a);
+  const int64_t Lk = a.N / Pk;
   const int shards = ring ? a.P : 1;
   CUtensorMap mq, mk, mv;
   const int view = operand_view(a, ring);
   if (encode_operand_map(&mq, a.q, a.B, shards, L, a.Hq, a.d, C::kBoxCols, kBM, view) != RM_OK ||
-      encode_operand_map(&mk, a.k, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK ||
-      encode_operand_map(&mv, a.v, a.B, shards, L, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK)
+      encode_operand_map(&mk, a.k, a.B, shards, Lk, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK ||
+      encode_operand_map(&mv, a.v, a.B, shards, Lk, a.Hkv, a.d, C::kBoxCols, kBN, view) != RM_OK)
     return RM_ERR_CUDA;
   FwdParams p;
   p.B = a.B;
@@ -614,6 +626,8 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.P = a.P;
+  p.Pk = Pk;
+  p.Lk = Lk;
   p.layout = a.layout;
   p.causal = a.causal;
   p.N = a.N;

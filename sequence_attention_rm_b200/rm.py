@@ -31,7 +31,7 @@ EXPORTED = (
     "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
     "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
     "rm_profile_get", "rm_usp_auto_select", "rm_usp_workspace_size", "rm_usp_attn_fwd",
-    "rm_usp_attn_bwd",
+    "rm_usp_attn_bwd", "rm_mesh2d_workspace_size", "rm_mesh2d_attn_fwd", "rm_mesh2d_attn_bwd",
 )
 
 
@@ -82,6 +82,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_usp_workspace_size": [D, i, i, ctypes.POINTER(sz)],
         "rm_usp_attn_fwd": [D, i, T, T, T, T, vp, vp, sz, vp],
         "rm_usp_attn_bwd": [D, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp],
+        "rm_mesh2d_workspace_size": [D, i, i, i, ctypes.POINTER(sz)],
+        "rm_mesh2d_attn_fwd": [D, i, i, T, T, T, T, vp, vp, sz, vp],
+        "rm_mesh2d_attn_bwd": [D, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -338,6 +341,42 @@ def usp_attn_bwd(q, k, v, o, lse, dout, *, P: int, ulysses: int, layout: str, ca
     _check(_lib.rm_usp_attn_bwd(ctypes.byref(dsc), ulysses, _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
                                 _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
                                 _stream(stream)))
+    return dq, dk, dv
+
+
+def mesh2d_workspace_size(dsc: RmAttnDesc, grid_q: int, grid_k: int, backward: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.rm_mesh2d_workspace_size(ctypes.byref(dsc), grid_q, grid_k, int(backward),
+                                         ctypes.byref(n)))
+    return n.value
+
+
+def mesh2d_attn_fwd(q, k, v, *, grid_q: int, grid_k: int, causal: bool,
+                    scale: float | None = None, out=None, lse=None, ws=None, stream=None):
+    """Mesh2D forward over a grid_q x grid_k grid of (query chunk, key chunk)
+    tiles; q/k/v [B, N, H, d] in token order -> (O, LSE [B, Hq, N])."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale)
+    out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    wp, wn = _workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, False), q.device, ws)
+    _check(_lib.rm_mesh2d_attn_fwd(ctypes.byref(dsc), grid_q, grid_k, _bnhd(q), _bnhd(k),
+                                   _bnhd(v), _bnhd(out), _ptr(lse), wp, wn, _stream(stream)))
+    return out, lse
+
+
+def mesh2d_attn_bwd(q, k, v, o, lse, dout, *, grid_q: int, grid_k: int, causal: bool,
+                    scale: float | None = None, dq=None, dk=None, dv=None, ws=None, stream=None):
+    """Mesh2D backward -> (dq, dk, dv) in the input dtype."""
+    B, N, Hq, d = q.shape
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale)
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    wp, wn = _workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, True), q.device, ws)
+    _check(_lib.rm_mesh2d_attn_bwd(ctypes.byref(dsc), grid_q, grid_k, _bnhd(q), _bnhd(k),
+                                   _bnhd(v), _bnhd(o), _ptr(lse), _bnhd(dout), _bnhd(dq),
+                                   _bnhd(dk), _bnhd(dv), wp, wn, _stream(stream)))
     return dq, dk, dv
 
 

@@ -165,3 +165,23 @@ def test_usp_workspace_sizes(rm):
     assert n.value == 2 * q_bytes + 2 * kv_bytes
     assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), 2, 1, ctypes.byref(n)) == 0
     assert n.value == 4 * q_bytes + 4 * kv_bytes + 16 * 16384 * 4
+
+
+@pytest.mark.parametrize("gq,gk,status", [(0, 1, 1), (2, 0, 1), (3, 1, 1), (2, 3, 1), (2, 17, 2)])
+def test_mesh2d_validation(rm, gq, gk, status):
+    n = ctypes.c_size_t(0)
+    d = _desc(rm)  # N = 16384
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), gq, gk, 0, ctypes.byref(n)) == status
+    assert rm.raw().rm_last_error()
+    d = _desc(rm, seq_lens=16)
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 2, 2, 0, ctypes.byref(n)) == 2
+
+
+def test_mesh2d_workspace_sizes(rm):
+    n = ctypes.c_size_t(0)
+    d = _desc(rm)  # bf16 B=1 Hq=16 Hkv=8 d=128 N=16384; P and layout are ignored
+    o_slot, lse_slot = 16384 * 16 * 128 * 4, 16384 * 16 * 4
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 4, 8, 0, ctypes.byref(n)) == 0
+    assert n.value == 8 * o_slot + 8 * lse_slot
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 4, 8, 1, ctypes.byref(n)) == 0
+    assert n.value == lse_slot + o_slot + 2 * (16384 * 8 * 128 * 4)
