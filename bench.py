@@ -276,29 +276,52 @@ def bench_ours(args, world, rank, local):
     value = total_flops / (step_ms_max * 1e-3) / 1e12
     kernels = kernel_table(records, args.steps, step_ms / args.steps, w)
 
-    # end-to-end: pinned host inputs in, results back to pinned host buffers
+    # end-to-end: pinned host inputs in, results back to pinned host buffers,
+    # every step.  Two device slots and three streams: step i+1's inputs are
+    # copied in and step i-1's results copied out while step i computes.
     pin = lambda t: t.pin_memory()
     hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
-    outs = [pin(torch.empty(t.shape, dtype=t.dtype)) for t in (step.o_g, step.dq_g, step.dk_g, step.dv_g, step.lse_g)]
+    slots = [step, Step(rm, w, *(torch.empty_like(t) for t in (q, k, v, do)))]
+    host_out = [[pin(torch.empty(t.shape, dtype=t.dtype))
+                 for t in (sl.o_g, sl.dq_g, sl.dk_g, sl.dv_g, sl.lse_g)] for sl in slots]
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in outs)
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    done_in, done_run, done_out = ([ev(), ev()] for _ in range(3))
 
-    def e2e_step():
-        for src, dst in ((hq, step.q), (hk, step.k), (hv, step.v), (hdo, step.do)):
-            dst.copy_(src, non_blocking=True)
-        step.run()
-        for src, dst in zip((step.o_g, step.dq_g, step.dk_g, step.dv_g, step.lse_g), outs):
-            dst.copy_(src, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        sl = slots[j]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(done_run[j])  # slot j's inputs free again
+            for src, dst in ((hq, sl.q), (hk, sl.k), (hv, sl.v), (hdo, sl.do)):
+                dst.copy_(src, non_blocking=True)
+            done_in[j].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(done_in[j])
+            if i >= 2:
+                s_run.wait_event(done_out[j])  # slot j's results copied out
+            sl.run()
+            done_run[j].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done_run[j])
+            for src, dst in zip((sl.o_g, sl.dq_g, sl.dk_g, sl.dv_g, sl.lse_g), host_out[j]):
+                dst.copy_(src, non_blocking=True)
+            done_out[j].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    for i in range(max(1, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record()
+    e0.record(s_in)
+    for i in range(args.steps):
+        e2e_step(i)
+    # the last results are on the host once s_out is done; it waited on
+    # everything before it
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
@@ -341,10 +364,12 @@ def bench_ours(args, world, rank, local):
     line["ring_fwd_tflops"] = round(fwd_tflops, 2)
     line["ring_bwd_tflops"] = round(bwd_tflops, 2)
     line["e2e"] = {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                   "d2h_bytes_per_step": d2h}
+                   "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4),
+                   "pipeline": "2 device slots; host->device copy, step and device->host copy "
+                               "on 3 streams (step i+1 in, step i-1 out during step i)"}
     line["gpu_launches"] = len(records)
     line["clocks"] = clk.summary()
-    del step, q, k, v, do
+    del step, slots, q, k, v, do
     torch.cuda.empty_cache()
 
     if not args.no_extras:
@@ -354,18 +379,48 @@ def bench_ours(args, world, rank, local):
     return line
 
 
-def _time(fn, reps, flush):
-    ts = []
+def _time(fn, reps, flush, rm=None):
+    """Median device time of fn() in ms.  A short spin kernel runs before the
+    start event, so the host has queued fn's launches before the GPU reaches
+    them and the interval holds no host time.  With `rm`, the median of the
+    summed per-launch event times the library records around its own kernels
+    is returned too: (kernels, call) (the kernels alone, no gaps between
+    launches)."""
+    ts, ks = [], []
     for _ in range(reps):
         if flush is not None:
             flush_l2(flush)
+        torch.cuda._sleep(SPIN_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if rm is not None:
+            rm.profile_enable(True)
         a.record()
         fn()
         b.record()
         torch.cuda.synchronize()
+        if rm is not None:
+            ks.append(sum(ms for _, ms in rm.profile_records()))
+            rm.profile_enable(False)
         ts.append(a.elapsed_time(b))
-    return statistics.median(ts)
+    if rm is None:
+        return statistics.median(ts)
+    return statistics.median(ks), statistics.median(ts)
+
+
+# about 1 ms of spinning at the B200's clocks: longer than the host needs to
+# queue any call timed here
+SPIN_CYCLES = 2_000_000
+
+
+def hbm_row(rm, fn, reps, flush, nbytes, hbm, peak_src, shape):
+    """An HBM-bound call: algorithmic bytes over the device time of its
+    kernels (the library's per-launch events), the whole call beside it."""
+    fn()
+    ms, call_ms = _time(fn, reps, flush, rm)
+    return {"shape": shape, "ms": round(ms, 4), "call_ms": round(call_ms, 4),
+            "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
+            "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes,
+            "timing": "kernel device time (per-launch CUDA events)"}
 
 
 def extras(rm, peaks, peak_src, dev, flush):
@@ -378,23 +433,16 @@ def extras(rm, peaks, peak_src, dev, flush):
     o_out = torch.empty(1, P * Lr, H, d, dtype=torch.bfloat16, device=dev)
     lse_out = torch.empty(1, H, P * Lr, device=dev)
     fn = lambda: rm.lse_merge(o_parts, lse_parts, torch.bfloat16, out=o_out, lse_out=lse_out)
-    fn()
-    ms = _time(fn, 10, flush)
     nbytes = P * (P * Lr * H * d * 4 + H * P * Lr * 4) + P * Lr * H * d * 2 + H * P * Lr * 4
-    out["lse_merge"] = {"shape": "8 partials x [1, 131072, 16, 128] fp32 -> bf16", "ms": round(ms, 4),
-                        "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
-                        "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    out["lse_merge"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                               "8 partials x [1, 131072, 16, 128] fp32 -> bf16")
     # pairwise merge (the running-state form): fp32 O_acc <- merge(O_acc, O_new), in place
     acc, lacc = o_parts[0], lse_parts[0]
     fn = lambda: rm.lse_merge([acc, o_parts[1]], [lacc, lse_parts[1]], torch.float32, out=acc,
                               lse_out=lacc)
-    fn()
-    ms = _time(fn, 10, flush)
     nbytes = 3 * P * Lr * H * d * 4 + 3 * H * P * Lr * 4
-    out["lse_merge_pairwise"] = {"shape": "2 partials x [1, 131072, 16, 128] fp32 -> fp32 in place",
-                                 "ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1),
-                                 "frac": round(nbytes / ms / 1e6 / hbm, 4), "peak": hbm,
-                                 "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    out["lse_merge_pairwise"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                                        "2 partials x [1, 131072, 16, 128] fp32 -> fp32 in place")
     del o_parts, lse_parts, o_out, lse_out
     # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and the fused K|V (8 K heads
     # then 8 V heads) of the same shape, seq -> head, one call each
@@ -403,13 +451,9 @@ def extras(rm, peaks, peak_src, dev, flush):
     y = torch.empty(8, 8 * 32768, 2, 128, dtype=torch.bfloat16, device=dev)
     y2 = torch.empty_like(y)
     fn = lambda: (rm.seq_head_repack(x, 8, out=y), rm.seq_head_repack(kv, 8, out=y2))
-    fn()
-    ms = _time(fn, 10, flush)
     nbytes = 2 * (x.numel() + kv.numel()) * 2
-    out["repack"] = {"shape": "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16",
-                     "ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1),
-                     "frac": round(nbytes / ms / 1e6 / hbm, 4), "peak": hbm,
-                     "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    out["repack"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                            "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16")
     del x, kv, y, y2
     # the causal striped 128k forward (fused ring over 8 virtual ranks)
     w3 = synthetic.STRIPED_128K
@@ -428,12 +472,9 @@ def extras(rm, peaks, peak_src, dev, flush):
     # layout permute of the striped 128k Q (global -> rank-major), 2 x 512 MiB
     o2 = torch.empty_like(q)
     fn = lambda: rm.layout_permute(q, "striped", 8, out=o2)
-    fn()
-    ms = _time(fn, 10, flush)
     nbytes = 2 * q.numel() * 2
-    out["permute"] = {"shape": "striped P=8 [1, 131072, 16, 128] bf16", "ms": round(ms, 4),
-                      "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
-                      "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    out["permute"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                             "striped P=8 [1, 131072, 16, 128] bf16")
     del q, k, v, o, lse, o2
     out["tabular_row_fwd"], out["tabular_feature_fwd"] = tabular(rm, flush, hbm, peak_src)
     out["usp_16k_fwd_bwd"] = usp_line(rm, flush, peaks, peak_src)
@@ -544,12 +585,9 @@ def tabular(rm, flush, hbm, peak_src):
     flse = torch.empty(w.batch * R, H, F, device="cuda")
     fn = lambda: rm.attn_block_fwd(fview(q), fview(k), fview(v), N=F, P=1, layout="contiguous",
                                    causal=False, q_rank=0, kv_rank=0, out=fo, lse=flse)
-    fn()
-    ms = _time(fn, 10, flush)
     nbytes = 4 * q.numel() * 2 + flse.numel() * 4
-    feat = {"shape": f"{w.batch * R * H} sequences x {F} tokens, d={E // H}", "ms": round(ms, 4),
-            "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / hbm, 4),
-            "peak": hbm, "peak_source": f"{peak_src} hbm_gbs", "bytes": nbytes}
+    feat = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                   f"{w.batch * R * H} sequences x {F} tokens, d={E // H}")
     return row, feat
 
 

@@ -51,13 +51,18 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
   const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nparts = NPARTS > 0 ? NPARTS : a.n_parts;
-  for (int64_t base = warp0 * rows_per_warp; base < rows; base += nwarps * rows_per_warp) {
-    const int64_t row = base + sub;
-    if (row >= rows) continue;
-    const int64_t t = row % a.Nq;
-    const int64_t bh = row / a.Nq;
-    const int h = (int)(bh % a.H);
-    const int b = (int)(bh / a.H);
+  // row = (b * H + h) * Nq + t.  The row index is split once; each pass then
+  // adds the grid stride to (t, h, b) with carries, so the loop divides nothing.
+  const int64_t step = nwarps * rows_per_warp;
+  int64_t row = warp0 * rows_per_warp + sub;
+  int64_t t = row % a.Nq;
+  int h = (int)((row / a.Nq) % a.H);
+  int b = (int)(row / a.Nq / a.H);
+  const int64_t st_t = step % a.Nq;
+  const int st_h = (int)((step / a.Nq) % a.H);
+  const int st_b = (int)(step / a.Nq / a.H);
+  for (; row < rows; row += step) {
+    const int64_t bh = (int64_t)b * a.H + h;
     const int64_t lidx = bh * a.lse_ld + t;
     const bool active = col < a.d;
     // every load of the row is issued before any of them is used (the O loads
@@ -109,6 +114,13 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
       store4(out, acc);
     }
     if ((lane % lanes) == 0) a.lse_out[lidx] = lse;
+    t += st_t;
+    int carry = t >= a.Nq;
+    if (carry) t -= a.Nq;
+    h += st_h + carry;
+    carry = h >= a.H;
+    if (carry) h -= a.H;
+    b += st_b + carry;
   }
 }
 

@@ -11,10 +11,17 @@
 // allow it (VEC), else element by element.
 #include <math.h>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace rm {
+
+rm_status encode_copy_map(CUtensorMap* map, const void* ptr, int esize, const int64_t (&dims)[5],
+                          const int64_t (&strides)[4], const int (&box)[5]);
+long long tc_wait_limit();
 
 namespace {
 
@@ -155,6 +162,282 @@ __global__ void __launch_bounds__(kThreads) small_seq_attn_kernel(AttnArgs a, in
   }
 }
 
+// bf16 operands with 16-byte rows: persistent blocks (two per SM) walk
+// batches of SB whole sequences through a two-stage shared-memory ring.  For
+// each batch one thread issues three asynchronous copies -- the Q, K and V
+// rows of the batch -- onto the stage's mbarrier, one batch ahead of the
+// batch being computed, so staging costs no per-element index arithmetic and
+// the next batch is in flight during the math.  Dense operands take one bulk
+// copy each (a batch is one run of memory); strided views take TMA boxes
+// (d, H, L, SB) of their [B, L, H, d] maps, which read as zero past the last
+// sequence.  One thread per
+// (sequence, query token, head) scores its keys from shared memory with
+// packed fp32 FMAs, writes its O row with 16-byte stores and parks its LSE in
+// shared memory, from which the block writes the [B, H, L] LSE rows in order.
+struct StagedLayout {
+  int SB;
+  uint32_t q_bytes, kv_bytes;  // box bytes (the TMA transaction sizes)
+  uint32_t off_k, off_v;       // within a stage
+  uint32_t stage_bytes;
+  uint32_t off_lse, off_bar, total;
+};
+
+constexpr int kStagedStages = 2;
+constexpr int kStagedCtasPerSm = 2;
+constexpr uint32_t kStagedStageBudget = 48 * 1024;  // one stage's three boxes
+
+__host__ __device__ inline uint32_t round128(uint32_t x) { return (x + 127u) & ~127u; }
+
+__host__ __device__ inline StagedLayout staged_layout(int SB, int L, int Hq, int Hkv, int d) {
+  StagedLayout g;
+  g.SB = SB;
+  g.q_bytes = (uint32_t)SB * L * Hq * d * 2;
+  g.kv_bytes = (uint32_t)SB * L * Hkv * d * 2;
+  g.off_k = round128(g.q_bytes);
+  g.off_v = g.off_k + round128(g.kv_bytes);
+  g.stage_bytes = g.off_v + round128(g.kv_bytes);
+  g.off_lse = kStagedStages * g.stage_bytes;
+  g.off_bar = (g.off_lse + (uint32_t)SB * Hq * L * 4 + 7u) & ~7u;
+  g.total = g.off_bar + 8 * kStagedStages;
+  return g;
+}
+
+// One contiguous run of global memory into shared memory through the bulk
+// copy unit, completing `bytes` on the mbarrier (16-byte aligned addresses,
+// size a multiple of 16; no multicast).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(tc::smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(tc::smem_u32(bar))
+      : "memory");
+}
+
+// bf16 pair (low, high halves of a 32-bit word) -> fp32 pair
+__device__ __forceinline__ float2 bf16x2_f32(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <int DMAX>
+__global__ void __launch_bounds__(kThreads, DMAX <= 32 ? kStagedCtasPerSm : 1)
+    small_seq_tma_kernel(const __grid_constant__ CUtensorMap mq,
+                         const __grid_constant__ CUtensorMap mk,
+                         const __grid_constant__ CUtensorMap mv, AttnArgs a, int q_rank,
+                         int kv_rank, StagedLayout g, int contiguous, long long wait_limit) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  using namespace tc;
+  const LayoutMap lay = make_layout(a.layout, a.N, a.P);
+  const int L = (int)lay.L;
+  const int d = a.d;
+  const int Hq = a.Hq, Hkv = a.Hkv;
+  const int group = Hq / Hkv;
+  float* lse_s = reinterpret_cast<float*>(smem + g.off_lse);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+  const int64_t nbatch = ((int64_t)a.B + g.SB - 1) / g.SB;
+  const int64_t mine =
+      nbatch > blockIdx.x ? (nbatch - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if ((smem_u32(smem) & 127u) != 0) {  // TMA boxes need a 128-byte aligned destination
+    if (threadIdx.x == 0) report_status(a.status, kStatusSmemAlign);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStagedStages; ++st) mbar_init(bars + st, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t k) {  // batch k of this block into stage k % 2
+    unsigned char* st = smem + (k & 1) * g.stage_bytes;
+    uint64_t* bar = bars + (k & 1);
+    const int bc = (int)((blockIdx.x + k * gridDim.x) * g.SB);
+    if (contiguous) {
+      // the batch's rows of each operand are one run: sb sequences of L*H*d
+      const int sb = a.B - bc < g.SB ? a.B - bc : g.SB;
+      const uint32_t qb = g.q_bytes / g.SB * sb, kvb = g.kv_bytes / g.SB * sb;
+      mbar_arrive_expect_tx(bar, qb + 2 * kvb);
+      const size_t off = (size_t)bc * a.q.stride_b * 2, koff = (size_t)bc * a.k.stride_b * 2;
+      bulk_load(st, reinterpret_cast<const char*>(a.q.ptr) + off, qb, bar);
+      bulk_load(st + g.off_k, reinterpret_cast<const char*>(a.k.ptr) + koff, kvb, bar);
+      bulk_load(st + g.off_v, reinterpret_cast<const char*>(a.v.ptr) + koff, kvb, bar);
+    } else {
+      mbar_arrive_expect_tx(bar, g.q_bytes + 2 * g.kv_bytes);
+      tma_load_5d(st, &mq, bar, 0, 0, 0, bc, 0);
+      tma_load_5d(st + g.off_k, &mk, bar, 0, 0, 0, bc, 0);
+      tma_load_5d(st + g.off_v, &mv, bar, 0, 0, 0, bc, 0);
+    }
+  };
+  if (threadIdx.x == 0 && mine > 0) issue(0);
+
+  const float qscale = a.scale * kLog2e;  // scores in log2 units
+  for (int64_t k = 0; k < mine; ++k) {
+    // the other stage was last read by batch k - 1, which every thread has
+    // finished (barrier at the end of the previous pass)
+    if (threadIdx.x == 0 && k + 1 < mine) {
+      fence_proxy_async_smem();  // this thread's reads of the stage before the TMA writes
+      issue(k + 1);
+    }
+    // a timeout ends the whole block together (no thread may be left at a
+    // barrier the others have passed)
+    const bool ok = mbar_wait(bars + (k & 1), (uint32_t)((k >> 1) & 1), wait_limit, a.status);
+    if (!__syncthreads_and(ok)) {
+      // boxes may still be landing: wait for them once more (bounded) before
+      // the block's shared memory is given up
+      if (threadIdx.x == 0) {
+        mbar_wait(bars + (k & 1), (uint32_t)((k >> 1) & 1), wait_limit, a.status);
+        if (k + 1 < mine)
+          mbar_wait(bars + ((k + 1) & 1), (uint32_t)(((k + 1) >> 1) & 1), wait_limit, a.status);
+      }
+      return;
+    }
+    const unsigned char* st = smem + (k & 1) * g.stage_bytes;
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(st);
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(st + g.off_k);
+    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(st + g.off_v);
+    const int64_t b0 = (blockIdx.x + k * gridDim.x) * g.SB;
+    const int sb = (int)((int64_t)a.B - b0 < g.SB ? (int64_t)a.B - b0 : g.SB);
+    const int work = sb * L * Hq;
+    for (int idx = threadIdx.x; idx < work; idx += kThreads) {
+      const int h = idx % Hq;
+      const int r = idx / Hq;  // s * L + t
+      const int t = r % L;
+      const int s = r / L;
+      const int kvh = h / group;
+      float2 q[DMAX / 2];
+      {
+        const uint4* q4 = reinterpret_cast<const uint4*>(qs + ((size_t)r * Hq + h) * d);
+#pragma unroll
+        for (int i = 0; i < DMAX / 8; ++i) {
+          if (8 * i < d) {
+            const uint4 w = q4[i];
+            q[4 * i] = bf16x2_f32(w.x);
+            q[4 * i + 1] = bf16x2_f32(w.y);
+            q[4 * i + 2] = bf16x2_f32(w.z);
+            q[4 * i + 3] = bf16x2_f32(w.w);
+          }
+        }
+      }
+      const int64_t tq = lay.pos(q_rank, t);
+      const __nv_bfloat16* kseq = ks + ((size_t)s * L * Hkv + kvh) * d;  // key 0 of sequence s
+      const __nv_bfloat16* vseq = vs + ((size_t)s * L * Hkv + kvh) * d;
+      float sc[kMaxL];
+      float m = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < kMaxL; ++u) {
+        sc[u] = -INFINITY;
+        if (u < L && (!a.causal || lay.pos(kv_rank, u) <= tq)) {
+          const uint4* k4 = reinterpret_cast<const uint4*>(kseq + (size_t)u * Hkv * d);
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < DMAX / 8; ++i) {
+            if (8 * i < d) {
+              const uint4 w = k4[i];
+              acc = __ffma2_rn(q[4 * i], bf16x2_f32(w.x), acc);
+              acc = __ffma2_rn(q[4 * i + 1], bf16x2_f32(w.y), acc);
+              acc = __ffma2_rn(q[4 * i + 2], bf16x2_f32(w.z), acc);
+              acc = __ffma2_rn(q[4 * i + 3], bf16x2_f32(w.w), acc);
+            }
+          }
+          sc[u] = (acc.x + acc.y) * qscale;
+          m = fmaxf(m, sc[u]);
+        }
+      }
+      float z = 0.f;
+      float2 o[DMAX / 2];
+#pragma unroll
+      for (int c = 0; c < DMAX / 2; ++c) o[c] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kMaxL; ++u) {
+        if (u < L && sc[u] != -INFINITY) {
+          const float p = ex2(sc[u] - m);
+          z += p;
+          const float2 p2 = make_float2(p, p);
+          const uint4* v4 = reinterpret_cast<const uint4*>(vseq + (size_t)u * Hkv * d);
+#pragma unroll
+          for (int i = 0; i < DMAX / 8; ++i) {
+            if (8 * i < d) {
+              const uint4 w = v4[i];
+              o[4 * i] = __ffma2_rn(p2, bf16x2_f32(w.x), o[4 * i]);
+              o[4 * i + 1] = __ffma2_rn(p2, bf16x2_f32(w.y), o[4 * i + 1]);
+              o[4 * i + 2] = __ffma2_rn(p2, bf16x2_f32(w.z), o[4 * i + 2]);
+              o[4 * i + 3] = __ffma2_rn(p2, bf16x2_f32(w.w), o[4 * i + 3]);
+            }
+          }
+        }
+      }
+      const float inv = z > 0.f ? 1.0f / z : 0.f;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o.ptr) + (b0 + s) * a.o.stride_b +
+                            (int64_t)t * a.o.stride_n + (int64_t)h * a.o.stride_h;
+#pragma unroll
+      for (int i = 0; i < DMAX / 8; ++i)
+        if (8 * i < d) {
+          uint4 w;
+          w.x = pack2_bf16(o[4 * i].x * inv, o[4 * i].y * inv);
+          w.y = pack2_bf16(o[4 * i + 1].x * inv, o[4 * i + 1].y * inv);
+          w.z = pack2_bf16(o[4 * i + 2].x * inv, o[4 * i + 2].y * inv);
+          w.w = pack2_bf16(o[4 * i + 3].x * inv, o[4 * i + 3].y * inv);
+          reinterpret_cast<uint4*>(orow)[i] = w;
+        }
+      lse_s[(s * Hq + h) * L + t] = z > 0.f ? (m + __log2f(z)) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
+    // LSE rows (b, h, 0..L-1) of the batch in memory order
+    const int nl = sb * Hq * L;
+    for (int idx = threadIdx.x; idx < nl; idx += kThreads) {
+      const int t = idx % L;
+      const int bh = idx / L;  // s * Hq + h
+      a.lse[((b0 + bh / Hq) * Hq + bh % Hq) * a.lse_ld + t] = lse_s[idx];
+    }
+    __syncthreads();  // lse_s and this stage are free again
+  }
+}
+
+// The [B, L, H, d] operand x as a TMA map with box (d, H, L, SB).
+rm_status staged_map(CUtensorMap* m, const rm_tensor& x, int64_t B, int L, int H, int d, int SB) {
+  const int64_t dims[5] = {d, H, L, B, 1};
+  const int64_t strides[4] = {x.stride_h * 2, x.stride_n * 2, x.stride_b * 2, x.stride_b * 2};
+  const int box[5] = {d, H, L, SB, 1};
+  return encode_copy_map(m, x.ptr, 2, dims, strides, box);
+}
+
+// Launches the TMA-staged kernel if the problem fits it; false (nothing
+// launched) otherwise, and the caller takes the one-thread-per-row kernel.
+bool try_launch_staged(const AttnArgs& a, int q_rank, int kv_rank, int64_t L, cudaStream_t stream,
+                       cudaError_t* err) {
+  if (a.B < 1 || a.Hq > 256 || a.Hkv > 256 || a.d % 8 || a.d > kMaxD || L > kMaxL) return false;
+  // TMA strides: nonzero multiples of 16 bytes; 16-byte aligned bases
+  for (const rm_tensor* x : {&a.q, &a.k, &a.v})
+    if (x->stride_b <= 0 || x->stride_n <= 0 || x->stride_h <= 0 || ((uintptr_t)x->ptr & 15))
+      return false;
+  int SB = 64;
+  while (SB > 1 && staged_layout(SB, (int)L, a.Hq, a.Hkv, a.d).stage_bytes > kStagedStageBudget)
+    --SB;
+  const StagedLayout g = staged_layout(SB, (int)L, a.Hq, a.Hkv, a.d);
+  if (g.stage_bytes > kStagedStageBudget) return false;
+  CUtensorMap mq, mk, mv;
+  if (staged_map(&mq, a.q, a.B, (int)L, a.Hq, a.d, SB) != RM_OK ||
+      staged_map(&mk, a.k, a.B, (int)L, a.Hkv, a.d, SB) != RM_OK ||
+      staged_map(&mv, a.v, a.B, (int)L, a.Hkv, a.d, SB) != RM_OK)
+    return false;
+  const int64_t nbatch = ((int64_t)a.B + SB - 1) / SB;
+  const bool narrow = a.d <= 32;
+  const int64_t cap = (int64_t)num_sms() * (narrow ? kStagedCtasPerSm : 1);
+  const unsigned grid = (unsigned)(nbatch < cap ? nbatch : cap);
+  // every batch of each operand one contiguous run (dense [B, L, H, d])
+  auto dense = [&](const rm_tensor& x, int H) {
+    return x.stride_h == a.d && x.stride_n == (int64_t)H * a.d && x.stride_b == L * H * a.d;
+  };
+  const int contiguous = dense(a.q, a.Hq) && dense(a.k, a.Hkv) && dense(a.v, a.Hkv) &&
+                         a.k.stride_b == a.v.stride_b;
+  auto kern = narrow ? small_seq_tma_kernel<32> : small_seq_tma_kernel<64>;
+  *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
+  if (*err != cudaSuccess) return true;
+  kern<<<grid, kThreads, g.total, stream>>>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous,
+                                            tc_wait_limit());
+  *err = cudaGetLastError();
+  return true;
+}
+
 template <typename T, int DMAX, bool VEC>
 cudaError_t launch(const AttnArgs& a, int q_rank, int kv_rank, int64_t total, cudaStream_t stream) {
   const int64_t need = (total + kThreads - 1) / kThreads;
@@ -193,6 +476,9 @@ cudaError_t launch_small_seq_fwd(const AttnArgs& a, int q_rank, int kv_rank, int
                    (a.o_f32 || (a.o.stride_b % 8 == 0 && a.o.stride_n % 8 == 0 &&
                                 a.o.stride_h % 8 == 0 && (uintptr_t)a.o.ptr % 16 == 0));
   ProfScope ps("small_seq_fwd", stream);
+  cudaError_t err = cudaSuccess;
+  if (bf16 && vec && !a.o_f32 && try_launch_staged(a, q_rank, kv_rank, L, stream, &err))
+    return err;
   return bf16 ? launch_t<__nv_bfloat16>(a, q_rank, kv_rank, total, vec, stream)
               : launch_t<float>(a, q_rank, kv_rank, total, vec, stream);
 }

@@ -93,9 +93,11 @@ def test_lse_merge(rm, out_dtype, n, B, H, Nq, d):
     assert np.all(np.isneginf(np64(l)[..., 1]))
 
 
-def test_lse_merge_in_place(rm):
-    o_parts = [synthetic.tensor(700 + i, (1, 50, 2, 32)).cuda() for i in range(3)]
-    lse_parts = [synthetic.tensor(710 + i, (1, 2, 50)).cuda() for i in range(3)]
+@pytest.mark.parametrize("n,Nq,H,d", [(3, 50, 2, 32), (2, 1001, 3, 128), (2, 517, 2, 64)])
+def test_lse_merge_in_place(rm, n, Nq, H, d):
+    # several rows per warp pass for two partials: row counts that leave a pass partly empty
+    o_parts = [synthetic.tensor(700 + i, (1, Nq, H, d)).cuda() for i in range(n)]
+    lse_parts = [synthetic.tensor(710 + i, (1, H, Nq)).cuda() for i in range(n)]
     ref_o, ref_l = omerge.lse_merge([np64(o) for o in o_parts], [np64(l) for l in lse_parts])
     rm.lse_merge(o_parts, lse_parts, torch.float32, out=o_parts[0], lse_out=lse_parts[0])
     assert_max_abs(np64(o_parts[0]), ref_o, F32_TOL)
