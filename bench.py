@@ -423,9 +423,34 @@ def hbm_row(rm, fn, reps, flush, nbytes, hbm, peak_src, shape):
             "timing": "kernel device time (per-launch CUDA events)"}
 
 
-def extras(rm, peaks, peak_src, dev, flush):
-    out = {}
+def extras(rm, peaks, peak_src, dev, flush, only=None):
+    """The extra measurements, by group; `only` runs one group (for a
+    profiler run of one kernel family on its own workload)."""
     hbm = peaks["hbm_gbs"]
+    groups = {
+        "merge": lambda: merge_lines(rm, dev, flush, hbm, peak_src),
+        "repack": lambda: repack_line(rm, dev, flush, hbm, peak_src),
+        "striped_128k": lambda: striped_lines(rm, dev, flush, peaks, hbm, peak_src),
+        "tabular_row": lambda: {"tabular_row_fwd": tabular(rm, flush, hbm, peak_src, "row")},
+        "tabular_feature": lambda: {"tabular_feature_fwd": tabular(rm, flush, hbm, peak_src,
+                                                                   "feature")},
+        "usp": lambda: {"usp_16k_fwd_bwd": usp_line(rm, flush, peaks, peak_src)},
+        "mesh2d": lambda: {"mesh2d_128k_fwd_bwd": mesh2d_line(rm, flush, peaks, peak_src)},
+    }
+    out = {}
+    for name, fn in groups.items():
+        if only is None or name == only:
+            out.update(fn())
+            torch.cuda.empty_cache()
+    return out
+
+
+EXTRA_GROUPS = ("merge", "repack", "striped_128k", "tabular_row", "tabular_feature", "usp",
+                "mesh2d")
+
+
+def merge_lines(rm, dev, flush, hbm, peak_src):
+    out = {}
     # LSE merge, striped-128k shapes: per rank 8 fp32 partials [16384, 16, 128] + LSE, 8 ranks
     Lr, H, d, P = 16384, 16, 128, 8
     o_parts = [torch.randn(1, P * Lr, H, d, device=dev) for _ in range(P)]
@@ -443,7 +468,10 @@ def extras(rm, peaks, peak_src, dev, flush):
     nbytes = 3 * P * Lr * H * d * 4 + 3 * H * P * Lr * 4
     out["lse_merge_pairwise"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
                                         "2 partials x [1, 131072, 16, 128] fp32 -> fp32 in place")
-    del o_parts, lse_parts, o_out, lse_out
+    return out
+
+
+def repack_line(rm, dev, flush, hbm, peak_src):
     # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and the fused K|V (8 K heads
     # then 8 V heads) of the same shape, seq -> head, one call each
     x = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
@@ -452,9 +480,13 @@ def extras(rm, peaks, peak_src, dev, flush):
     y2 = torch.empty_like(y)
     fn = lambda: (rm.seq_head_repack(x, 8, out=y), rm.seq_head_repack(kv, 8, out=y2))
     nbytes = 2 * (x.numel() + kv.numel()) * 2
-    out["repack"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
-                            "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> [8, 262144, 2, 128] bf16")
-    del x, kv, y, y2
+    return {"repack": hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                              "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> "
+                              "[8, 262144, 2, 128] bf16")}
+
+
+def striped_lines(rm, dev, flush, peaks, hbm, peak_src):
+    out = {}
     # the causal striped 128k forward (fused ring over 8 virtual ranks)
     w3 = synthetic.STRIPED_128K
     q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
@@ -475,10 +507,6 @@ def extras(rm, peaks, peak_src, dev, flush):
     nbytes = 2 * q.numel() * 2
     out["permute"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
                              "striped P=8 [1, 131072, 16, 128] bf16")
-    del q, k, v, o, lse, o2
-    out["tabular_row_fwd"], out["tabular_feature_fwd"] = tabular(rm, flush, hbm, peak_src)
-    out["usp_16k_fwd_bwd"] = usp_line(rm, flush, peaks, peak_src)
-    out["mesh2d_128k_fwd_bwd"] = mesh2d_line(rm, flush, peaks, peak_src)
     return out
 
 
@@ -550,17 +578,27 @@ def usp_line(rm, flush, peaks, peak_src):
 EX2_PER_CLK_SM = 16
 
 
-def tabular(rm, flush, hbm, peak_src):
+def tabular(rm, flush, hbm, peak_src, axis):
     """The tabular workload.  Row axis (20 sequences of 150000 rows, d = 24
     padded to 32, non-causal fused ring over 8 contiguous shards on strided
     views): TFLOP/s of its 4*d flops per pair against the tensor peak, and
     exponentials per second against the SFU rate (the d = 24 path does only
     96 MMA flops per exponential).  Feature axis (600000 sequences of 5
     tokens): GB/s of its algorithmic traffic (read Q, K, V, write O, LSE)
-    against HBM."""
+    against HBM.  `axis` is "row" or "feature"."""
     w = synthetic.TABULAR
     q, k, v = (t.cuda() for t in synthetic.tabular_inputs(w))
     R, F, E, H = w.rows, w.features, w.embed, w.heads
+    if axis == "feature":
+        fview = lambda x: x.view(w.batch * R, F, H, E // H)
+        fo = torch.empty(w.batch * R, F, H, E // H, dtype=torch.bfloat16, device="cuda")
+        flse = torch.empty(w.batch * R, H, F, device="cuda")
+        fn = lambda: rm.attn_block_fwd(fview(q), fview(k), fview(v), N=F, P=1,
+                                       layout="contiguous", causal=False, q_rank=0, kv_rank=0,
+                                       out=fo, lse=flse)
+        nbytes = 4 * q.numel() * 2 + flse.numel() * 4
+        return hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
+                       f"{w.batch * R * H} sequences x {F} tokens, d={E // H}")
     view = lambda x: x.view(w.batch, R, F * H, E // H)
     o = torch.empty(w.batch, R, F * H, E // H, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(w.batch, F * H, R, device="cuda")
@@ -579,16 +617,7 @@ def tabular(rm, flush, hbm, peak_src):
            "exp_per_s": round(ex2_rate / 1e12, 3), "exp_unit": "T exp2/s",
            "exp_frac": round(ex2_rate / ex2_peak, 4),
            "exp_peak_source": f"derived: {EX2_PER_CLK_SM}/clk/SM x {props.multi_processor_count} SMs x 1965 MHz"}
-    del o, lse
-    fview = lambda x: x.view(w.batch * R, F, H, E // H)
-    fo = torch.empty(w.batch * R, F, H, E // H, dtype=torch.bfloat16, device="cuda")
-    flse = torch.empty(w.batch * R, H, F, device="cuda")
-    fn = lambda: rm.attn_block_fwd(fview(q), fview(k), fview(v), N=F, P=1, layout="contiguous",
-                                   causal=False, q_rank=0, kv_rank=0, out=fo, lse=flse)
-    nbytes = 4 * q.numel() * 2 + flse.numel() * 4
-    feat = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
-                   f"{w.batch * R * H} sequences x {F} tokens, d={E // H}")
-    return row, feat
+    return row
 
 
 # ---------------------------------------------------------------------------
@@ -707,9 +736,20 @@ def main():
                     help="query heads in the oracle sample of cpu_baseline")
     ap.add_argument("--ref-sample-heads", type=int, default=4,
                     help="query heads in each --impl reference step")
+    ap.add_argument("--case", choices=EXTRA_GROUPS, default=None,
+                    help="run only this group of the extra measurements (no step, no baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case:
+        from sequence_attention_rm_b200 import rm
+        peaks, peak_src = load_peaks()
+        dev = torch.device("cuda", 0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        print(json.dumps({"case": args.case,
+                          "extras": extras(rm, peaks, peak_src, dev, flush, only=args.case)}),
+              flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

@@ -1,7 +1,7 @@
 // Ring backward that allocates nothing.
 //
-// The ring backward needs scratch device memory (the row term delta and the
-// fp32 dQ accumulator).  Most callers pass a workspace they allocated; some
+// The ring backward needs scratch device memory: the row term
+// delta = rowsum(dO * O), one fp32 value per (batch, query head, token).  Most callers pass a workspace they allocated; some
 // cannot: for example a runtime that reserved all device memory for its own
 // pool at start-up and hands out no raw allocations, or code that must not
 // call cudaMalloc because it would synchronise the device.  For them this
@@ -76,8 +76,8 @@ extern "C" rm_status rm_ring_attn_bwd_noalloc(const rm_attn_desc* desc, rm_tenso
   void* scratch = nullptr;
   s = rm::scratch_address(&scratch);
   if (s != RM_OK) return s;
-  // the ring backward zero-fills the dQ accumulator and overwrites delta in
-  // the scratch before reading them, so the previous call's contents are harmless
+  // the ring backward writes delta into the scratch before reading it, so the
+  // previous call's contents are harmless
   return rm_ring_attn_bwd(desc, q, k, v, o, lse, dout, dq, dk, dv, scratch, rm::kScratchBytes,
                           stream);
 }

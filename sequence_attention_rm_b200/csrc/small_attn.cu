@@ -162,29 +162,33 @@ __global__ void __launch_bounds__(kThreads) small_seq_attn_kernel(AttnArgs a, in
   }
 }
 
-// bf16 operands with 16-byte rows: persistent blocks (two per SM) walk
-// batches of SB whole sequences through a two-stage shared-memory ring.  For
-// each batch one thread issues three asynchronous copies -- the Q, K and V
-// rows of the batch -- onto the stage's mbarrier, one batch ahead of the
-// batch being computed, so staging costs no per-element index arithmetic and
-// the next batch is in flight during the math.  Dense operands take one bulk
-// copy each (a batch is one run of memory); strided views take TMA boxes
-// (d, H, L, SB) of their [B, L, H, d] maps, which read as zero past the last
-// sequence.  One thread per
-// (sequence, query token, head) scores its keys from shared memory with
-// packed fp32 FMAs, writes its O row with 16-byte stores and parks its LSE in
-// shared memory, from which the block writes the [B, H, L] LSE rows in order.
+// bf16 operands with 16-byte rows: a warp-specialised persistent kernel.
+// Batches of SB whole sequences flow through a ring of shared-memory stages:
+// a producer warp issues, per batch, three asynchronous copies -- the Q, K
+// and V rows of the batch -- onto the stage's "full" mbarrier, running up to
+// kStagedStages batches ahead; eight consumer warps attend and release the
+// stage on its "empty" mbarrier.  Dense operands take one bulk copy each (a
+// batch is one run of memory); strided views take TMA boxes (D, H, L, SB) of
+// their [B, L, H, D] maps, which read as zero past the last sequence.  So
+// staging costs no per-element index arithmetic and no block-wide barrier.
+// SB is chosen so that SB * L * Hq <= 256: each consumer thread owns one
+// fixed (sequence, query token, head) slot of every batch, decoded once,
+// scores its keys from shared memory with packed fp32 FMAs, and writes its O
+// row (16-byte stores) and its LSE (a batch's LSE values are one contiguous
+// range of the [B, H, L] output, so a warp's stores share few sectors).
+// Only when L * Hq > 256 (then SB = 1) does a thread take several slots.
 struct StagedLayout {
   int SB;
-  uint32_t q_bytes, kv_bytes;  // box bytes (the TMA transaction sizes)
+  uint32_t q_bytes, kv_bytes;  // box bytes of a full batch (the TMA transaction sizes)
   uint32_t off_k, off_v;       // within a stage
   uint32_t stage_bytes;
-  uint32_t off_lse, off_bar, total;
+  uint32_t off_bar, total;
 };
 
-constexpr int kStagedStages = 2;
-constexpr int kStagedCtasPerSm = 2;
-constexpr uint32_t kStagedStageBudget = 48 * 1024;  // one stage's three boxes
+constexpr int kStagedStages = 3;
+constexpr int kConsumerWarps = kThreads / 32;
+constexpr int kStagedThreads = kThreads + 32;     // consumers + one producer warp
+constexpr uint32_t kStagedSmemPerSm = 220 * 1024;  // shared memory the blocks of one SM share
 
 __host__ __device__ inline uint32_t round128(uint32_t x) { return (x + 127u) & ~127u; }
 
@@ -196,9 +200,8 @@ __host__ __device__ inline StagedLayout staged_layout(int SB, int L, int Hq, int
   g.off_k = round128(g.q_bytes);
   g.off_v = g.off_k + round128(g.kv_bytes);
   g.stage_bytes = g.off_v + round128(g.kv_bytes);
-  g.off_lse = kStagedStages * g.stage_bytes;
-  g.off_bar = (g.off_lse + (uint32_t)SB * Hq * L * 4 + 7u) & ~7u;
-  g.total = g.off_bar + 8 * kStagedStages;
+  g.off_bar = kStagedStages * g.stage_bytes;
+  g.total = g.off_bar + 16 * kStagedStages;  // full and empty barrier per stage
   return g;
 }
 
@@ -214,154 +217,187 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
-// bf16 pair (low, high halves of a 32-bit word) -> fp32 pair
-__device__ __forceinline__ float2 bf16x2_f32(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+// acc + a.lo * b.lo + a.hi * b.hi for two bf16 pairs a, b (32-bit words), with
+// fp32 accumulation: the mixed-precision FMA takes the bf16 halves directly
+// (a bf16 x bf16 product is exact in fp32), so nothing is unpacked.
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "=f"(r)
+      : "r"(a), "r"(b), "f"(acc));
+  return r;
+}
+// (o.x, o.y) += p * (v.lo, v.hi), p a bf16 in the low half of a 16-bit word
+__device__ __forceinline__ void axpy2_bf16(uint16_t p, uint32_t v, float2& o) {
+  asm("{\n\t.reg .b16 vl, vh;\n\t"
+      "mov.b32 {vl, vh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, %3, vl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, %3, vh, %1;\n\t}"
+      : "+f"(o.x), "+f"(o.y)
+      : "r"(v), "h"(p));
 }
 
-template <int DMAX>
-__global__ void __launch_bounds__(kThreads, DMAX <= 32 ? kStagedCtasPerSm : 1)
+// Registers per thread the launch bounds allow: two blocks per SM up to
+// D = 32, one block at D = 64.
+template <int D>
+constexpr int staged_blocks_per_sm() { return D <= 32 ? 2 : 1; }
+
+template <int D, int LMAX>
+__global__ void __launch_bounds__(kStagedThreads, staged_blocks_per_sm<D>())
     small_seq_tma_kernel(const __grid_constant__ CUtensorMap mq,
                          const __grid_constant__ CUtensorMap mk,
                          const __grid_constant__ CUtensorMap mv, AttnArgs a, int q_rank,
                          int kv_rank, StagedLayout g, int contiguous, long long wait_limit) {
   extern __shared__ __align__(128) unsigned char smem[];
   using namespace tc;
-  const LayoutMap lay = make_layout(a.layout, a.N, a.P);
-  const int L = (int)lay.L;
-  const int d = a.d;
+  constexpr int S = kStagedStages;
+  const int L = (int)(a.N / a.P);
   const int Hq = a.Hq, Hkv = a.Hkv;
-  const int group = Hq / Hkv;
-  float* lse_s = reinterpret_cast<float*>(smem + g.off_lse);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+  uint64_t* empty = full + S;
   const int64_t nbatch = ((int64_t)a.B + g.SB - 1) / g.SB;
   const int64_t mine =
       nbatch > blockIdx.x ? (nbatch - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if ((smem_u32(smem) & 127u) != 0) {  // TMA boxes need a 128-byte aligned destination
     if (threadIdx.x == 0) report_status(a.status, kStatusSmemAlign);
     return;
   }
   if (threadIdx.x == 0) {
-    for (int st = 0; st < kStagedStages; ++st) mbar_init(bars + st, 1);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(full + st, 1);
+      mbar_init(empty + st, kConsumerWarps);
+    }
     fence_barrier_init();
   }
   __syncthreads();
-  auto issue = [&](int64_t k) {  // batch k of this block into stage k % 2
-    unsigned char* st = smem + (k & 1) * g.stage_bytes;
-    uint64_t* bar = bars + (k & 1);
-    const int bc = (int)((blockIdx.x + k * gridDim.x) * g.SB);
-    if (contiguous) {
-      // the batch's rows of each operand are one run: sb sequences of L*H*d
-      const int sb = a.B - bc < g.SB ? a.B - bc : g.SB;
-      const uint32_t qb = g.q_bytes / g.SB * sb, kvb = g.kv_bytes / g.SB * sb;
-      mbar_arrive_expect_tx(bar, qb + 2 * kvb);
-      const size_t off = (size_t)bc * a.q.stride_b * 2, koff = (size_t)bc * a.k.stride_b * 2;
-      bulk_load(st, reinterpret_cast<const char*>(a.q.ptr) + off, qb, bar);
-      bulk_load(st + g.off_k, reinterpret_cast<const char*>(a.k.ptr) + koff, kvb, bar);
-      bulk_load(st + g.off_v, reinterpret_cast<const char*>(a.v.ptr) + koff, kvb, bar);
-    } else {
-      mbar_arrive_expect_tx(bar, g.q_bytes + 2 * g.kv_bytes);
-      tma_load_5d(st, &mq, bar, 0, 0, 0, bc, 0);
-      tma_load_5d(st + g.off_k, &mk, bar, 0, 0, 0, bc, 0);
-      tma_load_5d(st + g.off_v, &mv, bar, 0, 0, 0, bc, 0);
-    }
-  };
-  if (threadIdx.x == 0 && mine > 0) issue(0);
 
-  const float qscale = a.scale * kLog2e;  // scores in log2 units
-  for (int64_t k = 0; k < mine; ++k) {
-    // the other stage was last read by batch k - 1, which every thread has
-    // finished (barrier at the end of the previous pass)
-    if (threadIdx.x == 0 && k + 1 < mine) {
-      fence_proxy_async_smem();  // this thread's reads of the stage before the TMA writes
-      issue(k + 1);
-    }
-    // a timeout ends the whole block together (no thread may be left at a
-    // barrier the others have passed)
-    const bool ok = mbar_wait(bars + (k & 1), (uint32_t)((k >> 1) & 1), wait_limit, a.status);
-    if (!__syncthreads_and(ok)) {
-      // boxes may still be landing: wait for them once more (bounded) before
-      // the block's shared memory is given up
-      if (threadIdx.x == 0) {
-        mbar_wait(bars + (k & 1), (uint32_t)((k >> 1) & 1), wait_limit, a.status);
-        if (k + 1 < mine)
-          mbar_wait(bars + ((k + 1) & 1), (uint32_t)(((k + 1) >> 1) & 1), wait_limit, a.status);
+  if (warp == kConsumerWarps) {
+    // ---- producer ----------------------------------------------------------
+    if (lane != 0) return;
+    int64_t issued = 0;
+    for (; issued < mine; ++issued) {
+      const int st = (int)(issued % S);
+      if (issued >= S &&
+          !mbar_wait(empty + st, (uint32_t)((issued / S - 1) & 1), wait_limit, a.status))
+        break;
+      unsigned char* dst = smem + st * g.stage_bytes;
+      const int bc = (int)((blockIdx.x + issued * gridDim.x) * g.SB);
+      if (contiguous) {
+        // the batch's rows of each operand are one run: sb sequences of L*H*D
+        const int sb = a.B - bc < g.SB ? a.B - bc : g.SB;
+        const uint32_t qb = g.q_bytes / g.SB * sb, kvb = g.kv_bytes / g.SB * sb;
+        mbar_arrive_expect_tx(full + st, qb + 2 * kvb);
+        const size_t qoff = (size_t)bc * a.q.stride_b * 2, koff = (size_t)bc * a.k.stride_b * 2;
+        bulk_load(dst, reinterpret_cast<const char*>(a.q.ptr) + qoff, qb, full + st);
+        bulk_load(dst + g.off_k, reinterpret_cast<const char*>(a.k.ptr) + koff, kvb, full + st);
+        bulk_load(dst + g.off_v, reinterpret_cast<const char*>(a.v.ptr) + koff, kvb, full + st);
+      } else {
+        mbar_arrive_expect_tx(full + st, g.q_bytes + 2 * g.kv_bytes);
+        tma_load_5d(dst, &mq, full + st, 0, 0, 0, bc, 0);
+        tma_load_5d(dst + g.off_k, &mk, full + st, 0, 0, 0, bc, 0);
+        tma_load_5d(dst + g.off_v, &mv, full + st, 0, 0, 0, bc, 0);
       }
-      return;
     }
-    const unsigned char* st = smem + (k & 1) * g.stage_bytes;
-    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(st);
-    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(st + g.off_k);
-    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(st + g.off_v);
+    if (issued < mine) {
+      // a timeout: the copies already issued may still be landing; wait for
+      // the latest one of every stage (bounded) before leaving
+      for (int64_t j = issued - 1; j >= 0 && j >= issued - S; --j)
+        mbar_wait(full + (int)(j % S), (uint32_t)((j / S) & 1), wait_limit, a.status);
+    }
+    return;
+  }
+
+  // ---- consumers -------------------------------------------------------------
+  const LayoutMap lay = make_layout(a.layout, a.N, a.P);
+  const int group = Hq / Hkv;
+  const float qscale = a.scale * kLog2e;  // scores in log2 units
+  const int slots = g.SB * L * Hq;        // (s, t, h) slots of a full batch, h fastest
+  // this thread's first slot, decoded once
+  const int h0 = threadIdx.x % Hq;
+  const int t0 = (threadIdx.x / Hq) % L;
+  const int s0 = threadIdx.x / (Hq * L);
+  for (int64_t k = 0; k < mine; ++k) {
+    const int st = (int)(k % S);
+    const bool ok = mbar_wait(full + st, (uint32_t)((k / S) & 1), wait_limit, a.status);
+    if (!__all_sync(0xffffffffu, ok)) return;  // a timeout ends the warp as a whole
+    const unsigned char* base = smem + st * g.stage_bytes;
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(base);
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(base + g.off_k);
+    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(base + g.off_v);
     const int64_t b0 = (blockIdx.x + k * gridDim.x) * g.SB;
     const int sb = (int)((int64_t)a.B - b0 < g.SB ? (int64_t)a.B - b0 : g.SB);
-    const int work = sb * L * Hq;
-    for (int idx = threadIdx.x; idx < work; idx += kThreads) {
-      const int h = idx % Hq;
-      const int r = idx / Hq;  // s * L + t
-      const int t = r % L;
-      const int s = r / L;
+    for (int idx = threadIdx.x; idx < slots; idx += kThreads) {
+      int h = h0, t = t0, s = s0;
+      if (idx != (int)threadIdx.x) {
+        h = idx % Hq;
+        t = (idx / Hq) % L;
+        s = idx / (Hq * L);
+      }
+      if (s >= sb) break;  // the last batch may hold fewer sequences
       const int kvh = h / group;
-      float2 q[DMAX / 2];
+      uint32_t q[D / 2];  // raw bf16 pairs
       {
-        const uint4* q4 = reinterpret_cast<const uint4*>(qs + ((size_t)r * Hq + h) * d);
+        const uint4* q4 = reinterpret_cast<const uint4*>(qs + ((size_t)(s * L + t) * Hq + h) * D);
 #pragma unroll
-        for (int i = 0; i < DMAX / 8; ++i) {
-          if (8 * i < d) {
-            const uint4 w = q4[i];
-            q[4 * i] = bf16x2_f32(w.x);
-            q[4 * i + 1] = bf16x2_f32(w.y);
-            q[4 * i + 2] = bf16x2_f32(w.z);
-            q[4 * i + 3] = bf16x2_f32(w.w);
-          }
+        for (int i = 0; i < D / 8; ++i) {
+          const uint4 w = q4[i];
+          q[4 * i] = w.x;
+          q[4 * i + 1] = w.y;
+          q[4 * i + 2] = w.z;
+          q[4 * i + 3] = w.w;
         }
       }
       const int64_t tq = lay.pos(q_rank, t);
-      const __nv_bfloat16* kseq = ks + ((size_t)s * L * Hkv + kvh) * d;  // key 0 of sequence s
-      const __nv_bfloat16* vseq = vs + ((size_t)s * L * Hkv + kvh) * d;
-      float sc[kMaxL];
+      const __nv_bfloat16* kseq = ks + ((size_t)s * L * Hkv + kvh) * D;  // key 0 of sequence s
+      const __nv_bfloat16* vseq = vs + ((size_t)s * L * Hkv + kvh) * D;
+      float sc[LMAX];
       float m = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < kMaxL; ++u) {
+      for (int u = 0; u < LMAX; ++u) {
         sc[u] = -INFINITY;
         if (u < L && (!a.causal || lay.pos(kv_rank, u) <= tq)) {
-          const uint4* k4 = reinterpret_cast<const uint4*>(kseq + (size_t)u * Hkv * d);
-          float2 acc = make_float2(0.f, 0.f);
+          const uint4* k4 = reinterpret_cast<const uint4*>(kseq + (size_t)u * Hkv * D);
+          float acc0 = 0.f, acc1 = 0.f;  // two chains
 #pragma unroll
-          for (int i = 0; i < DMAX / 8; ++i) {
-            if (8 * i < d) {
-              const uint4 w = k4[i];
-              acc = __ffma2_rn(q[4 * i], bf16x2_f32(w.x), acc);
-              acc = __ffma2_rn(q[4 * i + 1], bf16x2_f32(w.y), acc);
-              acc = __ffma2_rn(q[4 * i + 2], bf16x2_f32(w.z), acc);
-              acc = __ffma2_rn(q[4 * i + 3], bf16x2_f32(w.w), acc);
-            }
+          for (int i = 0; i < D / 8; ++i) {
+            const uint4 w = k4[i];
+            acc0 = dot2_bf16(q[4 * i], w.x, acc0);
+            acc1 = dot2_bf16(q[4 * i + 1], w.y, acc1);
+            acc0 = dot2_bf16(q[4 * i + 2], w.z, acc0);
+            acc1 = dot2_bf16(q[4 * i + 3], w.w, acc1);
           }
-          sc[u] = (acc.x + acc.y) * qscale;
+          sc[u] = (acc0 + acc1) * qscale;
           m = fmaxf(m, sc[u]);
         }
       }
+      // O accumulates bf16(p) * V in fp32 (the probabilities enter the
+      // product in bf16, as they do in the tensor-core kernels' P V); the
+      // normaliser z sums the fp32 p
       float z = 0.f;
-      float2 o[DMAX / 2];
+      float2 o[D / 2];
 #pragma unroll
-      for (int c = 0; c < DMAX / 2; ++c) o[c] = make_float2(0.f, 0.f);
+      for (int c = 0; c < D / 2; ++c) o[c] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < kMaxL; ++u) {
+      for (int u = 0; u < LMAX; ++u) {
         if (u < L && sc[u] != -INFINITY) {
           const float p = ex2(sc[u] - m);
           z += p;
-          const float2 p2 = make_float2(p, p);
-          const uint4* v4 = reinterpret_cast<const uint4*>(vseq + (size_t)u * Hkv * d);
+          const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+          const uint16_t ph = *reinterpret_cast<const uint16_t*>(&pb);
+          const uint4* v4 = reinterpret_cast<const uint4*>(vseq + (size_t)u * Hkv * D);
 #pragma unroll
-          for (int i = 0; i < DMAX / 8; ++i) {
-            if (8 * i < d) {
-              const uint4 w = v4[i];
-              o[4 * i] = __ffma2_rn(p2, bf16x2_f32(w.x), o[4 * i]);
-              o[4 * i + 1] = __ffma2_rn(p2, bf16x2_f32(w.y), o[4 * i + 1]);
-              o[4 * i + 2] = __ffma2_rn(p2, bf16x2_f32(w.z), o[4 * i + 2]);
-              o[4 * i + 3] = __ffma2_rn(p2, bf16x2_f32(w.w), o[4 * i + 3]);
-            }
+          for (int i = 0; i < D / 8; ++i) {
+            const uint4 w = v4[i];
+            axpy2_bf16(ph, w.x, o[4 * i]);
+            axpy2_bf16(ph, w.y, o[4 * i + 1]);
+            axpy2_bf16(ph, w.z, o[4 * i + 2]);
+            axpy2_bf16(ph, w.w, o[4 * i + 3]);
           }
         }
       }
@@ -369,30 +405,22 @@ __global__ void __launch_bounds__(kThreads, DMAX <= 32 ? kStagedCtasPerSm : 1)
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o.ptr) + (b0 + s) * a.o.stride_b +
                             (int64_t)t * a.o.stride_n + (int64_t)h * a.o.stride_h;
 #pragma unroll
-      for (int i = 0; i < DMAX / 8; ++i)
-        if (8 * i < d) {
-          uint4 w;
-          w.x = pack2_bf16(o[4 * i].x * inv, o[4 * i].y * inv);
-          w.y = pack2_bf16(o[4 * i + 1].x * inv, o[4 * i + 1].y * inv);
-          w.z = pack2_bf16(o[4 * i + 2].x * inv, o[4 * i + 2].y * inv);
-          w.w = pack2_bf16(o[4 * i + 3].x * inv, o[4 * i + 3].y * inv);
-          reinterpret_cast<uint4*>(orow)[i] = w;
-        }
-      lse_s[(s * Hq + h) * L + t] = z > 0.f ? (m + __log2f(z)) * kLn2 : -INFINITY;
+      for (int i = 0; i < D / 8; ++i) {
+        uint4 w;
+        w.x = pack2_bf16(o[4 * i].x * inv, o[4 * i].y * inv);
+        w.y = pack2_bf16(o[4 * i + 1].x * inv, o[4 * i + 1].y * inv);
+        w.z = pack2_bf16(o[4 * i + 2].x * inv, o[4 * i + 2].y * inv);
+        w.w = pack2_bf16(o[4 * i + 3].x * inv, o[4 * i + 3].y * inv);
+        reinterpret_cast<uint4*>(orow)[i] = w;
+      }
+      a.lse[((b0 + s) * Hq + h) * a.lse_ld + t] = z > 0.f ? (m + __log2f(z)) * kLn2 : -INFINITY;
     }
-    __syncthreads();
-    // LSE rows (b, h, 0..L-1) of the batch in memory order
-    const int nl = sb * Hq * L;
-    for (int idx = threadIdx.x; idx < nl; idx += kThreads) {
-      const int t = idx % L;
-      const int bh = idx / L;  // s * Hq + h
-      a.lse[((b0 + bh / Hq) * Hq + bh % Hq) * a.lse_ld + t] = lse_s[idx];
-    }
-    __syncthreads();  // lse_s and this stage are free again
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + st);  // this warp is done with the stage
   }
 }
 
-// The [B, L, H, d] operand x as a TMA map with box (d, H, L, SB).
+// The [B, L, H, D] operand x as a TMA map with box (D, H, L, SB).
 rm_status staged_map(CUtensorMap* m, const rm_tensor& x, int64_t B, int L, int H, int d, int SB) {
   const int64_t dims[5] = {d, H, L, B, 1};
   const int64_t strides[4] = {x.stride_h * 2, x.stride_n * 2, x.stride_b * 2, x.stride_b * 2};
@@ -400,41 +428,61 @@ rm_status staged_map(CUtensorMap* m, const rm_tensor& x, int64_t B, int L, int H
   return encode_copy_map(m, x.ptr, 2, dims, strides, box);
 }
 
-// Launches the TMA-staged kernel if the problem fits it; false (nothing
+template <int D>
+cudaError_t launch_staged(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const AttnArgs& a, int q_rank, int kv_rank, const StagedLayout& g,
+                          int contiguous, int64_t nbatch, cudaStream_t stream) {
+  // the key loops unroll to 8 or 16 keys
+  auto kern = a.N / a.P <= 8 ? small_seq_tma_kernel<D, 8> : small_seq_tma_kernel<D, kMaxL>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
+  if (e != cudaSuccess) return e;
+  const int per_sm = (int)(kStagedSmemPerSm / g.total) < staged_blocks_per_sm<D>()
+                         ? (int)(kStagedSmemPerSm / g.total)
+                         : staged_blocks_per_sm<D>();
+  const int64_t cap = (int64_t)num_sms() * (per_sm < 1 ? 1 : per_sm);
+  const unsigned grid = (unsigned)(nbatch < cap ? nbatch : cap);
+  kern<<<grid, kStagedThreads, g.total, stream>>>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous,
+                                                  tc_wait_limit());
+  return cudaGetLastError();
+}
+
+// Launches the staged kernel if the problem fits it; false (nothing
 // launched) otherwise, and the caller takes the one-thread-per-row kernel.
 bool try_launch_staged(const AttnArgs& a, int q_rank, int kv_rank, int64_t L, cudaStream_t stream,
                        cudaError_t* err) {
-  if (a.B < 1 || a.Hq > 256 || a.Hkv > 256 || a.d % 8 || a.d > kMaxD || L > kMaxL) return false;
+  if (a.B < 1 || a.Hq > 256 || a.Hkv > 256 || L > kMaxL || (a.d != 24 && a.d != 32 && a.d != 64))
+    return false;
   // TMA strides: nonzero multiples of 16 bytes; 16-byte aligned bases
   for (const rm_tensor* x : {&a.q, &a.k, &a.v})
     if (x->stride_b <= 0 || x->stride_n <= 0 || x->stride_h <= 0 || ((uintptr_t)x->ptr & 15))
       return false;
-  int SB = 64;
-  while (SB > 1 && staged_layout(SB, (int)L, a.Hq, a.Hkv, a.d).stage_bytes > kStagedStageBudget)
-    --SB;
+  // one slot per consumer thread, and every stage within a third of the
+  // shared memory the SM's blocks share
+  int SB = (int)(kThreads / (L * a.Hq));
+  if (SB < 1) SB = 1;
+  if (SB > 256) SB = 256;
+  while (SB > 1 && staged_layout(SB, (int)L, a.Hq, a.Hkv, a.d).total > kStagedSmemPerSm / 2) --SB;
   const StagedLayout g = staged_layout(SB, (int)L, a.Hq, a.Hkv, a.d);
-  if (g.stage_bytes > kStagedStageBudget) return false;
+  if (g.total > kStagedSmemPerSm) return false;
   CUtensorMap mq, mk, mv;
   if (staged_map(&mq, a.q, a.B, (int)L, a.Hq, a.d, SB) != RM_OK ||
       staged_map(&mk, a.k, a.B, (int)L, a.Hkv, a.d, SB) != RM_OK ||
       staged_map(&mv, a.v, a.B, (int)L, a.Hkv, a.d, SB) != RM_OK)
     return false;
-  const int64_t nbatch = ((int64_t)a.B + SB - 1) / SB;
-  const bool narrow = a.d <= 32;
-  const int64_t cap = (int64_t)num_sms() * (narrow ? kStagedCtasPerSm : 1);
-  const unsigned grid = (unsigned)(nbatch < cap ? nbatch : cap);
   // every batch of each operand one contiguous run (dense [B, L, H, d])
   auto dense = [&](const rm_tensor& x, int H) {
     return x.stride_h == a.d && x.stride_n == (int64_t)H * a.d && x.stride_b == L * H * a.d;
   };
   const int contiguous = dense(a.q, a.Hq) && dense(a.k, a.Hkv) && dense(a.v, a.Hkv) &&
                          a.k.stride_b == a.v.stride_b;
-  auto kern = narrow ? small_seq_tma_kernel<32> : small_seq_tma_kernel<64>;
-  *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
-  if (*err != cudaSuccess) return true;
-  kern<<<grid, kThreads, g.total, stream>>>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous,
-                                            tc_wait_limit());
-  *err = cudaGetLastError();
+  const int64_t nbatch = ((int64_t)a.B + SB - 1) / SB;
+  if (a.d == 24)
+    *err = launch_staged<24>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous, nbatch, stream);
+  else if (a.d == 32)
+    *err = launch_staged<32>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous, nbatch, stream);
+  else
+    *err = launch_staged<64>(mq, mk, mv, a, q_rank, kv_rank, g, contiguous, nbatch, stream);
   return true;
 }
 
