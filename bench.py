@@ -423,14 +423,17 @@ def hbm_row(rm, fn, reps, flush, nbytes, hbm, peak_src, shape):
             "timing": "kernel device time (per-launch CUDA events)"}
 
 
-def extras(rm, peaks, peak_src, dev, flush, only=None):
+def extras(rm, peaks, peak_src, dev, flush, only=None, small=False):
     """The extra measurements, by group; `only` runs one group (for a
-    profiler run of one kernel family on its own workload)."""
+    profiler run of one kernel family on its own workload).  `small` shrinks
+    the merge, repack and permute shapes (token counts / 8, / 8 and / 2; still
+    larger than L2) so that a multi-pass profiler capture holds at most about
+    1 GB on the device; their lines then name the smaller shapes."""
     hbm = peaks["hbm_gbs"]
     groups = {
-        "merge": lambda: merge_lines(rm, dev, flush, hbm, peak_src),
-        "repack": lambda: repack_line(rm, dev, flush, hbm, peak_src),
-        "striped_128k": lambda: striped_lines(rm, dev, flush, peaks, hbm, peak_src),
+        "merge": lambda: merge_lines(rm, dev, flush, hbm, peak_src, 8 if small else 1),
+        "repack": lambda: repack_line(rm, dev, flush, hbm, peak_src, 8 if small else 1),
+        "striped_128k": lambda: striped_lines(rm, dev, flush, peaks, hbm, peak_src, small),
         "tabular_row": lambda: {"tabular_row_fwd": tabular(rm, flush, hbm, peak_src, "row")},
         "tabular_feature": lambda: {"tabular_feature_fwd": tabular(rm, flush, hbm, peak_src,
                                                                    "feature")},
@@ -449,10 +452,11 @@ EXTRA_GROUPS = ("merge", "repack", "striped_128k", "tabular_row", "tabular_featu
                 "mesh2d")
 
 
-def merge_lines(rm, dev, flush, hbm, peak_src):
+def merge_lines(rm, dev, flush, hbm, peak_src, div=1):
     out = {}
     # LSE merge, striped-128k shapes: per rank 8 fp32 partials [16384, 16, 128] + LSE, 8 ranks
-    Lr, H, d, P = 16384, 16, 128, 8
+    Lr, H, d, P = 16384 // div, 16, 128, 8
+    n = P * Lr
     o_parts = [torch.randn(1, P * Lr, H, d, device=dev) for _ in range(P)]
     lse_parts = [torch.randn(1, H, P * Lr, device=dev) for _ in range(P)]
     o_out = torch.empty(1, P * Lr, H, d, dtype=torch.bfloat16, device=dev)
@@ -460,35 +464,43 @@ def merge_lines(rm, dev, flush, hbm, peak_src):
     fn = lambda: rm.lse_merge(o_parts, lse_parts, torch.bfloat16, out=o_out, lse_out=lse_out)
     nbytes = P * (P * Lr * H * d * 4 + H * P * Lr * 4) + P * Lr * H * d * 2 + H * P * Lr * 4
     out["lse_merge"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
-                               "8 partials x [1, 131072, 16, 128] fp32 -> bf16")
+                               f"8 partials x [1, {n}, 16, 128] fp32 -> bf16")
     # pairwise merge (the running-state form): fp32 O_acc <- merge(O_acc, O_new), in place
     acc, lacc = o_parts[0], lse_parts[0]
     fn = lambda: rm.lse_merge([acc, o_parts[1]], [lacc, lse_parts[1]], torch.float32, out=acc,
                               lse_out=lacc)
     nbytes = 3 * P * Lr * H * d * 4 + 3 * H * P * Lr * 4
     out["lse_merge_pairwise"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
-                                        "2 partials x [1, 131072, 16, 128] fp32 -> fp32 in place")
+                                        f"2 partials x [1, {n}, 16, 128] fp32 -> fp32 in place")
     return out
 
 
-def repack_line(rm, dev, flush, hbm, peak_src):
+def repack_line(rm, dev, flush, hbm, peak_src, div=1):
     # Ulysses repack, 256k-zigzag shapes: Q [8 x 32768, 16, 128] and the fused K|V (8 K heads
     # then 8 V heads) of the same shape, seq -> head, one call each
-    x = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
-    kv = torch.randn(8, 32768, 16, 128, device=dev).to(torch.bfloat16)
-    y = torch.empty(8, 8 * 32768, 2, 128, dtype=torch.bfloat16, device=dev)
+    Ln = 32768 // div
+    x = torch.randn(8, Ln, 16, 128, device=dev).to(torch.bfloat16)
+    kv = torch.randn(8, Ln, 16, 128, device=dev).to(torch.bfloat16)
+    y = torch.empty(8, 8 * Ln, 2, 128, dtype=torch.bfloat16, device=dev)
     y2 = torch.empty_like(y)
     fn = lambda: (rm.seq_head_repack(x, 8, out=y), rm.seq_head_repack(kv, 8, out=y2))
     nbytes = 2 * (x.numel() + kv.numel()) * 2
     return {"repack": hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
-                              "seq->head Q and fused K|V, each [8, 32768, 16, 128] -> "
-                              "[8, 262144, 2, 128] bf16")}
+                              f"seq->head Q and fused K|V, each [8, {Ln}, 16, 128] -> "
+                              f"[8, {8 * Ln}, 2, 128] bf16")}
 
 
-def striped_lines(rm, dev, flush, peaks, hbm, peak_src):
+def striped_lines(rm, dev, flush, peaks, hbm, peak_src, small=False):
     out = {}
-    # the causal striped 128k forward (fused ring over 8 virtual ranks)
     w3 = synthetic.STRIPED_128K
+    if small:  # the permute alone, on half the tokens
+        q = torch.randn(1, w3.N // 2, w3.Hq, w3.d, device=dev).to(torch.bfloat16)
+        o2 = torch.empty_like(q)
+        fn = lambda: rm.layout_permute(q, "striped", 8, out=o2)
+        out["permute"] = hbm_row(rm, fn, 10, flush, 2 * q.numel() * 2, hbm, peak_src,
+                                 f"striped P=8 [1, {w3.N // 2}, 16, 128] bf16")
+        return out
+    # the causal striped 128k forward (fused ring over 8 virtual ranks)
     q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
     k = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
     v = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
@@ -738,6 +750,8 @@ def main():
                     help="query heads in each --impl reference step")
     ap.add_argument("--case", choices=EXTRA_GROUPS, default=None,
                     help="run only this group of the extra measurements (no step, no baseline)")
+    ap.add_argument("--small", action="store_true",
+                    help="with --case: the smaller merge / repack / permute shapes (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -747,7 +761,8 @@ def main():
         dev = torch.device("cuda", 0)
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         print(json.dumps({"case": args.case,
-                          "extras": extras(rm, peaks, peak_src, dev, flush, only=args.case)}),
+                          "extras": extras(rm, peaks, peak_src, dev, flush, only=args.case,
+                                           small=args.small)}),
               flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
