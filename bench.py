@@ -17,15 +17,23 @@ ranks: forward 4*d and backward 10*d flops per visible (query, key) pair,
 causal pairs only.  With --gpus N every rank runs an independent replica of
 the workload (the path has no data exchange on one GPU), so scaling is weak.
 
+``e2e`` is the same step through the same public calls with the inputs copied
+in from pinned host memory and every result copied back, each step,
+pipelined over two device buffer slots and three streams.
+
 Extra measurements on the same line: the LSE merge (8 partials per rank of the
-striped 128k shapes), the Ulysses repack (the 256k zigzag Q shape) and the
-striped layout permute (the 128k Q shape) in GB/s against HBM, the causal
-striped 128k forward against the bf16 tensor peak, and the tabular row-axis
-attention (d = 24) against the tensor peak and the exp unit.
+striped 128k shapes, and the two-part in-place merge), the Ulysses repack (the
+256k zigzag Q shape), the striped layout permute (the 128k Q shape) and the
+tabular feature-axis attention in GB/s against HBM (device time of their own
+kernels); the causal striped 128k forward against the bf16 tensor peak; the
+tabular row-axis attention (d = 24) against the tensor peak and the exp unit;
+USP (Ulysses x ring) and Mesh2D fwd+bwd.  ``--case <group> [--small]`` runs one
+group of these alone (for a profiler run).
 
 ``--impl reference`` times the CPU fp64 oracle instead, on a bounded sample of
-the same workload (2048 queries of one query head, forward and backward against
-every key they see), and prints the same metric with "impl": "reference".
+the same workload (2048 queries of --ref-sample-heads query heads, forward and
+backward against every key they see), and prints the same metric with
+"impl": "reference"; under torchrun only rank 0 runs it.
 """
 
 from __future__ import annotations
@@ -76,19 +84,20 @@ def flops_bwd(w) -> float:
 # ---------------------------------------------------------------------------
 # distributed plumbing (independent replicas; barrier + max-over-ranks timing)
 # ---------------------------------------------------------------------------
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """One process per GPU from the torchrun environment.  The benchmark uses
+    NCCL; the CPU tests of this plumbing use gloo (no device is touched)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -99,12 +108,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Units all ranks processed over the slowest rank's time, per second:
+    every rank runs the same replica, so the job did world * steps steps in
+    max_ms."""
+    return units_per_rank_step * steps * world / (max_ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -272,8 +290,8 @@ def bench_ours(args, world, rank, local):
     fwd_ms = statistics.mean(p[1] for p in per)
     bwd_ms = statistics.mean(p[2] for p in per)
     step_ms_max = max_over_ranks(step_ms, world)
-    total_flops = (flops_fwd(w) + flops_bwd(w)) * args.steps * world
-    value = total_flops / (step_ms_max * 1e-3) / 1e12
+    step_flops = flops_fwd(w) + flops_bwd(w)
+    value = whole_job_rate(step_flops, args.steps, world, step_ms_max) / 1e12
     kernels = kernel_table(records, args.steps, step_ms / args.steps, w)
 
     # end-to-end: pinned host inputs in, results back to pinned host buffers,
@@ -324,7 +342,7 @@ def bench_ours(args, world, rank, local):
     e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_rate(step_flops, args.steps, world, e2e_ms) / 1e12
 
     line = {
         "metric": METRIC,
