@@ -42,7 +42,9 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 }
 
 // ---- LSE merge --------------------------------------------------------------
-template <typename OutT, int NPARTS>
+// SAME: every partial and the output have the same element strides, so one
+// row offset serves all of them (no per-part 64-bit address arithmetic).
+template <typename OutT, int NPARTS, bool SAME>
 __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, int rows_per_warp) {
   const int lane = threadIdx.x & 31;
   const int sub = lane / lanes;      // row slot within the warp
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
     const int64_t bh = (int64_t)b * a.H + h;
     const int64_t lidx = bh * a.lse_ld + t;
     const bool active = col < a.d;
+    const int64_t off0 = b * a.o_sb[0] + t * a.o_sn[0] + h * a.o_sh[0] + col;
     // every load of the row is issued before any of them is used (the O loads
     // do not wait for the LSE values), so one row costs one memory latency
     float4 x[kMaxMergeParts];
@@ -72,7 +75,9 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
 #pragma unroll
     for (int i = 0; i < kMaxMergeParts; ++i) {
       if (i < nparts) {
-        if (active) x[i] = load4(a.o_ptr[i] + b * a.o_sb[i] + t * a.o_sn[i] + h * a.o_sh[i] + col);
+        if (active)
+          x[i] = load4(a.o_ptr[i] +
+                       (SAME ? off0 : b * a.o_sb[i] + t * a.o_sn[i] + h * a.o_sh[i] + col));
         l[i] = a.lse_ptr[i][lidx];
       }
     }
@@ -110,7 +115,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
       }
     }
     if (active) {
-      OutT* out = reinterpret_cast<OutT*>(a.out) + b * a.out_sb + t * a.out_sn + h * a.out_sh + col;
+      OutT* out = reinterpret_cast<OutT*>(a.out) +
+                  (SAME ? off0 : b * a.out_sb + t * a.out_sn + h * a.out_sh + col);
       store4(out, acc);
     }
     if ((lane % lanes) == 0) a.lse_out[lidx] = lse;
@@ -195,13 +201,13 @@ int grid_for_rows(int64_t rows, int rows_per_warp) {
   return (int)(blocks < 1 ? 1 : blocks);
 }
 
-template <typename OutT>
+template <typename OutT, bool SAME>
 cudaError_t merge_dispatch(const MergeArgs& a, RowGroup g, int grid, cudaStream_t s) {
   switch (a.n_parts) {
-    case 2: lse_merge_kernel<OutT, 2><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    case 4: lse_merge_kernel<OutT, 4><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    case 8: lse_merge_kernel<OutT, 8><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    default: lse_merge_kernel<OutT, 0><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 2: lse_merge_kernel<OutT, 2, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 4: lse_merge_kernel<OutT, 4, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 8: lse_merge_kernel<OutT, 8, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    default: lse_merge_kernel<OutT, 0, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
   }
   return cudaGetLastError();
 }
@@ -213,9 +219,15 @@ cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stre
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(a.d);
   int grid = grid_for_rows(rows, g.rows_per_warp);
+  bool same = a.out_sb == a.o_sb[0] && a.out_sn == a.o_sn[0] && a.out_sh == a.o_sh[0];
+  for (int i = 1; i < a.n_parts; ++i)
+    same = same && a.o_sb[i] == a.o_sb[0] && a.o_sn[i] == a.o_sn[0] && a.o_sh[i] == a.o_sh[0];
   ProfScope ps("lse_merge", stream);
-  return out_bf16 ? merge_dispatch<__nv_bfloat16>(a, g, grid, stream)
-                  : merge_dispatch<float>(a, g, grid, stream);
+  if (same)
+    return out_bf16 ? merge_dispatch<__nv_bfloat16, true>(a, g, grid, stream)
+                    : merge_dispatch<float, true>(a, g, grid, stream);
+  return out_bf16 ? merge_dispatch<__nv_bfloat16, false>(a, g, grid, stream)
+                  : merge_dispatch<float, false>(a, g, grid, stream);
 }
 
 cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, rm_tensor o,

@@ -135,3 +135,21 @@ def test_launch_profiler_records_each_launch(rm):
     assert all(ms > 0 for _, ms in recs)
     rm.layout_permute(x, "zigzag", 2)
     assert rm.profile_records() == []  # disabled: nothing recorded
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_lse_merge_mixed_strides(rm, out_dtype):
+    """Partials whose strides differ (a head view of a wider tensor, a dense
+    tensor) and an output view with its own strides."""
+    B, Nq, H, d = 2, 301, 3, 64
+    wide = synthetic.tensor(920, (B, Nq, H + 2, d)).cuda()
+    o_parts = [wide[:, :, 1:1 + H], synthetic.tensor(921, (B, Nq, H, d)).cuda()]
+    lse_parts = [synthetic.tensor(930 + i, (B, H, Nq), scale=3.0).cuda() for i in range(2)]
+    ref_o, ref_l = omerge.lse_merge([np64(o) for o in o_parts], [np64(l) for l in lse_parts])
+    out_wide = torch.zeros(B, Nq, H + 1, d, dtype=out_dtype, device="cuda")
+    out = out_wide[:, :, :H]
+    o, l = rm.lse_merge(o_parts, lse_parts, out_dtype, out=out)
+    tol = F32_TOL if out_dtype == torch.float32 else BF16_O_TOL
+    assert_max_abs(np64(out), ref_o, tol, "merged O")
+    assert_max_abs(np64(l), ref_l, 1e-5, "merged LSE")
+    assert not out_wide[:, :, H].any()  # the column outside the view is untouched
