@@ -143,6 +143,11 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 template <int DP>
 constexpr int kEmuPairs = DP >= 128 ? 0 : 6;
 
+// P of a tile is handed to the PV MMA in kPParts parts (each kBN / kPParts
+// keys, its own barrier), so O += P V starts on the first keys while the
+// softmax is still exponentiating the rest.
+constexpr int kPParts = 2;
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -167,6 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_o_done = bars + 11;
   uint64_t* bar_drain = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  // [2][kPParts - 1]: P of the first parts of a tile written (the last part is bar_p_full)
+  uint64_t* bar_p_part = bars + 14;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -245,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_s_full + x, 1);
+      for (int q = 0; q + 1 < kPParts; ++q) mbar_init(bar_p_part + x * (kPParts - 1) + q, 128);
       mbar_init(bar_p_full + x, 128);
     }
     mbar_init(bar_o_done, 1);
@@ -335,12 +343,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < DP / 16; ++k)
           mma_ss(tmem + scol, kmajor_desc<DP>(qaddr, k), kmajor_desc<DP>(kaddr, k), idS, k > 0);
       };
-      auto issue_pv = [&](uint32_t scol, uint32_t ocol, int st, bool first) {
+      // O += P V over the keys of one part of the tile (kBN / kPParts keys):
+      // each part starts as soon as the softmax has written it
+      auto issue_pv_part = [&](uint32_t scol, uint32_t ocol, int st, bool first, int part) {
         const uint32_t vaddr = vbase + st * C::kTileBytes;
+        constexpr int kSteps = kBN / 16 / kPParts;
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k)
+        for (int kk = 0; kk < kSteps; ++kk) {
+          const int k = part * kSteps + kk;
           mma_ts(tmem + ocol, tmem + scol + k * 8, v_desc<DP>(vaddr, k), idO,
                  (first && k == 0) ? 0u : 1u);
+        }
+      };
+      auto issue_pv = [&](int x, uint32_t scol, uint32_t ocol, int st, int j) -> bool {
+#pragma unroll
+        for (int part = 0; part < kPParts; ++part) {
+          uint64_t* bar = part + 1 < kPParts ? bar_p_part + x * (kPParts - 1) + part
+                                             : bar_p_full + x;
+          if (!mbar_wait(bar, j & 1, limit, p.status)) return false;
+          fence_after_sync();
+          issue_pv_part(scol, ocol, st, j == 0, part);
+        }
+        return true;
       };
       bool ok = mbar_wait(bar_q, 0, limit, p.status);
       if (ok && n > 0) {
@@ -357,18 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = j & 1;
         const int nx = (j + 1) & 1;
         if (!mbar_wait(bar_v_full + st, (j >> 1) & 1, limit, p.status)) break;
-        if (!mbar_wait(bar_p_full + 0, j & 1, limit, p.status)) break;
-        fence_after_sync();
-        issue_pv(C::kS0, C::kO0, st, j == 0);
+        if (!issue_pv(0, C::kS0, C::kO0, st, j)) break;
         if (j + 1 < n) {
           if (!mbar_wait(bar_k_full + nx, ((j + 1) >> 1) & 1, limit, p.status)) break;
           fence_after_sync();
           issue_s(q0, C::kS0, nx);
           mma_commit(bar_s_full + 0);
         }
-        if (!mbar_wait(bar_p_full + 1, j & 1, limit, p.status)) break;
-        fence_after_sync();
-        issue_pv(C::kS1, C::kO1, st, j == 0);
+        if (!issue_pv(1, C::kS1, C::kO1, st, j)) break;
         mma_commit(bar_kv_empty + st);
         if (j + 1 < n) {
           issue_s(q1, C::kS1, nx);
@@ -393,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + ((uint32_t)lane_base << 16) + (X ? C::kS1 : C::kS0);
     const uint32_t tO = tmem + ((uint32_t)lane_base << 16) + (X ? C::kO1 : C::kO0);
     uint64_t* s_full = bar_s_full + X;
+    uint64_t* p_part = bar_p_part + X * (kPParts - 1);
     uint64_t* p_full = bar_p_full + X;
     float m = -INFINITY;  // running max of the scaled scores, log2 units
     float l = 0.f;        // running row sum (relative to m)
@@ -485,6 +506,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[i] = pack_bf16(p2.x, p2.y);
           }
           tmem_st16(tS + c * 16, pk);
+          constexpr int kChunksPerPart = kBN / 32 / kPParts;
+          if ((c + 1) % kChunksPerPart == 0 && c + 1 < kBN / 32) {
+            // a part of P is written: the PV MMA may start on its keys
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(p_part + (c + 1) / kChunksPerPart - 1);
+          }
         }
         l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
         tmem_wait_st();
