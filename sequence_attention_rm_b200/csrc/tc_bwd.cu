@@ -141,8 +141,14 @@ constexpr int kHalf = BQ / 2;  // query columns per math warpgroup
 constexpr int kQStages = 3;   // Q is read by S^T(i) and dK(i): the longer-lived operand
 constexpr int kDOStages = 2;  // dO by dP^T(i) and dV(i)
 constexpr int kThreads = 384;
-constexpr int kWarpTma = 8;
-constexpr int kWarpMma = 9;
+// Warp w runs on SM sub-partition w % 4, so the math warps 0-7 put two warps
+// on each; the TMA and MMA warps go to sub-partitions 3 and 2.  With them on
+// 0 and 1 (warps 8 and 9), clock64 traces showed the two math warps beside
+// the MMA warp finishing each tile ~900 cycles after the others, which then
+// waited for them at the per-tile LSE / D staging barrier; warps 11 and 10
+// measured 4.4% less kernel time (interleaved A/B on the 16k step).
+constexpr int kWarpTma = 11;
+constexpr int kWarpMma = 10;
 constexpr int kRegsMath = 200;
 constexpr int kRegsOther = 104;
 static_assert(2 * 128 * kRegsMath + 128 * kRegsOther <= kThreads * 168, "register split");
