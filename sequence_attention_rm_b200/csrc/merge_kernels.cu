@@ -167,6 +167,59 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(int B, int64_t N, i
   }
 }
 
+// bf16 operands with 16-byte rows (d % 8 == 0): 8 elements per lane, LANES
+// lanes per head row, so a warp pass covers 32 / LANES rows of a token; the
+// loads of kAhead passes are issued before any row is reduced.  The grid is
+// sized to the blocks that fit on the device at once (one wave).
+template <int LANES>
+__global__ void __launch_bounds__(256) bwd_delta_bf16_kernel(int B, int64_t N, int H, int d,
+                                                             rm_tensor o, rm_tensor dout,
+                                                             float* __restrict__ delta) {
+  constexpr int kRows = 32 / LANES;  // head rows per warp pass
+  constexpr int kAhead = 4;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LANES;
+  const int col = (lane % LANES) * 8;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t tokens = (int64_t)B * N;
+  for (int64_t bt = warp0; bt < tokens; bt += nwarps) {
+    const int64_t t = bt % N;
+    const int64_t b = bt / N;
+    const __nv_bfloat16* orow =
+        reinterpret_cast<const __nv_bfloat16*>(o.ptr) + b * o.stride_b + t * o.stride_n;
+    const __nv_bfloat16* drow =
+        reinterpret_cast<const __nv_bfloat16*>(dout.ptr) + b * dout.stride_b + t * dout.stride_n;
+    for (int h0 = 0; h0 < H; h0 += kRows * kAhead) {
+      uint4 x[kAhead], y[kAhead];
+#pragma unroll
+      for (int j = 0; j < kAhead; ++j) {
+        const int h = h0 + j * kRows + sub;
+        x[j] = y[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (h < H && col < d) {
+          x[j] = *reinterpret_cast<const uint4*>(orow + (int64_t)h * o.stride_h + col);
+          y[j] = *reinterpret_cast<const uint4*>(drow + (int64_t)h * dout.stride_h + col);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kAhead; ++j) {
+        const int h = h0 + j * kRows + sub;
+        const uint32_t xa[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+        const uint32_t ya[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
+        float v = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v = fmaf(__uint_as_float(xa[e] << 16), __uint_as_float(ya[e] << 16), v);
+          v = fmaf(__uint_as_float(xa[e] & 0xffff0000u), __uint_as_float(ya[e] & 0xffff0000u), v);
+        }
+#pragma unroll
+        for (int off = LANES >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (h < H && (lane % LANES) == 0) delta[(b * H + h) * N + t] = v;
+      }
+    }
+  }
+}
+
 // ---- fp32 -> output dtype ---------------------------------------------------
 template <typename OutT>
 __global__ void __launch_bounds__(256) convert_f32_kernel(int B, int64_t N, int H, int d,
@@ -230,11 +283,43 @@ cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stre
                   : merge_dispatch<float, false>(a, g, grid, stream);
 }
 
+template <int LANES>
+cudaError_t launch_delta_bf16(int B, int64_t N, int H, int d, rm_tensor o, rm_tensor dout,
+                              float* delta, cudaStream_t stream) {
+  static int per_sm[64] = {0};  // resident blocks per SM, by device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& k = per_sm[dev & 63];
+  if (k <= 0 &&
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, bwd_delta_bf16_kernel<LANES>, 256, 0) !=
+           cudaSuccess ||
+       k <= 0))
+    k = 4;
+  const int64_t warps = (int64_t)B * N;  // one token per warp pass
+  const int64_t need = (warps + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * k;
+  const int grid = (int)(need < cap ? need : cap);
+  bwd_delta_bf16_kernel<LANES><<<grid, 256, 0, stream>>>(B, N, H, d, o, dout, delta);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, rm_tensor o,
                                   rm_tensor dout, float* delta, float* zero_fill,
                                   cudaStream_t stream) {
   const int64_t rows = (int64_t)B * H * N;
   if (rows == 0) return cudaSuccess;
+  auto rows16 = [](const rm_tensor& x) {
+    return ((uintptr_t)x.ptr % 16) == 0 && x.stride_b % 8 == 0 && x.stride_n % 8 == 0 &&
+           x.stride_h % 8 == 0;
+  };
+  if (in_bf16 && !zero_fill && d % 8 == 0 && d <= 128 && rows16(o) && rows16(dout)) {
+    ProfScope ps("bwd_preprocess", stream);
+    const int need = d / 8;
+    if (need > 8) return launch_delta_bf16<16>(B, N, H, d, o, dout, delta, stream);
+    if (need > 4) return launch_delta_bf16<8>(B, N, H, d, o, dout, delta, stream);
+    if (need > 2) return launch_delta_bf16<4>(B, N, H, d, o, dout, delta, stream);
+    return launch_delta_bf16<2>(B, N, H, d, o, dout, delta, stream);
+  }
   RowGroup g = row_group(d);
   int grid = grid_for_rows((int64_t)B * N, 1);  // one token per warp pass
   ProfScope ps("bwd_preprocess", stream);

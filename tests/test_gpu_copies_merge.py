@@ -105,7 +105,8 @@ def test_lse_merge_in_place(rm, n, Nq, H, d):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("B,N,H,d", [(1, 7, 3, 128), (2, 130, 16, 128), (1, 33, 20, 24), (1, 5, 2, 4)])
+@pytest.mark.parametrize("B,N,H,d", [(1, 7, 3, 128), (2, 130, 16, 128), (1, 33, 20, 24), (1, 5, 2, 4),
+                                     (3, 65, 8, 64), (1, 40, 5, 32), (1, 9, 3, 12)])
 def test_bwd_preprocess(rm, dtype, B, N, H, d):
     o = synthetic.tensor(800, (B, N, H, d), dtype)
     do = synthetic.tensor(801, (B, N, H, d), dtype)
@@ -153,3 +154,16 @@ def test_lse_merge_mixed_strides(rm, out_dtype):
     assert_max_abs(np64(out), ref_o, tol, "merged O")
     assert_max_abs(np64(l), ref_l, 1e-5, "merged LSE")
     assert not out_wide[:, :, H].any()  # the column outside the view is untouched
+
+
+@pytest.mark.parametrize("offset", [8, 4])
+def test_bwd_preprocess_strided_views(rm, offset):
+    """Head views inside wider rows: 16-byte aligned rows (offset 8 elements)
+    take the 16-byte-lane kernel, 8-byte aligned rows (offset 4) the 8-byte one."""
+    B, N, H, d = 2, 77, 6, 64
+    wide_o = synthetic.tensor(810, (B, N, H, d + 16), torch.bfloat16).cuda()
+    wide_do = synthetic.tensor(811, (B, N, H, d + 16), torch.bfloat16).cuda()
+    o, do = wide_o[..., offset:offset + d], wide_do[..., offset:offset + d]
+    ref = oatt.delta_from_output(np64(do), np64(o))
+    got = rm.attn_bwd_preprocess(o, do)
+    assert_max_abs(np64(got), ref, 1e-4 * max(1.0, np.abs(ref).max()), "delta")
