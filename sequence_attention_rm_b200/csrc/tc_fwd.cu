@@ -104,6 +104,19 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int k) {
   const uint32_t addr = tile_addr + (col / C::kBoxCols) * C::kBoxBytes + (col % C::kBoxCols) * 2;
   return smem_desc(addr, 16, 8 * C::kRowBytes, C::kSwz);
 }
+// Byte offset of K-step k (columns [16k, 16k + 16)) within a K-major tile:
+// kmajor_desc(tile, k) and kmajor_desc(tile, 0) differ by kmajor_off(k) >> 4
+// in the address field of the low word.
+template <int DP>
+__host__ __device__ constexpr uint32_t kmajor_off(int k) {
+  using C = FwdCfg<DP>;
+  return (uint32_t)((k * 16 / C::kBoxCols) * C::kBoxBytes + (k * 16 % C::kBoxCols) * 2);
+}
+// A descriptor from its low word and a high word that does not depend on the
+// address (the stride / swizzle fields).
+__device__ __forceinline__ uint64_t desc_of(uint32_t hi, uint32_t lo) {
+  return ((uint64_t)hi << 32) | lo;
+}
 // V tile as the MN-major B operand of O += P V: K-step k covers kv rows
 // [16k, 16k+16); the d axis is split over boxes kBoxBytes apart.
 template <int DP>
@@ -337,22 +350,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = shard_of(step);
         n += max(0, tile_end(s) - tile_begin(s));
       }
+      // descriptors as a constant high word and a low word per tile: a K-step
+      // adds a constant to the low word (the address field does not carry:
+      // shared memory is below 256 KB)
+      const uint32_t hiK = (uint32_t)(kmajor_desc<DP>(q0, 0) >> 32);
+      const uint32_t hiV = (uint32_t)(v_desc<DP>(vbase, 0) >> 32);
+      const uint32_t loK0 = (uint32_t)kmajor_desc<DP>(kbase, 0);
+      const uint32_t loV0 = (uint32_t)v_desc<DP>(vbase, 0);
       auto issue_s = [&](uint32_t qaddr, uint32_t scol, int st) {
-        const uint32_t kaddr = kbase + st * C::kTileBytes;
+        const uint32_t lq = (uint32_t)kmajor_desc<DP>(qaddr, 0);
+        const uint32_t lk = loK0 + st * (C::kTileBytes >> 4);
 #pragma unroll
         for (int k = 0; k < DP / 16; ++k)
-          mma_ss(tmem + scol, kmajor_desc<DP>(qaddr, k), kmajor_desc<DP>(kaddr, k), idS, k > 0);
+          mma_ss(tmem + scol, desc_of(hiK, lq + (kmajor_off<DP>(k) >> 4)),
+                 desc_of(hiK, lk + (kmajor_off<DP>(k) >> 4)), idS, k > 0);
       };
       // O += P V over the keys of one part of the tile (kBN / kPParts keys):
       // each part starts as soon as the softmax has written it
       auto issue_pv_part = [&](uint32_t scol, uint32_t ocol, int st, bool first, int part) {
-        const uint32_t vaddr = vbase + st * C::kTileBytes;
+        const uint32_t lv = loV0 + st * (C::kTileBytes >> 4);
         constexpr int kSteps = kBN / 16 / kPParts;
 #pragma unroll
         for (int kk = 0; kk < kSteps; ++kk) {
           const int k = part * kSteps + kk;
-          mma_ts(tmem + ocol, tmem + scol + k * 8, v_desc<DP>(vaddr, k), idO,
-                 (first && k == 0) ? 0u : 1u);
+          mma_ts(tmem + ocol, tmem + scol + k * 8, desc_of(hiV, lv + ((k * 16 * C::kRowBytes) >> 4)),
+                 idO, (first && k == 0) ? 0u : 1u);
         }
       };
       auto issue_pv = [&](int x, uint32_t scol, uint32_t ocol, int st, int j) -> bool {
