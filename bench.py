@@ -228,8 +228,8 @@ class Step:
 FLOPS_PER_PAIR = {"tc_fwd_kernel": 4, "tc_bwd_dkdv_kernel": 8, "tc_bwd_dq_kernel": 6}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from the committed
 # ncu captures of the current kernels (profiles/); None until captured.
-TRAFFIC = {"tc_fwd_kernel": 174_120_000, "tc_bwd_dkdv_kernel": 253_200_000,
-           "tc_bwd_dq_kernel": 251_290_000}
+TRAFFIC = {"tc_fwd_kernel": 173_660_000, "tc_bwd_dkdv_kernel": 252_780_000,
+           "tc_bwd_dq_kernel": 251_850_000}
 
 
 def kernel_table(records, steps, step_ms, w):
