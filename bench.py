@@ -408,7 +408,8 @@ def _time(fn, reps, flush, rm=None):
     for _ in range(reps):
         if flush is not None:
             flush_l2(flush)
-        torch.cuda._sleep(SPIN_CYCLES)
+        if _spin is not None:  # keep the GPU busy while the host queues fn
+            _spin(SPIN_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if rm is not None:
             rm.profile_enable(True)
@@ -426,8 +427,10 @@ def _time(fn, reps, flush, rm=None):
 
 
 # about 1 ms of spinning at the B200's clocks: longer than the host needs to
-# queue any call timed here
+# queue any call timed here.  torch's spin kernel is a private helper; without
+# it the call times include host time, the kernels' own event times do not.
 SPIN_CYCLES = 2_000_000
+_spin = getattr(torch.cuda, "_sleep", None)
 
 
 def hbm_row(rm, fn, reps, flush, nbytes, hbm, peak_src, shape):
