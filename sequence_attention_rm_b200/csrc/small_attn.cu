@@ -1,14 +1,20 @@
 // Attention over very short sequences (L <= 16 tokens, d <= 64): the
 // "local" backend of the Mosaic page (attention over a 5-token feature axis
 // of a tabular tensor).  A 128-row tensor-core tile would be >95% padding
-// here and the problem is HBM-bound, so the work is spread as thinly as it
-// goes: one thread per (sequence, query token, head), heads fastest, so the
-// threads of a warp read consecutive head rows of one token (coalesced) and
-// share each key / value row through L1.  A thread keeps its query row in
-// registers (pre-scaled into log2 units), scores the L keys, takes the
-// softmax with the SFU exp2, accumulates O and writes O and the LSE.
-// Rows are read as 16-byte vectors when every stride and the base pointers
-// allow it (VEC), else element by element.
+// here and the problem is HBM-bound, so one thread owns one (sequence, query
+// token, head): it keeps its query row in registers, scores the L keys,
+// takes the softmax with the SFU exp2, accumulates O and writes O and the
+// LSE.  Two kernels:
+//  - small_seq_tma_kernel (bf16 operands and output, d in {24, 32, 64}):
+//    persistent and warp-specialised; a producer warp copies whole batches
+//    of sequences into a shared-memory ring (bulk or TMA copies) and the
+//    consumer threads read rows from shared memory, with mixed-precision
+//    bf16 FMAs (see the comment above the kernel);
+//  - small_seq_attn_kernel (fp32 operands, fp32 partial outputs): rows read
+//    from global memory, heads fastest so that the threads of a warp read
+//    consecutive head rows of one token and share key / value rows through
+//    L1; 16-byte vectors when every stride and the base pointers allow it
+//    (VEC), else element by element.
 #include <math.h>
 
 #include <cudaTypedefs.h>
