@@ -151,10 +151,12 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 // Pairs (of the 16 in each 32-column chunk of a row) whose exponentials use
 // exp2_fma2 instead of the SFU: for d <= 64 the SFU outweighs the tensor
-// work (6 of 16 pairs measured 4.6% faster on the d = 24 tabular rows); for
-// d = 128 every split measured slower, so all go to the SFU.
+// work (on the d = 24 tabular rows 6 of 16 pairs measured 4.6% faster than
+// none; with the MMA thread's cheaper descriptors 4 measured 5.0% faster than
+// 6, and 8 slower); for d = 128 every split measured slower, so all go to
+// the SFU.
 template <int DP>
-constexpr int kEmuPairs = DP >= 128 ? 0 : 6;
+constexpr int kEmuPairs = DP >= 128 ? 0 : 4;
 
 // P of a tile is handed to the PV MMA in kPParts parts (each kBN / kPParts
 // keys, its own barrier), so O += P V starts on the first keys while the
