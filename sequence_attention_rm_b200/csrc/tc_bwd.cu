@@ -252,8 +252,8 @@ struct Walk {
 
 // Warp roles (384 threads): warps 0-3 and 4-7 are two math warpgroups that
 // split every 128-query tile by columns (queries 0-63 / 64-127) over all 128
-// key lanes, then write dK (warps 0-3) and dV (warps 4-7); warp 8 TMA producer
-// (K, V once; Q into a 3-stage ring, dO into a 2-stage ring); warp 9 MMA
+// key lanes, then write dK (warps 0-3) and dV (warps 4-7); warp kWarpTma (11) TMA producer
+// (K, V once; Q into a 3-stage ring, dO into a 2-stage ring); warp kWarpMma (10) MMA
 // issuer.  All four contractions are M=128, N=128: S^T, dP^T from shared
 // memory; dV and dK take P^T and dS^T from TMEM, so only Q and dO are read
 // from shared memory for them.  The warpgroups copy S^T(i) into registers and
