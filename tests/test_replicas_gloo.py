@@ -6,7 +6,8 @@ processes share is host logic: the rendezvous, the barriers around the timed
 region, the max over ranks of the device time, the whole-job rate (units of
 all ranks over the slowest rank's time), and the rule that only rank 0 runs
 and prints the reference arm.  All of that is exercised here with world size
-2 over gloo; nothing touches a GPU.
+2 over gloo; nothing touches a GPU.  The reference arm's JSON line (the CPU
+oracle on a bounded sample) is checked against the contract too.
 """
 
 import json
@@ -70,3 +71,25 @@ def test_single_process_rate():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.whole_job_rate(1.0e12, 10, 1, 20.0) == pytest.approx(1.0e12 * 10 / 20e-3)
+
+
+def test_reference_line_contract():
+    """The reference arm (the CPU oracle on a bounded sample) prints the same
+    metric and units as the GPU arm, marked impl = reference, with its own
+    cpu_baseline and an e2e that moves no bytes over the host link."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        steps, warmup, ref_sample_heads = 1, 3, 1
+
+    line = bench.bench_reference(Args, 1, 0)
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["value"] > 0 and line["higher_is_better"]
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert "1 of 16 query heads" in cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0
+    assert e2e["d2h_bytes_per_step"] == 0
