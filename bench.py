@@ -2,38 +2,48 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (one "step"): the Llama-like causal ring -- B=1, 16 query heads / 8
-KV heads, d=128, N=16384 bf16 tokens, P=2 virtual ranks in the zigzag
-(load-balanced) layout, forward + backward:
-  fused ring forward -> ring backward (delta preprocess, key-stationary dK/dV
-  kernel, query-stationary dQ kernel), on operands in their global token
-  order: each virtual rank's tiles are fetched through the zigzag layout by
-  the kernels' TMA coordinates and O, LSE, dQ, dK, dV are written back in
-  global order, so the step has no separate permute pass (the permute kernel
-  itself is timed in the extras).
+Workload (one "step"): the long causal zigzag workload -- B=1, 16 query heads
+/ 8 KV heads, d=128, N=262144 bf16 tokens, P=8 virtual ranks in the zigzag
+(load-balanced) layout, forward + backward, plus the Ulysses seq->head repack
+of Q and of the fused K|V ([8 x 32768, 16, 128] -> [8 x 262144, 2, 128], one
+call each):
+  repack Q, repack K|V, fused ring forward -> ring backward (delta
+  preprocess, key-stationary dK/dV kernel, query-stationary dQ kernel), on
+  operands in their global token order: each virtual rank's tiles are fetched
+  through the zigzag layout by the kernels' TMA coordinates and O, LSE, dQ,
+  dK, dV are written back in global order, so the step has no separate
+  permute pass (the permute kernel itself is timed in the extras).  K and V
+  are two head views of one fused [1, N, 16, 128] buffer.
 Inputs are seeded synthetic tensors already resident in HBM; L2 (126 MB) is
 flushed between timed steps.  ``value`` is algorithmic TFLOP/s summed over all
 ranks: forward 4*d and backward 10*d flops per visible (query, key) pair,
-causal pairs only.  With --gpus N every rank runs an independent replica of
-the workload (the path has no data exchange on one GPU), so scaling is weak.
+causal pairs only (the repack adds time, no flops).  With --gpus N every rank
+runs an independent replica of the workload (the path has no data exchange on
+one GPU), so scaling is weak.
+
+``roofline`` is the step's dominant kernel against the bf16 tensor peak: the
+burst figure, or the sustained one when the timed region ran for seconds in
+the power-capped regime its clock record shows.
 
 ``e2e`` is the same step through the same public calls with the inputs copied
-in from pinned host memory and every result copied back, each step,
-pipelined over two device buffer slots and three streams.
+in from pinned host memory and every result (O, LSE, dQ, dK, dV and the two
+repacked tensors) copied back, each step, pipelined over two device buffer
+slots and three streams.
 
-Extra measurements on the same line: the LSE merge (8 partials per rank of the
-striped 128k shapes, and the two-part in-place merge), the Ulysses repack (the
-256k zigzag Q shape), the striped layout permute (the 128k Q shape) and the
+Extra measurements on the same line: fwd+bwd of the causal striped 128k and
+the Llama-like zigzag 16k workloads; the LSE merge (8 partials per rank of
+the striped 128k shapes, and the two-part in-place merge), the Ulysses repack
+(the 256k shapes), the striped layout permute (the 128k Q shape) and the
 tabular feature-axis attention in GB/s against HBM (device time of their own
-kernels); the causal striped 128k forward against the bf16 tensor peak; the
-tabular row-axis attention (d = 24) against the tensor peak and the exp unit;
-USP (Ulysses x ring) and Mesh2D fwd+bwd.  ``--case <group> [--small]`` runs one
-group of these alone (for a profiler run).
+kernels); the tabular row-axis attention (d = 24) against the tensor peak and
+the exp unit; USP (Ulysses x ring) and Mesh2D fwd+bwd.  ``--case <group>
+[--small]`` runs one group of these alone (for a profiler run).
 
 ``--impl reference`` times the CPU fp64 oracle instead, on a bounded sample of
-the same workload (2048 queries of --ref-sample-heads query heads, forward and
-backward against every key they see), and prints the same metric with
-"impl": "reference"; under torchrun only rank 0 runs it.
+the same workload (the last --ref-sample-queries queries of query head 0,
+forward and backward against every key they see), and prints the same metric
+with "impl": "reference"; under torchrun only rank 0 runs it.  ``cpu_baseline``
+times the same sample.
 """
 
 from __future__ import annotations
@@ -56,6 +66,10 @@ sys.path.insert(0, ROOT)
 from sequence_attention_rm_b200 import synthetic  # noqa: E402
 
 METRIC = "ring-attn fwd+bwd TFLOP/s and % of BF16 peak at 1 B200; merge GB/s % HBM"
+HEADLINE = synthetic.LONG_ZIGZAG_256K
+HEADLINE_NAME = ("long-causal-zigzag-256k: B=1 Hq=16 Hkv=8 d=128 N=262144 bf16 P=8 zigzag causal "
+                 "fwd+bwd + seq->head repack of Q and fused K|V [8 x 32768, 16, 128] -> "
+                 "[8 x 262144, 2, 128]")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -192,44 +206,83 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 class Step:
-    """Pre-allocated buffers and the hot-path step of one workload: the fused
-    ring forward and the ring backward on global-order operands."""
+    """Pre-allocated buffers and one hot-path step of a workload, on operands
+    in their global token order: the Ulysses seq->head repack of Q and of the
+    fused K|V, the fused ring forward and the ring backward.
 
-    def __init__(self, rm, w, q, k, v, do):
+    K and V live in one fused buffer [B, N, 2 Hkv, d] (the Hkv K heads, then
+    the Hkv V heads of every token); the ring reads them as two strided head
+    views, and the repack moves the buffer as 2 Hkv heads, so that the K/V
+    exchange is one all-to-all (ringmaster "Status": the Ulysses leg fuses
+    K/V).  The repack treats the global-order tensors as P contiguous
+    sequence shards [P, N / P, H, d] and writes head-sharded [P, N, H / P, d]
+    tensors, each rank's heads over the whole sequence in global order."""
+
+    def __init__(self, rm, w, q, kv, do, repack=True):
         self.rm, self.w = rm, w
-        self.q, self.k, self.v, self.do = q, k, v, do
+        self.q, self.kv, self.do = q, kv, do
+        self.k, self.v = kv[:, :, :w.Hkv], kv[:, :, w.Hkv:]
         e = lambda t: torch.empty_like(t)
-        self.o_g, self.dq_g, self.dk_g, self.dv_g = e(q), e(q), e(k), e(v)
-        self.lse_g = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
+        self.o, self.dq = e(q), e(q)
+        self.dk = torch.empty(q.shape[:2] + (w.Hkv, w.d), dtype=q.dtype, device=q.device)
+        self.dv = torch.empty_like(self.dk)
+        self.lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
         dsc = rm.desc(w.dtype, w.B, w.Hq, w.Hkv, w.d, w.N, w.P, w.layout, w.causal,
                       order="global")
         self.ws = torch.empty(max(rm.ring_workspace_size(dsc, True), 256), dtype=torch.uint8,
                               device=q.device)
-        self.launches_per_step = 1 + 3  # forward; delta, dK/dV, dQ
+        self.repack = repack and w.B == 1
+        if self.repack:
+            P, L = w.P, w.N // w.P
+            self.q_shards = q.view(P, L, w.Hq, w.d)
+            self.kv_shards = kv.view(P, L, 2 * w.Hkv, w.d)
+            self.qh = torch.empty((P, w.N, w.Hq // P, w.d), dtype=q.dtype, device=q.device)
+            self.kvh = torch.empty((P, w.N, 2 * w.Hkv // P, w.d), dtype=q.dtype, device=q.device)
+        # repack Q, repack K|V; forward; delta, dK/dV, dQ
+        self.launches_per_step = (2 if self.repack else 0) + 1 + 3
+
+    def outputs(self):
+        out = [self.o, self.lse, self.dq, self.dk, self.dv]
+        return out + ([self.qh, self.kvh] if self.repack else [])
+
+    def repack_bytes(self) -> int:
+        if not self.repack:
+            return 0
+        return 2 * (self.q.numel() + self.kv.numel()) * self.q.element_size()
 
     def run(self, ev=None):
         rm, w = self.rm, self.w
         lay, P = w.layout, w.P
         if ev:
             ev[0].record()
-        rm.ring_attn_fwd(self.q, self.k, self.v, P=P, layout=lay, causal=w.causal,
-                         order="global", out=self.o_g, lse=self.lse_g)
+        if self.repack:
+            rm.seq_head_repack(self.q_shards, P, out=self.qh)
+            rm.seq_head_repack(self.kv_shards, P, out=self.kvh)
         if ev:
             ev[1].record()
-        rm.ring_attn_bwd(self.q, self.k, self.v, self.o_g, self.lse_g, self.do, P=P, layout=lay,
-                         causal=w.causal, order="global", dq=self.dq_g, dk=self.dk_g,
-                         dv=self.dv_g, ws=self.ws)
+        rm.ring_attn_fwd(self.q, self.k, self.v, P=P, layout=lay, causal=w.causal,
+                         order="global", out=self.o, lse=self.lse)
         if ev:
             ev[2].record()
+        rm.ring_attn_bwd(self.q, self.k, self.v, self.o, self.lse, self.do, P=P, layout=lay,
+                         causal=w.causal, order="global", dq=self.dq, dk=self.dk, dv=self.dv,
+                         ws=self.ws)
+        if ev:
+            ev[3].record()
+
+
+def fused_kv(k, v):
+    """[B, N, Hkv, d] K and V -> one [B, N, 2 Hkv, d] buffer (K heads first)."""
+    return torch.cat([k, v], dim=2).contiguous()
 
 
 # Algorithmic flops per launch of each attention kernel, per visible (query,
 # key) pair: the contractions the kernel performs for its outputs.
 FLOPS_PER_PAIR = {"tc_fwd_kernel": 4, "tc_bwd_dkdv_kernel": 8, "tc_bwd_dq_kernel": 6}
-# dram__bytes_read.sum + dram__bytes_write.sum per launch from the committed
-# ncu captures of the current kernels (profiles/); None until captured.
-TRAFFIC = {"tc_fwd_kernel": 173_660_000, "tc_bwd_dkdv_kernel": 252_780_000,
-           "tc_bwd_dq_kernel": 251_850_000}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel on
+# the headline workload, from the committed ncu capture of the current
+# kernels (profiles/); None until captured.
+TRAFFIC = {}
 
 
 def kernel_table(records, steps, step_ms, w):
@@ -259,21 +312,40 @@ def time_events(pairs):
     return [a.elapsed_time(b) for a, b in pairs]
 
 
+def tensor_peak(peaks, peak_src, timed_s, clocks):
+    """The bf16 peak a tensor-core kernel is judged against: the burst figure
+    (a short region at full clocks), unless the timed region lasted seconds
+    and its clock record shows the power-capped regime in which the
+    sustained figure was measured (SM clock at most 85% of its maximum under
+    load, with sw_power_cap active)."""
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = (timed_s >= 2.0 and mhz is not None and mx
+              and mhz <= 0.85 * mx and "sw_power_cap" in clocks.get("reasons", []))
+    if capped:
+        return sustained, (f"{peak_src} bf16_tflops_sustained: the timed region ran {timed_s:.1f} s "
+                           f"at a median {mhz:.0f} of {mx:.0f} MHz under sw_power_cap")
+    return burst, f"{peak_src} bf16_tflops (burst)"
+
+
 def bench_ours(args, world, rank, local):
     from sequence_attention_rm_b200 import rm
 
     peaks, peak_src = load_peaks()
-    w = synthetic.LLAMA_ZIGZAG
+    w = HEADLINE
     dev = torch.device("cuda", local)
     q_h, k_h, v_h, do_h = synthetic.attention_inputs(w)
-    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
-    step = Step(rm, w, q, k, v, do)
+    kv_h = fused_kv(k_h, v_h)
+    del k_h, v_h
+    q, kv, do = (t.to(dev) for t in (q_h, kv_h, do_h))
+    step = Step(rm, w, q, kv, do)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     rm.profile_enable(True)  # per-launch CUDA events on the launching stream
@@ -285,25 +357,31 @@ def bench_ours(args, world, rank, local):
     barrier(world)
     records = rm.profile_records()
     rm.profile_enable(False)
-    per = [time_events([(e[0], e[2]), (e[0], e[1]), (e[1], e[2])]) for e in evs]
+    per = [time_events([(e[0], e[3]), (e[0], e[1]), (e[1], e[2]), (e[2], e[3])]) for e in evs]
     step_ms = sum(p[0] for p in per)
-    fwd_ms = statistics.mean(p[1] for p in per)
-    bwd_ms = statistics.mean(p[2] for p in per)
+    repack_ms = statistics.mean(p[1] for p in per)
+    fwd_ms = statistics.mean(p[2] for p in per)
+    bwd_ms = statistics.mean(p[3] for p in per)
     step_ms_max = max_over_ranks(step_ms, world)
     step_flops = flops_fwd(w) + flops_bwd(w)
     value = whole_job_rate(step_flops, args.steps, world, step_ms_max) / 1e12
     kernels = kernel_table(records, args.steps, step_ms / args.steps, w)
+    clocks = clk.summary()
 
-    # end-to-end: pinned host inputs in, results back to pinned host buffers,
-    # every step.  Two device slots and three streams: step i+1's inputs are
-    # copied in and step i-1's results copied out while step i computes.
+    # end-to-end: pinned host inputs in, every result back to pinned host
+    # buffers, every step.  Two device slots and three streams: step i+1's
+    # inputs are copied in and step i-1's results copied out while step i
+    # computes.
     pin = lambda t: t.pin_memory()
-    hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
-    slots = [step, Step(rm, w, *(torch.empty_like(t) for t in (q, k, v, do)))]
-    host_out = [[pin(torch.empty(t.shape, dtype=t.dtype))
-                 for t in (sl.o_g, sl.dq_g, sl.dk_g, sl.dv_g, sl.lse_g)] for sl in slots]
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    hq, hkv, hdo = pin(q_h), pin(kv_h), pin(do_h)
+    del q_h, kv_h, do_h
+    slots = [step, Step(rm, w, *(torch.empty_like(t) for t in (q, kv, do)))]
+    # one set of host result buffers: the device->host copies of successive
+    # steps run in order on one stream, so each step's results overwrite the
+    # previous ones (8 GiB of pinned host memory in all, inputs included)
+    host_out = [pin(torch.empty(t.shape, dtype=t.dtype)) for t in step.outputs()]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hkv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
     s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev = lambda: torch.cuda.Event()
     done_in, done_run, done_out = ([ev(), ev()] for _ in range(3))
@@ -314,7 +392,7 @@ def bench_ours(args, world, rank, local):
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(done_run[j])  # slot j's inputs free again
-            for src, dst in ((hq, sl.q), (hk, sl.k), (hv, sl.v), (hdo, sl.do)):
+            for src, dst in ((hq, sl.q), (hkv, sl.kv), (hdo, sl.do)):
                 dst.copy_(src, non_blocking=True)
             done_in[j].record(s_in)
         with torch.cuda.stream(s_run):
@@ -325,7 +403,7 @@ def bench_ours(args, world, rank, local):
             done_run[j].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(done_run[j])
-            for src, dst in zip((sl.o_g, sl.dq_g, sl.dk_g, sl.dv_g, sl.lse_g), host_out[j]):
+            for src, dst in zip(sl.outputs(), host_out):
                 dst.copy_(src, non_blocking=True)
             done_out[j].record(s_out)
 
@@ -357,54 +435,60 @@ def bench_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "llama-causal-zigzag-16k: B=1 Hq=16 Hkv=8 d=128 N=16384 bf16 "
-                               "P=2 zigzag causal fwd+bwd",
+        "config": {"workload": HEADLINE_NAME,
                    "global_batch": w.B * world, "seq_len": w.N,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "flushed between steps (256 MiB write); inputs 192 MiB > L2"},
+                   "l2": "flushed between steps (256 MiB write); inputs 3 GiB > L2"},
     }
-    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    bwd_tflops = flops_bwd(w) / (bwd_ms * 1e-3) / 1e12
-    fwd_tflops = flops_fwd(w) / (fwd_ms * 1e-3) / 1e12
-    # the dominant tensor-core kernel of the step (the others are HBM copies
-    # worth a few percent of it)
+    peak, peak_note = tensor_peak(peaks, peak_src, step_ms / 1e3, clocks)
+    # the dominant tensor-core kernel of the step
     top = max((k for k in kernels if "TFLOP/s" in kernels[k]), key=lambda k: kernels[k]["share"])
     tk = kernels[top]
     line["roofline"] = {
-        "bound": "tensor", "kernel": top, "achieved": tk["TFLOP/s"], "peak": sustained,
-        "unit": "TFLOP/s", "frac": round(tk["TFLOP/s"] / sustained, 4),
-        "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": TRAFFIC.get(top),
+        "bound": "tensor", "kernel": top, "achieved": tk["TFLOP/s"], "peak": peak,
+        "unit": "TFLOP/s", "frac": round(tk["TFLOP/s"] / peak, 4), "peak_source": peak_note,
+        "traffic": TRAFFIC.get(top),
         "frac_of_burst": round(tk["TFLOP/s"] / peaks["bf16_tflops"], 4),
+        "frac_of_sustained": round(tk["TFLOP/s"] / peaks.get("bf16_tflops_sustained",
+                                                             peaks["bf16_tflops"]), 4),
         "flops_per_launch": tk["flops"], "ms_per_launch": tk["ms"],
     }
     line["kernels"] = kernels
-    line["calls_ms"] = {"ring_fwd": round(fwd_ms, 4), "ring_bwd": round(bwd_ms, 4)}
-    line["ring_fwd_tflops"] = round(fwd_tflops, 2)
-    line["ring_bwd_tflops"] = round(bwd_tflops, 2)
+    line["calls_ms"] = {"repack_q_kv": round(repack_ms, 4), "ring_fwd": round(fwd_ms, 4),
+                        "ring_bwd": round(bwd_ms, 4)}
+    line["ring_fwd_tflops"] = round(flops_fwd(w) / (fwd_ms * 1e-3) / 1e12, 2)
+    line["ring_bwd_tflops"] = round(flops_bwd(w) / (bwd_ms * 1e-3) / 1e12, 2)
+    rb = step.repack_bytes()
+    line["repack_gbs"] = round(rb / repack_ms / 1e6, 1)
     line["e2e"] = {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4),
                    "pipeline": "2 device slots; host->device copy, step and device->host copy "
                                "on 3 streams (step i+1 in, step i-1 out during step i)"}
     line["gpu_launches"] = len(records)
-    line["clocks"] = clk.summary()
-    del step, slots, q, k, v, do
+    line["clocks"] = clocks
+    del step, slots, q, kv, do, host_out, hq, hkv, hdo
     torch.cuda.empty_cache()
 
     if not args.no_extras:
         line["extras"] = extras(rm, peaks, peak_src, dev, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_sample_heads)
+        line["cpu_baseline"] = cpu_baseline(args.ref_sample_queries)
     return line
 
 
-def _time(fn, reps, flush, rm=None):
+_RECORDS = []  # per-launch (name, ms) of the last _time(..., keep=True) call
+
+
+def _time(fn, reps, flush, rm=None, keep=False):
     """Median device time of fn() in ms.  A short spin kernel runs before the
     start event, so the host has queued fn's launches before the GPU reaches
     them and the interval holds no host time.  With `rm`, the median of the
     summed per-launch event times the library records around its own kernels
     is returned too: (kernels, call) (the kernels alone, no gaps between
-    launches)."""
+    launches); with `keep` the per-launch records are left in _RECORDS."""
     ts, ks = [], []
+    if keep:
+        _RECORDS.clear()
     for _ in range(reps):
         if flush is not None:
             flush_l2(flush)
@@ -418,7 +502,10 @@ def _time(fn, reps, flush, rm=None):
         b.record()
         torch.cuda.synchronize()
         if rm is not None:
-            ks.append(sum(ms for _, ms in rm.profile_records()))
+            recs = rm.profile_records()
+            ks.append(sum(ms for _, ms in recs))
+            if keep:
+                _RECORDS.extend(recs)
             rm.profile_enable(False)
         ts.append(a.elapsed_time(b))
     if rm is None:
@@ -455,6 +542,7 @@ def extras(rm, peaks, peak_src, dev, flush, only=None, small=False):
         "merge": lambda: merge_lines(rm, dev, flush, hbm, peak_src, 8 if small else 1),
         "repack": lambda: repack_line(rm, dev, flush, hbm, peak_src, 8 if small else 1),
         "striped_128k": lambda: striped_lines(rm, dev, flush, peaks, hbm, peak_src, small),
+        "llama_16k": lambda: llama_16k_line(rm, flush, peaks, peak_src),
         "tabular_row": lambda: {"tabular_row_fwd": tabular(rm, flush, hbm, peak_src, "row")},
         "tabular_feature": lambda: {"tabular_feature_fwd": tabular(rm, flush, hbm, peak_src,
                                                                    "feature")},
@@ -469,8 +557,8 @@ def extras(rm, peaks, peak_src, dev, flush, only=None, small=False):
     return out
 
 
-EXTRA_GROUPS = ("merge", "repack", "striped_128k", "tabular_row", "tabular_feature", "usp",
-                "mesh2d")
+EXTRA_GROUPS = ("merge", "repack", "striped_128k", "llama_16k", "tabular_row", "tabular_feature",
+                "usp", "mesh2d")
 
 
 def merge_lines(rm, dev, flush, hbm, peak_src, div=1):
@@ -511,6 +599,51 @@ def repack_line(rm, dev, flush, hbm, peak_src, div=1):
                               f"[8, {8 * Ln}, 2, 128] bf16")}
 
 
+def step_line(rm, w, flush, peaks, peak_src, reps):
+    """fwd+bwd of workload w (fused ring forward + ring backward on
+    global-order operands, as in the headline step, without the repack):
+    per-call times, TFLOP/s and the kernels' per-launch rates.  Burst peak:
+    each timed call lasts well under a second."""
+    q_h, k_h, v_h, do_h = synthetic.attention_inputs(w)
+    dev = torch.device("cuda")
+    q, kv, do = q_h.to(dev), fused_kv(k_h, v_h).to(dev), do_h.to(dev)
+    del q_h, k_h, v_h, do_h
+    st = Step(rm, w, q, kv, do, repack=False)
+    fwd = lambda: rm.ring_attn_fwd(st.q, st.k, st.v, P=w.P, layout=w.layout, causal=w.causal,
+                                   order="global", out=st.o, lse=st.lse)
+    bwd = lambda: rm.ring_attn_bwd(st.q, st.k, st.v, st.o, st.lse, st.do, P=w.P, layout=w.layout,
+                                   causal=w.causal, order="global", dq=st.dq, dk=st.dk, dv=st.dv,
+                                   ws=st.ws)
+    fwd()
+    bwd()
+    _, ms_f = _time(fwd, reps, flush, rm, keep=True)
+    recs = list(_RECORDS)
+    _, ms_b = _time(bwd, reps, flush, rm, keep=True)
+    recs += _RECORDS
+    burst = peaks["bf16_tflops"]
+    tf_f = flops_fwd(w) / (ms_f * 1e-3) / 1e12
+    tf_b = flops_bwd(w) / (ms_b * 1e-3) / 1e12
+    tf = (flops_fwd(w) + flops_bwd(w)) / ((ms_f + ms_b) * 1e-3) / 1e12
+    kern = {}
+    for name, ms in recs:
+        kern.setdefault(name, []).append(ms)
+    kernels = {}
+    for name, v in kern.items():
+        e = {"ms": round(statistics.median(v), 4)}
+        if name in FLOPS_PER_PAIR:
+            e["TFLOP/s"] = round(FLOPS_PER_PAIR[name] * w.d * causal_pairs(w)
+                                 / (statistics.median(v) * 1e-3) / 1e12, 2)
+            e["frac"] = round(e["TFLOP/s"] / burst, 4)
+        kernels[name] = e
+    del st, q, kv, do
+    return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} N={w.N} P={w.P} "
+                        f"{w.layout} causal fwd+bwd", "fwd_ms": round(ms_f, 3),
+            "bwd_ms": round(ms_b, 3), "fwd_TFLOP/s": round(tf_f, 2), "bwd_TFLOP/s": round(tf_b, 2),
+            "TFLOP/s": round(tf, 2), "frac": round(tf / burst, 4), "fwd_frac": round(tf_f / burst, 4),
+            "peak": burst, "peak_source": f"{peak_src} bf16_tflops (burst: calls of under a second)",
+            "kernels": kernels}
+
+
 def striped_lines(rm, dev, flush, peaks, hbm, peak_src, small=False):
     out = {}
     w3 = synthetic.STRIPED_128K
@@ -521,26 +654,21 @@ def striped_lines(rm, dev, flush, peaks, hbm, peak_src, small=False):
         out["permute"] = hbm_row(rm, fn, 10, flush, 2 * q.numel() * 2, hbm, peak_src,
                                  f"striped P=8 [1, {w3.N // 2}, 16, 128] bf16")
         return out
-    # the causal striped 128k forward (fused ring over 8 virtual ranks)
-    q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
-    k = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
-    v = torch.randn(1, w3.N, w3.Hkv, w3.d, device=dev).mul_(0.5).to(torch.bfloat16)
-    o = torch.empty_like(q)
-    lse = torch.empty(1, w3.Hq, w3.N, device=dev)
-    fn = lambda: rm.ring_attn_fwd(q, k, v, P=8, layout="striped", causal=True, out=o, lse=lse)
-    fn()
-    ms = _time(fn, 3, flush)
-    tf = flops_fwd(w3) / (ms * 1e-3) / 1e12
-    out["striped_128k_fwd"] = {"ms": round(ms, 3), "TFLOP/s": round(tf, 2),
-                               "frac": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
-                               "peak_source": f"{peak_src} bf16_tflops (burst: one kernel timed alone)"}
+    # the causal striped 128k workload, fwd+bwd (the forward alone is its gate)
+    out["striped_128k_fwd_bwd"] = step_line(rm, w3, flush, peaks, peak_src, 3)
+    torch.cuda.empty_cache()
     # layout permute of the striped 128k Q (global -> rank-major), 2 x 512 MiB
+    q = torch.randn(1, w3.N, w3.Hq, w3.d, device=dev).to(torch.bfloat16)
     o2 = torch.empty_like(q)
     fn = lambda: rm.layout_permute(q, "striped", 8, out=o2)
     nbytes = 2 * q.numel() * 2
     out["permute"] = hbm_row(rm, fn, 10, flush, nbytes, hbm, peak_src,
                              "striped P=8 [1, 131072, 16, 128] bf16")
     return out
+
+
+def llama_16k_line(rm, flush, peaks, peak_src):
+    return {"llama_16k_fwd_bwd": step_line(rm, synthetic.LLAMA_ZIGZAG, flush, peaks, peak_src, 10)}
 
 
 def mesh2d_line(rm, flush, peaks, peak_src):
@@ -570,8 +698,8 @@ def mesh2d_line(rm, flush, peaks, peak_src):
     tf = (flops_fwd(w) + flops_bwd(w)) / ((ms_f + ms_b) * 1e-3) / 1e12
     return {"grid": f"{g} x {g} (36 live tiles)", "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3),
             "fwd_TFLOP/s": round(tf_f, 2), "TFLOP/s": round(tf, 2),
-            "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
-            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peak_src} bf16_tflops (burst: calls of under a second)",
             "note": "fwd: 36 tile launches + 8 merges; bwd: delta, 2 x 36 tile launches (fp32 "
                     "accumulators), 3 converts"}
 
@@ -600,8 +728,8 @@ def usp_line(rm, flush, peaks, peak_src):
     ms = _time(fn, 5, flush)
     tf = (flops_fwd(w) + flops_bwd(w)) / (ms * 1e-3) / 1e12
     return {"split": f"ulysses {u} x ring {p_ring} ({w.layout})", "ms": round(ms, 4),
-            "TFLOP/s": round(tf, 2), "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
-            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "TFLOP/s": round(tf, 2), "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peak_src} bf16_tflops (burst: calls of under a second)",
             "note": "includes the 8 repack launches of Q/K/V/O/dO and dQ/dK/dV"}
 
 
@@ -656,32 +784,47 @@ def tabular(rm, flush, hbm, peak_src, axis):
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline / reference arm)
 # ---------------------------------------------------------------------------
-SAMPLE_ROWS = (4096, 6144)  # local query indices of virtual rank 0 in the sample
+_INPUTS = {}
 
 
-def oracle_sample(heads: int = 1):
-    """The oracle's ring fwd+bwd for 2048 queries of virtual rank 0 of `heads`
-    query head(s) (with their KV head) of the Llama-like zigzag workload: the
-    queries' partials against both KV shards, their LSE merge, then their
-    backward contributions (their dQ, their share of dK / dV).  The rows are
-    rank 0's local indices 4096..6143, global positions 12288..14335 (the
-    second zigzag chunk), whose score rows are mostly visible.
-    Returns (seconds, algorithmic flops of the sample)."""
+def _headline_inputs():
+    """The headline workload's inputs (drawn once per process: 17 s of CPU)."""
+    if "w" not in _INPUTS:
+        _INPUTS["w"] = synthetic.attention_inputs(HEADLINE)
+    return _INPUTS["w"]
+
+
+def sample_desc(n_queries: int) -> str:
+    w = HEADLINE
+    return (f"oracle ring fwd+bwd (numpy fp64) for the last {n_queries} queries (global positions "
+            f"{w.N - n_queries}-{w.N - 1}, virtual rank 0's second zigzag chunk) of query head 0, "
+            f"against all {w.N} keys they see in the {w.P} KV shards, N={w.N} zigzag P={w.P}; "
+            f"the repack is not part of the sample")
+
+
+def oracle_sample(n_queries: int = 512):
+    """The oracle's ring fwd+bwd for the last `n_queries` queries of query
+    head 0 (with KV head 0) of the headline workload: their partials against
+    every KV shard in ring order, the LSE merge, the row term, then their
+    backward contributions (their dQ, their share of dK / dV) against every
+    shard.  Rows of the sequence's end see nearly every key, so the sample is
+    the workload's densest part.  Returns (seconds, algorithmic flops)."""
     from oracle import attention as oatt
     from oracle import layouts as olay
     from oracle import merge as omerge
     from oracle import ring as oring
-    w = synthetic.LLAMA_ZIGZAG
-    q, k, v, do = synthetic.attention_inputs(w)
-    hk = max(1, heads // (w.Hq // w.Hkv))
-    f = lambda t, n: t[:, :, :n].float().numpy().astype(np.float64)
-    qs, ks, vs, dos = f(q, heads), f(k, hk), f(v, hk), f(do, heads)
-    L, r = w.N // w.P, 0
-    j0, j1 = SAMPLE_ROWS
+    w = HEADLINE
+    q, k, v, do = _headline_inputs()
+    f = lambda t: t[:, :, :1].float().numpy().astype(np.float64)
+    qs, ks, vs, dos = f(q), f(k), f(v), f(do)
+    L, C = w.N // w.P, w.N // (2 * w.P)
     t0 = time.perf_counter()
     perm = lambda x: olay.permute(x, w.layout, w.P)
     qr, kr, vr, dor = perm(qs), perm(ks), perm(vs), perm(dos)
     pos = [olay.rank_positions(w.layout, w.N, w.P, s) for s in range(w.P)]
+    r = 0
+    j0, j1 = L - n_queries, L  # the end of rank 0's second chunk (2P - 1)
+    assert j1 - j0 <= C
     rows = slice(r * L + j0, r * L + j1)
     qpos = pos[r][j0:j1]
     parts = []
@@ -697,7 +840,7 @@ def oracle_sample(heads: int = 1):
                                       delta, causal=w.causal, q_pos=qpos, k_pos=pos[s])
     secs = time.perf_counter() - t0
     # visible pairs: the query at global position t sees t + 1 keys
-    pairs = int((qpos + 1).sum()) * heads
+    pairs = int((qpos + 1).sum())
     return secs, 14.0 * w.d * pairs
 
 
@@ -719,39 +862,44 @@ def _cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(heads: int):
-    secs, flops = oracle_sample(heads)
-    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
-            "cpu_model": _cpu_model(), "kind": "oracle",
-            "sample": f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions "
-                      f"12288-14335, virtual rank 0) of {heads} of 16 query heads, N=16384 zigzag "
-                      f"P=2; {secs:.1f} s"}
+def cpu_baseline(n_queries: int, reps: int = 3):
+    """The oracle on `reps` runs of the sample (about 10-30 s of CPU in all);
+    the rate extrapolated to the whole headline step is stated beside it."""
+    secs, flops = 0.0, 0.0
+    for _ in range(reps):
+        s_, f_ = oracle_sample(n_queries)
+        secs += s_
+        flops += f_
+    rate = flops / secs
+    step_flops = flops_fwd(HEADLINE) + flops_bwd(HEADLINE)
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
+            "cpu_model": _cpu_model(), "kind": "oracle", "sample": sample_desc(n_queries),
+            "runs": reps, "seconds": round(secs, 2),
+            "extrapolated_step_s": round(step_flops / rate, 1),
+            "extrapolated": "the whole fwd+bwd step at the sample's rate"}
 
 
 def bench_reference(args, world, rank):
     if rank != 0:
         return None
     for _ in range(args.warmup):
-        oracle_sample(args.ref_sample_heads)
+        oracle_sample(args.ref_sample_queries)
     secs, flops = 0.0, 0.0
     for _ in range(args.steps):
-        s, f = oracle_sample(args.ref_sample_heads)
-        secs += s
-        flops += f
+        s_, f_ = oracle_sample(args.ref_sample_queries)
+        secs += s_
+        flops += f_
     value = flops / secs / 1e12
-    sample = (f"oracle ring fwd+bwd (numpy fp64) for 2048 queries (global positions 12288-14335, "
-              f"virtual rank 0) of {args.ref_sample_heads} of 16 query heads, N=16384 zigzag P=2, "
-              f"per step")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "llama-causal-zigzag-16k: B=1 Hq=16 Hkv=8 d=128 N=16384 bf16 "
-                               "P=2 zigzag causal fwd+bwd", "global_batch": 1, "seq_len": 16384,
+        "config": {"workload": HEADLINE_NAME, "global_batch": 1, "seq_len": HEADLINE.N,
                    "parallelism": "single"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(),
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle",
+                         "sample": sample_desc(args.ref_sample_queries) + ", per step"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -765,10 +913,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-heads", type=int, default=16,
-                    help="query heads in the oracle sample of cpu_baseline")
-    ap.add_argument("--ref-sample-heads", type=int, default=4,
-                    help="query heads in each --impl reference step")
+    ap.add_argument("--ref-sample-queries", type=int, default=512,
+                    help="queries in each oracle sample (cpu_baseline and --impl reference)")
     ap.add_argument("--case", choices=EXTRA_GROUPS, default=None,
                     help="run only this group of the extra measurements (no step, no baseline)")
     ap.add_argument("--small", action="store_true",

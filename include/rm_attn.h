@@ -230,11 +230,21 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
  * rm_ring_attn_bwd, minus the workspace: the scratch comes from a fixed
  * 64 MiB device array inside the library, so rm_ring_workspace_size(desc, 1)
  * must be at most 64 MiB (else RM_ERR_WORKSPACE, nothing launched).
- * The array is resolved on the first call on each device (with that device
- * current); make that first call before any stream capture.  Every GPU that
- * has made a call holds the 64 MiB until the process exits.  All calls share
- * the one array per device: calls whose kernels overlap on the GPU (several
- * streams, or several threads) race and give wrong results -- serialise them.
+ * When the 64 MiB is reserved depends on how CUDA loads modules: with lazy
+ * loading (CUDA_MODULE_LOADING=LAZY, the default of recent runtimes) the
+ * first call in a context loads the library's device code and reserves it
+ * then; with eager loading every context that loads the library reserves it
+ * at once, whether or not it ever calls this function.  Either way it stays
+ * reserved until the context ends.  So make the first call in each context
+ * before any stream capture and before the caller hands the rest of device
+ * memory to its own pool: under lazy loading that first call may otherwise
+ * fail with RM_ERR_CUDA for lack of memory.  The array's device address is
+ * looked up on every call in the current context, so a device reset or a
+ * context switch between calls is safe.  All calls share the one array per
+ * context: calls whose kernels overlap on the GPU (several streams, or
+ * several threads) race and give wrong results -- serialise them.  Each call
+ * writes the scratch it reads before reading it, so the previous call's
+ * contents do not reach its results.
  * Calls no cudaMalloc / cudaFree / allocating library routine. */
 rm_status rm_ring_attn_bwd_noalloc(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
                                    rm_tensor v, rm_tensor o, const float* lse,
@@ -346,6 +356,15 @@ const char* rm_last_error(void);
  * mbarrier nothing arrives at, giving up after `spin_limit` polls, and records
  * RM_ERR_TIMEOUT in the device status word.  Faults and hangs nothing. */
 rm_status rm_debug_expire_wait(uint32_t spin_limit, void* stream);
+
+/* Test hook for the polynomial exponential that the tensor-core forward uses
+ * on the FMA pipe for part of its softmax at head dims up to 64 (the pages fix
+ * no way of computing exp; this is an implementation choice of the kernel):
+ * y[i] = that function's 2^x[i] for i < n.  x, y: device fp32 arrays of n
+ * elements (caller-owned; they must not overlap).  Stated accuracy: relative
+ * error at most 7.5e-5 for x in [-125, 127]; inputs below -125 (and -inf)
+ * are clamped to -125.  RM_ERR_INVALID_ARG for n < 0 or null pointers. */
+rm_status rm_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /* ---- launch timing ------------------------------------------------------ */
 

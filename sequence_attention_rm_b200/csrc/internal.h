@@ -95,5 +95,6 @@ cudaError_t launch_small_seq_fwd(const AttnArgs& a, int q_rank, int kv_rank, int
 
 cudaError_t launch_debug_expire_wait(uint32_t spin_limit, unsigned int* status,
                                      cudaStream_t stream);
+cudaError_t launch_debug_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 }  // namespace rm

@@ -1,15 +1,13 @@
 // Ring backward that allocates nothing.
 //
 // The ring backward needs scratch device memory: the row term
-// delta = rowsum(dO * O), one fp32 value per (batch, query head, token).  Most callers pass a workspace they allocated; some
-// cannot: for example a runtime that reserved all device memory for its own
+// delta = rowsum(dO * O), one fp32 value per (batch, query head, token).
+// Most callers pass a workspace they allocated; some cannot: for example a runtime that reserved all device memory for its own
 // pool at start-up and hands out no raw allocations, or code that must not
 // call cudaMalloc because it would synchronise the device.  For them this
 // file keeps one fixed scratch array in device memory and forwards to the
 // ordinary ring backward with it as the workspace.
 #include <stdio.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -24,33 +22,23 @@ constexpr size_t kScratchBytes = 64ull << 20;  // 64 MiB on every device that us
 // cudaGetSymbolAddress below.
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices];
-
-// Device address of the scratch on the current device, resolved once per
-// device with that device current.
+// Device address of the scratch in the current context, looked up on every
+// call.  A __device__ array's address belongs to the context that loaded the
+// module, not to the device ordinal: after cudaDeviceReset, or with another
+// driver-API context current, an address cached from an earlier call would
+// point into memory that is no longer (or never was) this context's.  Once
+// the module is loaded the lookup is a table search.
 rm_status scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    set_last_error("rm_ring_attn_bwd_noalloc: no usable current device");
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+  if (e != cudaSuccess || !p) {
+    char buf[256];
+    snprintf(buf, sizeof(buf), "rm_ring_attn_bwd_noalloc: cudaGetSymbolAddress failed: %s",
+             cudaGetErrorString(e));
+    set_last_error(buf);
     return RM_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess || !p) {
-      char buf[256];
-      snprintf(buf, sizeof(buf), "rm_ring_attn_bwd_noalloc: cudaGetSymbolAddress failed: %s",
-               cudaGetErrorString(e));
-      set_last_error(buf);
-      return RM_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return RM_OK;
 }
 

@@ -39,7 +39,6 @@ rm_status cuda_fail(cudaError_t e, const char* where) {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_sms[kMaxDevices];
-unsigned int* g_status_ptr[kMaxDevices];
 
 int current_device() {
   int dev = 0;
@@ -190,15 +189,15 @@ int num_sms() {
   return g_sms[dev];
 }
 
+// The status word's device address in the current context.  It is looked up
+// on every call, not cached: a __device__ variable's address belongs to the
+// context that loaded the module, and a caller may switch contexts or reset
+// the device between calls (the lookup is a table search once the module is
+// loaded).
 unsigned int* status_word() {
-  int dev = current_device();
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = (unsigned int*)p;
-  }
-  return g_status_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  return (unsigned int*)p;
 }
 
 }  // namespace rm
@@ -233,6 +232,13 @@ rm_status rm_get_device_status(void* stream) {
   if (v & kStatusTimeout) return fail(RM_ERR_TIMEOUT, "a device-side bounded wait expired");
   if (v & kStatusSmemAlign)
     return fail(RM_ERR_CUDA, "a kernel found its dynamic shared memory not 1024-byte aligned");
+  return RM_OK;
+}
+
+rm_status rm_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y)))
+    return fail(RM_ERR_INVALID_ARG, "rm_debug_exp2_poly: bad pointers or size");
+  RM_CUDA(launch_debug_exp2_poly(x, y, n, (cudaStream_t)stream), "exp2 poly launch");
   return RM_OK;
 }
 

@@ -29,7 +29,7 @@ EXPORTED = (
     "rm_attn_block_fwd", "rm_attn_block_bwd", "rm_attn_bwd_preprocess", "rm_lse_merge",
     "rm_ring_workspace_size", "rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_layout_permute",
     "rm_seq_head_repack", "rm_get_device_status", "rm_status_string", "rm_last_error",
-    "rm_debug_expire_wait", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
+    "rm_debug_expire_wait", "rm_debug_exp2_poly", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
     "rm_profile_get", "rm_usp_auto_select", "rm_usp_workspace_size", "rm_usp_attn_fwd",
     "rm_usp_attn_bwd", "rm_mesh2d_workspace_size", "rm_mesh2d_attn_fwd", "rm_mesh2d_attn_bwd",
 )
@@ -74,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_seq_head_repack": [i, i, i64, i, i, i, vp, vp, vp],
         "rm_get_device_status": [vp],
         "rm_debug_expire_wait": [ctypes.c_uint32, vp],
+        "rm_debug_exp2_poly": [vp, vp, i64, vp],
         "rm_ring_attn_bwd_noalloc": [D, T, T, T, T, vp, T, T, T, T, vp],
         "rm_profile_enable": [i],
         "rm_profile_count": [],
@@ -387,6 +388,15 @@ def get_device_status(stream=None) -> int:
 
 def debug_expire_wait(spin_limit: int, stream=None) -> None:
     _check(_lib.rm_debug_expire_wait(spin_limit, _stream(stream)))
+
+
+def debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The forward's FMA-pipe 2^x on a contiguous fp32 CUDA tensor (test hook)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("debug_exp2_poly needs a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(_lib.rm_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def profile_enable(on: bool) -> None:

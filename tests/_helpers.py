@@ -33,11 +33,28 @@ def assert_max_abs(got, ref, tol, what=""):
     assert err <= tol, f"{what}: max-abs error {err:.3e} > {tol:.1e}"
 
 
+def rel_l2(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = float(np.linalg.norm(ref))
+    return float(np.linalg.norm(got - ref)) / den if den > 0 else float(np.linalg.norm(got))
+
+
 def assert_grad_close(got, ref, tol=BF16_GRAD_TOL, what=""):
+    """Max-abs within tol x max(1, max|ref|); prints the scale and the
+    relative L2 error beside it (shown with pytest -s or on failure)."""
     ref = np.asarray(ref, dtype=np.float64)
     scale = max(1.0, float(np.abs(ref).max()) if ref.size else 1.0)
     err = max_abs(got, ref)
-    assert err <= tol * scale, f"{what}: max-abs error {err:.3e} > {tol:.1e} x {scale:.2f}"
+    rl2 = rel_l2(got, ref) if ref.size else 0.0
+    print(f"{what}: max-abs {err:.3e} (bound {tol:.1e} x scale {scale:.3f}), rel-L2 {rl2:.3e}")
+    assert err <= tol * scale, \
+        f"{what}: max-abs error {err:.3e} > {tol:.1e} x {scale:.2f} (rel-L2 {rl2:.3e})"
+
+
+def assert_f32_close(got, ref, what=""):
+    """fp32 inputs: max-abs within 1e-5 x max(1, max|ref|)."""
+    assert_grad_close(got, ref, tol=F32_TOL, what=what)
 
 
 def requires_cuda():

@@ -147,6 +147,12 @@ def test_usp_auto_select_matches_the_rule(rm):
     assert rm.usp_auto_select(64, 16, 32, node_size=8) == (8, 4)
 
 
+def test_usp_auto_select_hand_table(rm):
+    from tests.test_oracle_usp import SELECTOR_TABLE
+    for (hq, hkv, world, node), want in SELECTOR_TABLE:
+        assert rm.usp_auto_select(hq, hkv, world, node_size=node) == want
+
+
 @pytest.mark.parametrize("kw,u", [(dict(), 3), (dict(), 16), (dict(N=16386, P=2), 4),
                                   (dict(Hq=12, Hkv=6), 4),
                                   (dict(seq_lens=16), 2)])  # no segments under USP

@@ -11,7 +11,7 @@ from oracle import layouts as olay
 from oracle import merge as omerge
 from oracle import repack as orepack
 from sequence_attention_rm_b200 import synthetic
-from tests._helpers import BF16_O_TOL, F32_TOL, assert_max_abs, gpu, np64
+from tests._helpers import BF16_O_TOL, F32_TOL, assert_f32_close, assert_max_abs, gpu, np64
 
 pytestmark = gpu
 
@@ -60,13 +60,28 @@ def test_seq_head_repack_bit_exact(rm, dtype, P, L, H, d):
     assert np.array_equal(orepack.head_to_seq(ref, P), _bits(x))
 
 
-def test_repack_workload_shapes(rm):
-    # Q [8 x 2048, 16, 128] and fused K|V [8 x 2048, 8+8, 128] sequence-sharded -> head-sharded
-    for H in (16, 8):
-        x = synthetic.tensor(5000 + H, (8, 2048, H, 128), torch.bfloat16)
-        y = rm.seq_head_repack(x.cuda(), 8)
-        assert y.shape == (8, 8 * 2048, H // 8, 128)
-        assert np.array_equal(_bits(y), orepack.seq_to_head(_bits(x), 8))
+@pytest.mark.parametrize("L", [2048, 32768], ids=["8x2048", "8x32768-full"])
+def test_repack_workload_shapes(rm, L):
+    """The 256k zigzag workload's repack at its full size (L = 32768 tokens per
+    rank; 1 GiB per tensor) and at 1/16 of it: Q [8 x L, 16, 128], the fused
+    K|V (8 K heads then 8 V heads) of the same shape, and K alone
+    [8 x L, 8, 128], sequence-sharded -> head-sharded and back, bit for bit
+    against the oracle's index loops."""
+    for seed, H in ((5000, 16), (5001, 16), (5002, 8)):
+        x = synthetic.tensor(seed + L, (8, L, H, 128), torch.bfloat16)
+        xb = _bits(x)
+        xd = x.cuda()
+        y = rm.seq_head_repack(xd, 8)
+        assert y.shape == (8, 8 * L, H // 8, 128)
+        ref = orepack.seq_to_head(xb, 8)
+        assert np.array_equal(_bits(y), ref)
+        # head -> seq on the oracle's head-sharded tensor (not on the kernel's)
+        back = rm.seq_head_repack(torch.from_numpy(ref).view(torch.bfloat16).cuda(), 8,
+                                  head_to_seq=True)
+        assert np.array_equal(_bits(back), orepack.head_to_seq(ref, 8))
+        assert np.array_equal(_bits(back), xb)
+        del xd, y, back
+        torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
@@ -112,7 +127,7 @@ def test_bwd_preprocess(rm, dtype, B, N, H, d):
     do = synthetic.tensor(801, (B, N, H, d), dtype)
     ref = oatt.delta_from_output(np64(do), np64(o))
     got = rm.attn_bwd_preprocess(o.cuda(), do.cuda())
-    assert_max_abs(np64(got), ref, 1e-4 * max(1.0, np.abs(ref).max()), "delta")
+    assert_f32_close(np64(got), ref, "delta")
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(rm):
@@ -166,4 +181,4 @@ def test_bwd_preprocess_strided_views(rm, offset):
     o, do = wide_o[..., offset:offset + d], wide_do[..., offset:offset + d]
     ref = oatt.delta_from_output(np64(do), np64(o))
     got = rm.attn_bwd_preprocess(o, do)
-    assert_max_abs(np64(got), ref, 1e-4 * max(1.0, np.abs(ref).max()), "delta")
+    assert_f32_close(np64(got), ref, "delta")

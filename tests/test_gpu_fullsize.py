@@ -2,7 +2,8 @@
 workloads (16k zigzag P=2, 128k striped P=8, 256k zigzag P=8): the
 rank-major ring (after a layout permute) is checked against the oracle, and
 the launch configuration bench.py times (fused ring forward and ring
-backward on global-order operands) must reproduce its results bit for bit.
+backward on global-order operands, K and V as views of one fused buffer)
+must reproduce its results bit for bit.
 
 The oracle cannot materialise these problems, so it checks what it can
 compute exactly one by one:
@@ -73,7 +74,19 @@ def test_full_size_ring_fwd_bwd(rm, w):
     assert torch.equal(og.cpu(), o_g) and torch.equal(lg.cpu(), lse_g), "global-order forward"
     for name, a, ref in zip(("dq", "dk", "dv"), grads, (dq_g, dk_g, dv_g)):
         assert torch.equal(a.cpu(), ref), f"global-order {name}"
-    del qd, kd, vd, dod, og, lg, grads
+    del kd, vd, og, lg, grads
+    torch.cuda.empty_cache()
+    # ... and with K and V as head views of one fused [B, N, 2 Hkv, d] buffer
+    # (K heads first), the operand form bench.py times
+    kv = torch.cat([k, v], dim=2).to(dev)
+    kf, vf = kv[:, :, :w.Hkv], kv[:, :, w.Hkv:]
+    og, lg = rm.ring_attn_fwd(qd, kf, vf, P=w.P, layout=w.layout, causal=True, order="global")
+    grads = rm.ring_attn_bwd(qd, kf, vf, og, lg, dod, P=w.P, layout=w.layout, causal=True,
+                             order="global")
+    assert torch.equal(og.cpu(), o_g) and torch.equal(lg.cpu(), lse_g), "fused K|V forward"
+    for name, a, ref in zip(("dq", "dk", "dv"), grads, (dq_g, dk_g, dv_g)):
+        assert torch.equal(a.cpu(), ref), f"fused K|V {name}"
+    del qd, kv, kf, vf, dod, og, lg, grads
     torch.cuda.empty_cache()
     assert rm.get_device_status() == rm.RM_OK
 

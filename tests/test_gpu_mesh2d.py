@@ -10,7 +10,8 @@ import torch
 
 from oracle import mesh2d as omesh
 from sequence_attention_rm_b200 import synthetic
-from tests._helpers import (BF16_LSE_TOL, BF16_O_TOL, F32_TOL, assert_grad_close, assert_max_abs,
+from tests._helpers import (BF16_LSE_TOL, BF16_O_TOL, F32_TOL, assert_f32_close, assert_grad_close,
+                            assert_max_abs,
                             gpu, np64)
 
 pytestmark = gpu
@@ -61,7 +62,7 @@ def test_mesh2d_matches_oracle(rm, case):
     for name, g, ref in zip(("dq", "dk", "dv"), grads, g_ref):
         assert g.dtype == dtype
         if dtype == torch.float32:
-            assert_max_abs(np64(g), ref, 1e-4, name)
+            assert_f32_close(np64(g), ref, name)
         else:
             assert_grad_close(np64(g), ref, what=name)
 

@@ -10,7 +10,8 @@ from oracle import attention as oatt
 from oracle import layouts as olay
 from oracle import usp as ousp
 from sequence_attention_rm_b200 import synthetic
-from tests._helpers import (BF16_LSE_TOL, BF16_O_TOL, F32_TOL, assert_grad_close, assert_max_abs,
+from tests._helpers import (BF16_LSE_TOL, BF16_O_TOL, F32_TOL, assert_f32_close, assert_grad_close,
+                            assert_max_abs,
                             gpu, np64)
 
 pytestmark = gpu
@@ -57,7 +58,7 @@ def test_usp_matches_oracle(rm, case):
     grads = rm.usp_attn_bwd(qg, kg, vg, o, l, dog, P=P, ulysses=U, layout=layout, causal=causal)
     for name, g, ref in zip(("dq", "dk", "dv"), grads, g_ref):
         if dtype == torch.float32:
-            assert_max_abs(np64(g), ref, 1e-4, name)
+            assert_f32_close(np64(g), ref, name)
         else:
             assert_grad_close(np64(g), ref, what=name)
 

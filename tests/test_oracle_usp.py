@@ -56,17 +56,42 @@ def test_usp_head_groups_are_independent():
     assert not np.allclose(o1[:, :, 2:], o2[:, :, 2:])
 
 
-def test_auto_select_rule_by_brute_force():
+# (Hq, Hkv, world, node_size) -> (ulysses, ring), worked out by hand from the
+# reading of ringmaster "Why" (an auto-selector driven by the KV-head count and
+# the world size; the Ulysses degree is capped by the KV heads): the Ulysses
+# degree is the largest u that divides both the world and the KV-head count
+# and fits in one node; the ring takes the rest of the world.
+SELECTOR_TABLE = [
+    ((16, 8, 8, 8), (8, 1)),      # the whole world fits the 8 KV heads
+    ((16, 8, 16, 8), (8, 2)),
+    ((32, 4, 16, 8), (4, 4)),     # capped by 4 KV heads
+    ((64, 16, 32, 8), (8, 4)),    # capped by the node size
+    ((64, 16, 32, 16), (16, 2)),
+    ((8, 1, 8, 8), (1, 8)),       # one KV head: ring only
+    ((16, 8, 1, 8), (1, 1)),      # one device
+    ((12, 3, 6, 8), (3, 2)),      # non-power-of-two world and head count
+    ((12, 3, 4, 8), (1, 4)),      # 3 and 4 share no factor
+    ((24, 6, 12, 8), (6, 2)),
+    ((24, 6, 12, 4), (3, 4)),     # 6 divides both but exceeds the node
+    ((16, 8, 6, 8), (2, 3)),
+    ((10, 5, 10, 8), (5, 2)),
+    ((14, 7, 7, 8), (7, 1)),
+    ((2, 2, 3, 8), (1, 3)),
+    ((48, 12, 24, 8), (6, 4)),
+]
+
+
+@pytest.mark.parametrize("args,want", SELECTOR_TABLE, ids=lambda x: str(x))
+def test_auto_select_hand_table(args, want):
+    hq, hkv, world, node = args
+    assert usp.auto_select(hq, hkv, world, node_size=node) == want
+
+
+def test_auto_select_split_covers_the_world():
     for hkv in (1, 2, 3, 4, 8, 16):
-        for group in (1, 2, 4):
-            for world in (1, 2, 4, 6, 8, 12, 16, 32):
-                u, r = usp.auto_select(hkv * group, hkv, world)
-                assert u * r == world
-                ok = [x for x in range(1, world + 1) if world % x == 0 and hkv % x == 0 and x <= 8]
-                assert u == max(ok)
-    assert usp.auto_select(16, 8, 8) == (8, 1)
-    assert usp.auto_select(32, 4, 16) == (4, 4)
-    assert usp.auto_select(64, 16, 32, node_size=8) == (8, 4)
+        for world in (1, 2, 4, 6, 8, 12, 16, 32):
+            u, r = usp.auto_select(hkv * 2, hkv, world)
+            assert u * r == world and hkv % u == 0 and u <= 8
 
 
 def test_usp_rejects_bad_splits():

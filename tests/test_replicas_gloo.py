@@ -42,7 +42,7 @@ def _rank_main(rank: int, world: int, port: int, out_dir: str):
     rate = bench.whole_job_rate(2.0e12, 4, w, slowest)
 
     class Args:  # the reference arm's arguments; ranks other than 0 must not run it
-        steps, warmup, ref_sample_heads = 1, 3, 1
+        steps, warmup, ref_sample_queries = 1, 3, 64
 
     ref = bench.bench_reference(Args, w, r) if r != 0 else "not run"
     bench.barrier(w)
@@ -81,7 +81,7 @@ def test_reference_line_contract():
     import bench
 
     class Args:
-        steps, warmup, ref_sample_heads = 1, 3, 1
+        steps, warmup, ref_sample_queries = 1, 3, 64
 
     line = bench.bench_reference(Args, 1, 0)
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC
@@ -89,7 +89,9 @@ def test_reference_line_contract():
     assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
-    assert "1 of 16 query heads" in cb["sample"]
+    assert "last 64 queries" in cb["sample"] and "query head 0" in cb["sample"]
+    assert line["config"]["workload"] == bench.HEADLINE_NAME
+    assert line["config"]["seq_len"] == 262144
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0
     assert e2e["d2h_bytes_per_step"] == 0
