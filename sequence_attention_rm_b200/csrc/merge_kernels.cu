@@ -246,21 +246,45 @@ __global__ void __launch_bounds__(256) convert_f32_kernel(int B, int64_t N, int 
   }
 }
 
-int grid_for_rows(int64_t rows, int rows_per_warp) {
+// Blocks of a 256-thread kernel resident on one SM at once, from the
+// occupancy calculator (registers decide it), cached per device and kernel.
+template <auto Kernel>
+int resident_blocks() {
+  static int per_sm[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& k = per_sm[dev & 63];
+  if (k <= 0 &&
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, Kernel, 256, 0) != cudaSuccess || k <= 0))
+    k = 4;
+  return k;
+}
+
+// Grid of a grid-stride row kernel: enough 8-warp blocks for every warp to
+// get a row group, capped at one wave of resident blocks (a second, partial
+// wave would leave SMs idle at the end while the rest stream).
+int grid_for_rows(int64_t rows, int rows_per_warp, int blocks_per_sm) {
   int64_t warps = (rows + rows_per_warp - 1) / rows_per_warp;
   int64_t blocks = (warps + 7) / 8;
-  int64_t cap = (int64_t)num_sms() * 8;
+  int64_t cap = (int64_t)num_sms() * blocks_per_sm;
   if (blocks > cap) blocks = cap;
   return (int)(blocks < 1 ? 1 : blocks);
 }
 
+template <typename OutT, int NPARTS, bool SAME>
+void launch_merge_kernel(const MergeArgs& a, RowGroup g, int64_t rows, cudaStream_t s) {
+  constexpr auto kern = lse_merge_kernel<OutT, NPARTS, SAME>;
+  const int grid = grid_for_rows(rows, g.rows_per_warp, resident_blocks<kern>());
+  kern<<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp);
+}
+
 template <typename OutT, bool SAME>
-cudaError_t merge_dispatch(const MergeArgs& a, RowGroup g, int grid, cudaStream_t s) {
+cudaError_t merge_dispatch(const MergeArgs& a, RowGroup g, int64_t rows, cudaStream_t s) {
   switch (a.n_parts) {
-    case 2: lse_merge_kernel<OutT, 2, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    case 4: lse_merge_kernel<OutT, 4, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    case 8: lse_merge_kernel<OutT, 8, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
-    default: lse_merge_kernel<OutT, 0, SAME><<<grid, 256, 0, s>>>(a, g.lanes, g.rows_per_warp); break;
+    case 2: launch_merge_kernel<OutT, 2, SAME>(a, g, rows, s); break;
+    case 4: launch_merge_kernel<OutT, 4, SAME>(a, g, rows, s); break;
+    case 8: launch_merge_kernel<OutT, 8, SAME>(a, g, rows, s); break;
+    default: launch_merge_kernel<OutT, 0, SAME>(a, g, rows, s); break;
   }
   return cudaGetLastError();
 }
@@ -271,30 +295,21 @@ cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stre
   const int64_t rows = (int64_t)a.B * a.H * a.Nq;
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(a.d);
-  int grid = grid_for_rows(rows, g.rows_per_warp);
   bool same = a.out_sb == a.o_sb[0] && a.out_sn == a.o_sn[0] && a.out_sh == a.o_sh[0];
   for (int i = 1; i < a.n_parts; ++i)
     same = same && a.o_sb[i] == a.o_sb[0] && a.o_sn[i] == a.o_sn[0] && a.o_sh[i] == a.o_sh[0];
   ProfScope ps("lse_merge", stream);
   if (same)
-    return out_bf16 ? merge_dispatch<__nv_bfloat16, true>(a, g, grid, stream)
-                    : merge_dispatch<float, true>(a, g, grid, stream);
-  return out_bf16 ? merge_dispatch<__nv_bfloat16, false>(a, g, grid, stream)
-                  : merge_dispatch<float, false>(a, g, grid, stream);
+    return out_bf16 ? merge_dispatch<__nv_bfloat16, true>(a, g, rows, stream)
+                    : merge_dispatch<float, true>(a, g, rows, stream);
+  return out_bf16 ? merge_dispatch<__nv_bfloat16, false>(a, g, rows, stream)
+                  : merge_dispatch<float, false>(a, g, rows, stream);
 }
 
 template <int LANES>
 cudaError_t launch_delta_bf16(int B, int64_t N, int H, int d, rm_tensor o, rm_tensor dout,
                               float* delta, cudaStream_t stream) {
-  static int per_sm[64] = {0};  // resident blocks per SM, by device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int& k = per_sm[dev & 63];
-  if (k <= 0 &&
-      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, bwd_delta_bf16_kernel<LANES>, 256, 0) !=
-           cudaSuccess ||
-       k <= 0))
-    k = 4;
+  const int k = resident_blocks<bwd_delta_bf16_kernel<LANES>>();
   const int64_t warps = (int64_t)B * N;  // one token per warp pass
   const int64_t need = (warps + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * k;
@@ -321,14 +336,19 @@ cudaError_t launch_bwd_preprocess(int in_bf16, int B, int64_t N, int H, int d, r
     return launch_delta_bf16<2>(B, N, H, d, o, dout, delta, stream);
   }
   RowGroup g = row_group(d);
-  int grid = grid_for_rows((int64_t)B * N, 1);  // one token per warp pass
   ProfScope ps("bwd_preprocess", stream);
-  if (in_bf16)
-    bwd_preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        B, N, H, d, o, dout, delta, zero_fill, g.lanes, g.rows_per_warp);
-  else
-    bwd_preprocess_kernel<float><<<grid, 256, 0, stream>>>(B, N, H, d, o, dout, delta, zero_fill,
-                                                           g.lanes, g.rows_per_warp);
+  if (in_bf16) {
+    constexpr auto kern = bwd_preprocess_kernel<__nv_bfloat16>;
+    // one token per warp pass
+    const int grid = grid_for_rows((int64_t)B * N, 1, resident_blocks<kern>());
+    kern<<<grid, 256, 0, stream>>>(B, N, H, d, o, dout, delta, zero_fill, g.lanes,
+                                   g.rows_per_warp);
+  } else {
+    constexpr auto kern = bwd_preprocess_kernel<float>;
+    const int grid = grid_for_rows((int64_t)B * N, 1, resident_blocks<kern>());
+    kern<<<grid, 256, 0, stream>>>(B, N, H, d, o, dout, delta, zero_fill, g.lanes,
+                                   g.rows_per_warp);
+  }
   return cudaGetLastError();
 }
 
@@ -337,14 +357,16 @@ cudaError_t launch_convert_f32(int out_bf16, int B, int64_t N, int H, int d, rm_
   const int64_t rows = (int64_t)B * N * H;
   if (rows == 0) return cudaSuccess;
   RowGroup g = row_group(d);
-  int grid = grid_for_rows(rows, g.rows_per_warp);
   ProfScope ps("convert_f32", stream);
-  if (out_bf16)
-    convert_f32_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes,
-                                                                g.rows_per_warp);
-  else
-    convert_f32_kernel<float><<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes,
-                                                        g.rows_per_warp);
+  if (out_bf16) {
+    constexpr auto kern = convert_f32_kernel<__nv_bfloat16>;
+    const int grid = grid_for_rows(rows, g.rows_per_warp, resident_blocks<kern>());
+    kern<<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes, g.rows_per_warp);
+  } else {
+    constexpr auto kern = convert_f32_kernel<float>;
+    const int grid = grid_for_rows(rows, g.rows_per_warp, resident_blocks<kern>());
+    kern<<<grid, 256, 0, stream>>>(B, N, H, d, in, out, g.lanes, g.rows_per_warp);
+  }
   return cudaGetLastError();
 }
 
