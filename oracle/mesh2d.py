@@ -24,6 +24,11 @@ Readings of what the page leaves open:
   probabilities from the final LSE of its rows and uses D_t = dO_t . O_t of
   the final O (as in ``ring``); dQ of chunk i sums over the tiles of row i,
   dK / dV of chunk j over the tiles of column j.
+- Packed and right-padded batches: every tile takes the segment ids of its
+  global positions (``seg``, as in ``attention``), so a key is visible only
+  inside its query's segment; a row with no visible key in a tile has a
+  -inf partial there, and one with none in any tile ends with O = 0 and
+  LSE = -inf.
 
 Tensors are in global token order: q, dout [B, N, Hq, d]; k, v [B, N, Hkv, d];
 lse [B, Hq, N].
@@ -55,7 +60,7 @@ def tile_has_pairs(n: int, grid_q: int, grid_k: int, i: int, j: int, causal: boo
 
 
 def mesh2d_forward(q, k, v, grid_q: int, grid_k: int, causal: bool, scale=None,
-                   return_partials=False):
+                   return_partials=False, seg=None):
     """(o [B, N, Hq, dv], lse [B, Hq, N]); with return_partials also
     partials[i][j] = (o, lse) of tile (i, j) before merging."""
     q = np.asarray(q, dtype=np.float64)
@@ -72,7 +77,8 @@ def mesh2d_forward(q, k, v, grid_q: int, grid_k: int, causal: bool, scale=None,
         for j in range(grid_k):
             kp = chunk(n, grid_k, j)
             row.append(attention.attention_forward(
-                q[:, qp], k[:, kp], v[:, kp], scale=scale, causal=causal, q_pos=qp, k_pos=kp))
+                q[:, qp], k[:, kp], v[:, kp], scale=scale, causal=causal, q_pos=qp, k_pos=kp,
+                seg=seg))
         o_i, lse_i = merge.lse_merge([a for a, _ in row], [b for _, b in row])
         o[:, qp] = o_i
         lse[:, :, qp] = lse_i
@@ -82,7 +88,8 @@ def mesh2d_forward(q, k, v, grid_q: int, grid_k: int, causal: bool, scale=None,
     return o, lse
 
 
-def mesh2d_backward(q, k, v, o, lse, dout, grid_q: int, grid_k: int, causal: bool, scale=None):
+def mesh2d_backward(q, k, v, o, lse, dout, grid_q: int, grid_k: int, causal: bool, scale=None,
+                    seg=None):
     """(dq, dk, dv) in global token order, from the final o and lse."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -101,7 +108,7 @@ def mesh2d_backward(q, k, v, o, lse, dout, grid_q: int, grid_k: int, causal: boo
             kp = chunk(n, grid_k, j)
             gq, gk, gv = attention.attention_backward_block(
                 q[:, qp], k[:, kp], v[:, kp], dout[:, qp], lse[:, :, qp], delta[:, :, qp],
-                scale=scale, causal=causal, q_pos=qp, k_pos=kp)
+                scale=scale, causal=causal, q_pos=qp, k_pos=kp, seg=seg)
             dq[:, qp] += gq
             dk[:, kp] += gk
             dv[:, kp] += gv

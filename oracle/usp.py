@@ -21,6 +21,11 @@ Readings of what the page leaves open:
 - Auto-selection (``auto_select``): the largest Ulysses degree that divides the
   world size and the KV-head count (the Ulysses cap) and fits in one node;
   the ring degree is the rest of the world.
+- Packed and right-padded batches (ringmaster "Status": packing by global
+  position boundaries works whatever the context-parallel strategy): the
+  head exchange moves whole heads and keeps every token's global position,
+  so each head group's ring takes the same segment ids (``seg``, by global
+  position, as in ``attention``) as the unsharded problem.
 """
 
 from __future__ import annotations
@@ -75,7 +80,16 @@ def _head_to_seq(y, p_ring: int, p_ulysses: int):
     return out
 
 
-def usp_forward(q, k, v, layout: str, p_ring: int, p_ulysses: int, causal: bool, scale=None):
+def _seg_of(seg, b):
+    """Segment ids of batch entry b: seg is None, [N] (shared) or [B, N]."""
+    if seg is None:
+        return None
+    seg = np.asarray(seg)
+    return seg[b] if seg.ndim == 2 else seg
+
+
+def usp_forward(q, k, v, layout: str, p_ring: int, p_ulysses: int, causal: bool, scale=None,
+                seg=None):
     """(o, lse): o [B, N, Hq, d] rank-major for p_ring, lse [B, Hq, N]."""
     q = np.asarray(q, dtype=np.float64)
     b_, n, hq, d = q.shape
@@ -88,14 +102,14 @@ def usp_forward(q, k, v, layout: str, p_ring: int, p_ulysses: int, causal: bool,
     for b in range(b_):
         for u in range(p_ulysses):
             o_u, l_u = ring.ring_forward(yq[b, u][None], yk[b, u][None], yv[b, u][None], layout,
-                                         p_ring, causal, scale)
+                                         p_ring, causal, scale, seg=_seg_of(seg, b))
             yo[b, u] = o_u[0]
             lse[b, u * hg:(u + 1) * hg] = l_u[0]
     return _head_to_seq(yo, p_ring, p_ulysses), lse
 
 
 def usp_backward(q, k, v, o, lse, dout, layout: str, p_ring: int, p_ulysses: int, causal: bool,
-                 scale=None):
+                 scale=None, seg=None):
     """(dq, dk, dv) rank-major for p_ring, from the final o and lse."""
     q = np.asarray(q, dtype=np.float64)
     b_, n, hq, d = q.shape
@@ -110,7 +124,8 @@ def usp_backward(q, k, v, o, lse, dout, layout: str, p_ring: int, p_ulysses: int
         for u in range(p_ulysses):
             gq, gk, gv = ring.ring_backward(yq[b, u][None], yk[b, u][None], yv[b, u][None],
                                             yo[b, u][None], lse[b, u * hg:(u + 1) * hg][None],
-                                            ydo[b, u][None], layout, p_ring, causal, scale)
+                                            ydo[b, u][None], layout, p_ring, causal, scale,
+                                            seg=_seg_of(seg, b))
             ydq[b, u], ydk[b, u], ydv[b, u] = gq[0], gk[0], gv[0]
     return (_head_to_seq(ydq, p_ring, p_ulysses), _head_to_seq(ydk, p_ring, p_ulysses),
             _head_to_seq(ydv, p_ring, p_ulysses))

@@ -75,3 +75,52 @@ def test_ring_with_segments_equals_plain(layout, p):
     g = ring.ring_backward(perm(q), perm(k), perm(v), o, l, perm(do), layout, p, True, seg=seg)
     for a, b in zip(g, g_ref):
         np.testing.assert_allclose(layouts.unpermute(a, layout, p), b, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["packed", "padded"])
+@pytest.mark.parametrize("layout", layouts.LAYOUTS)
+def test_usp_with_segments_equals_plain(kind, layout):
+    """USP (Ulysses 2 x ring 2) with segment ids = the plain function with the
+    same ids, after un-permuting: the head exchange keeps global positions."""
+    from oracle import usp
+    p, u, n = 2, 2, 32
+    b_ = 1 if kind == "packed" else 2
+    q, k, v, do = _rand(b_, n, 4, 4), _rand(b_, n, 2, 4), _rand(b_, n, 2, 4), _rand(b_, n, 4, 4)
+    seg = (attention.segments_from_boundaries([0, 3, 11, 12, 29], n) if kind == "packed"
+           else attention.segments_from_lengths([n, 13], n))
+    o_ref, l_ref = attention.attention_forward(q, k, v, causal=True, seg=seg)
+    g_ref = attention.attention_backward(q, k, v, do, causal=True, seg=seg)
+    perm = lambda x: layouts.permute(x, layout, p)
+    o, l = usp.usp_forward(perm(q), perm(k), perm(v), layout, p, u, True, seg=seg)
+    np.testing.assert_allclose(layouts.unpermute(o, layout, p), o_ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(layouts.unpermute(l, layout, p, axis=2), l_ref, rtol=1e-12)
+    g = usp.usp_backward(perm(q), perm(k), perm(v), o, l, perm(do), layout, p, u, True, seg=seg)
+    for a, b in zip(g, g_ref):
+        np.testing.assert_allclose(layouts.unpermute(a, layout, p), b, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["packed", "padded"])
+@pytest.mark.parametrize("grid", [(2, 2), (4, 2), (2, 4), (3, 1)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_mesh2d_with_segments_equals_plain(kind, grid, causal):
+    """Mesh2D tiles with segment ids, merged per query chunk = the plain
+    function with the same ids; rows that see no key at all (padding) end
+    with O = 0 and LSE = -inf and get zero gradients."""
+    from oracle import mesh2d
+    gq, gk = grid
+    n = 24
+    b_ = 1 if kind == "packed" else 2
+    q, k, v, do = _rand(b_, n, 4, 4), _rand(b_, n, 2, 4), _rand(b_, n, 2, 4), _rand(b_, n, 4, 4)
+    seg = (attention.segments_from_boundaries([0, 5, 6, 17, 21], n) if kind == "packed"
+           else attention.segments_from_lengths([19, 7], n))
+    o_ref, l_ref = attention.attention_forward(q, k, v, causal=causal, seg=seg)
+    g_ref = attention.attention_backward(q, k, v, do, causal=causal, seg=seg)
+    o, l = mesh2d.mesh2d_forward(q, k, v, gq, gk, causal, seg=seg)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l, l_ref, rtol=1e-12)
+    g = mesh2d.mesh2d_backward(q, k, v, o, l, do, gq, gk, causal, seg=seg)
+    for a, b in zip(g, g_ref):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+    pad = np.asarray(seg).reshape(b_, n) < 0
+    assert np.all(np.isneginf(np.moveaxis(l, 1, 2)[pad]))
+    assert np.all(o[pad] == 0) and np.all(g[0][pad] == 0)
