@@ -82,6 +82,9 @@ struct Segs {
   int nseg;
   const int* lens;  // right padding lengths, or null
   int64_t N;
+  // batch entries per lens entry: a call whose batch entries are the
+  // lens_div head groups of each caller batch entry (USP) reads lens[b / lens_div]
+  int lens_div = 1;
   __device__ __forceinline__ void range(int b, int64_t t, int64_t& start, int64_t& end) const {
     if (cu) {
       if (t >= cu[nseg]) {
@@ -98,7 +101,7 @@ struct Segs {
       start = cu[lo];
       end = cu[hi];
     } else if (lens) {
-      const int64_t len = lens[b];
+      const int64_t len = lens[lens_div > 1 ? b / lens_div : b];
       if (t < len) {
         start = 0;
         end = len;

@@ -78,6 +78,7 @@ struct AttnArgs {
   const int* cu_seqlens; // packing boundaries (device) or null
   int num_segments;
   const int* seq_lens;   // right-padding lengths (device) or null
+  int seg_div;           // batch entries per seq_lens entry (>= 1; USP head groups)
   unsigned int* status;
 };
 __host__ __device__ inline int kv_shards(const AttnArgs& a) { return a.Pk > 0 ? a.Pk : a.P; }

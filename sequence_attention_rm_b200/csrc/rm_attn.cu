@@ -48,6 +48,18 @@ int current_device() {
 
 int esize_of(rm_dtype t) { return t == RM_BF16 ? 2 : 4; }
 
+// Inner batch entries per caller batch entry, for the segment arrays.  USP
+// runs its ring with every (batch entry, head group) as a batch entry of its
+// own, so u inner entries share one seq_lens entry, and a packed batch (which
+// the caller gives with B == 1) reaches the ring with B == u.  USP sets it for
+// the duration of its inner calls on the calling thread; 1 everywhere else.
+thread_local int t_seg_div = 1;
+struct SegDivScope {
+  int prev;
+  explicit SegDivScope(int u) : prev(t_seg_div) { t_seg_div = u; }
+  ~SegDivScope() { t_seg_div = prev; }
+};
+
 rm_status check_desc(const rm_attn_desc* d) {
   if (!d) return fail(RM_ERR_INVALID_ARG, "desc is NULL");
   if (d->dtype != RM_F32 && d->dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
@@ -68,10 +80,8 @@ rm_status check_desc(const rm_attn_desc* d) {
     return fail(RM_ERR_INVALID_ARG, "bad token order");
   if (d->cu_seqlens && d->seq_lens)
     return fail(RM_ERR_INVALID_ARG, "cu_seqlens and seq_lens are exclusive");
-  if (d->cu_seqlens && (d->num_segments < 1 || d->B != 1))
+  if (d->cu_seqlens && (d->num_segments < 1 || d->B != t_seg_div))
     return fail(RM_ERR_INVALID_ARG, "packing needs num_segments >= 1 and B == 1");
-  if ((d->cu_seqlens || d->seq_lens) && d->dtype != RM_BF16)
-    return fail(RM_ERR_UNSUPPORTED, "packed / right-padded batches need bf16 (tensor-core path)");
   if (!(d->scale == d->scale) || isinf(d->scale)) return fail(RM_ERR_INVALID_ARG, "bad scale");
   if (d->dtype == RM_BF16) {
     if (!tc_supported_head_dim(d->d))
@@ -374,6 +384,7 @@ static AttnArgs attn_args(const rm_attn_desc* desc, int64_t lse_ld) {
   a.cu_seqlens = desc->cu_seqlens;
   a.num_segments = desc->cu_seqlens ? desc->num_segments : 0;
   a.seq_lens = desc->seq_lens;
+  a.seg_div = t_seg_div;
   a.status = status_word();
   return a;
 }
@@ -586,8 +597,6 @@ namespace {
 rm_status usp_desc(const rm_attn_desc* desc, int u, rm_attn_desc* out) {
   RM_TRY(check_desc(desc));
   if (u < 1) return fail(RM_ERR_INVALID_ARG, "ulysses degree must be >= 1");
-  if (desc->cu_seqlens || desc->seq_lens)
-    return fail(RM_ERR_UNSUPPORTED, "USP with packed / right-padded batches is not supported");
   if (desc->Hq % u || desc->Hkv % u)
     return fail(RM_ERR_INVALID_ARG, "ulysses degree %d must divide Hq (%d) and Hkv (%d)", u,
                 desc->Hq, desc->Hkv);
@@ -614,7 +623,10 @@ rm_status usp_ws(const rm_attn_desc* desc, int u, int backward, UspWs* w) {
   // forward: q, o, k, v; backward: q, o, dout, dq and k, v, dk, dv
   w->ring_off = backward ? 4 * w->q + 4 * w->kv : 2 * w->q + 2 * w->kv;
   size_t rb = 0;
-  RM_TRY(rm_ring_workspace_size(&d2, backward, &rb));
+  {
+    SegDivScope scope(u);
+    RM_TRY(rm_ring_workspace_size(&d2, backward, &rb));
+  }
   w->ring_bytes = rb;
   w->total = w->ring_off + align_up(rb);
   return RM_OK;
@@ -679,10 +691,14 @@ rm_status rm_usp_attn_fwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
   RM_TRY(usp_repack(desc, u, desc->Hq, 0, q.ptr, yq, st));
   RM_TRY(usp_repack(desc, u, desc->Hkv, 0, k.ptr, yk, st));
   RM_TRY(usp_repack(desc, u, desc->Hkv, 0, v.ptr, yv, st));
-  // lse [B, Hq, N] is [B*u, Hq/u, N]: the ring writes it in place
-  RM_TRY(rm_ring_attn_fwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
-                          dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
-                          base + w.ring_off, w.ring_bytes, stream));
+  // lse [B, Hq, N] is [B*u, Hq/u, N]: the ring writes it in place.  Segment
+  // boundaries are global positions, which the head exchange keeps.
+  {
+    SegDivScope scope(u);
+    RM_TRY(rm_ring_attn_fwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
+                            dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
+                            base + w.ring_off, w.ring_bytes, stream));
+  }
   return usp_repack(desc, u, desc->Hq, 1, yo, o.ptr, st);
 }
 
@@ -716,11 +732,14 @@ rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
   RM_TRY(usp_repack(desc, u, hkv, 0, v.ptr, yv, st));
   RM_TRY(usp_repack(desc, u, hq, 0, o.ptr, yo, st));
   RM_TRY(usp_repack(desc, u, hq, 0, dout.ptr, ydo, st));
-  RM_TRY(rm_ring_attn_bwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
-                          dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
-                          dense_t(ydo, d2, d2.Hq), dense_t(ydq, d2, d2.Hq),
-                          dense_t(ydk, d2, d2.Hkv), dense_t(ydv, d2, d2.Hkv), base + w.ring_off,
-                          w.ring_bytes, stream));
+  {
+    SegDivScope scope(u);
+    RM_TRY(rm_ring_attn_bwd(&d2, dense_t(yq, d2, d2.Hq), dense_t(yk, d2, d2.Hkv),
+                            dense_t(yv, d2, d2.Hkv), dense_t(yo, d2, d2.Hq), lse,
+                            dense_t(ydo, d2, d2.Hq), dense_t(ydq, d2, d2.Hq),
+                            dense_t(ydk, d2, d2.Hkv), dense_t(ydv, d2, d2.Hkv), base + w.ring_off,
+                            w.ring_bytes, stream));
+  }
   RM_TRY(usp_repack(desc, u, hq, 1, ydq, dq.ptr, st));
   RM_TRY(usp_repack(desc, u, hkv, 1, ydk, dk.ptr, st));
   return usp_repack(desc, u, hkv, 1, ydv, dv.ptr, st);
@@ -745,8 +764,6 @@ rm_status mesh2d_desc(const rm_attn_desc* desc, int grid_q, int grid_k, rm_attn_
   out->order = RM_ORDER_RANK_MAJOR;
   RM_TRY(check_desc(out));
   if (desc->N % grid_k) return fail(RM_ERR_INVALID_ARG, "grid_k must divide N");
-  if (desc->cu_seqlens || desc->seq_lens)
-    return fail(RM_ERR_UNSUPPORTED, "Mesh2D with packed / right-padded batches is not supported");
   return RM_OK;
 }
 

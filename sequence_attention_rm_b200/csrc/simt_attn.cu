@@ -57,6 +57,26 @@ __device__ __forceinline__ void stage(float (*dst)[DMAX], const float* base, int
   }
 }
 
+// The CTA's range of local keys: the union [min lo, max hi) of the ranges its
+// rows contribute (`mine`: this thread contributes [lo, hi)); empty ranges
+// give [0, 0).  Every thread of the CTA must call it.
+__device__ __forceinline__ void cta_key_range(unsigned long long* shared, bool mine, int64_t lo,
+                                              int64_t hi, int64_t& cta_lo, int64_t& cta_hi) {
+  __syncthreads();  // the previous step's readers are done with `shared`
+  if (threadIdx.x == 0) {
+    shared[0] = ~0ull;
+    shared[1] = 0ull;
+  }
+  __syncthreads();
+  if (mine) {
+    atomicMin(&shared[0], (unsigned long long)lo);
+    atomicMax(&shared[1], (unsigned long long)hi);
+  }
+  __syncthreads();
+  cta_hi = (int64_t)shared[1];
+  cta_lo = cta_hi > 0 ? (int64_t)shared[0] : 0;
+}
+
 // ---------------------------------------------------------------------------
 template <int DMAX>
 __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_rank, int kv_rank) {
@@ -75,6 +95,12 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
   const bool live = j < L;
   const int64_t qrow = (ring ? (int64_t)r * L : 0) + j;
   const int64_t tq = live ? lay.pos(r, j) : 0;
+  // global positions [qf, ql] of the keys this row may see (causal rule and
+  // segment of a packed or right-padded batch)
+  const Segs sg{a.cu_seqlens, a.num_segments, a.seq_lens, a.N, a.seg_div > 1 ? a.seg_div : 1};
+  int64_t qf = 0, ql = -1;
+  if (live) sg.query_span(b, tq, a.causal, qf, ql);
+  __shared__ unsigned long long cta_range[2];
 
   Slice<DMAX> q, acc;
   const float* qp = reinterpret_cast<const float*>(a.q.ptr) + b * a.q.stride_b + qrow * a.q.stride_n +
@@ -87,20 +113,21 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
   for (int c = 0; c < DMAX / 4; ++c) acc.v[c] = 0.f;
   float m = -INFINITY, l = 0.f;
 
-  const int64_t j_last = min((int64_t)(blockIdx.x + 1) * kRows, L) - 1;
-  const int64_t t_last = lay.pos(r, j_last);
   const int nsteps = ring ? a.P : 1;
   for (int step = 0; step < nsteps; ++step) {
     const int s = ring ? ((r - step) % a.P + a.P) % a.P : kv_rank;
-    // keys of shard s this row (and this CTA) may see
-    const int64_t row_lim = !live ? 0 : (a.causal ? kmap.visible_count(s, tq) : kmap.L);
-    const int64_t cta_lim = a.causal ? kmap.visible_count(s, t_last) : kmap.L;
+    // local keys [row_lo, row_hi) of shard s this row may see (positions are
+    // increasing in the local index), and their union over the CTA's rows
+    const int64_t row_lo = live ? kmap.visible_count(s, qf - 1) : 0;
+    const int64_t row_hi = live ? kmap.visible_count(s, ql) : 0;
+    int64_t cta_lo, cta_hi;
+    cta_key_range(cta_range, sub == 0 && row_hi > row_lo, row_lo, row_hi, cta_lo, cta_hi);
     const int64_t kv0 = ring ? (int64_t)s * L : 0;
     const float* kb = reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
                       kv0 * a.k.stride_n;
     const float* vb = reinterpret_cast<const float*>(a.v.ptr) + b * a.v.stride_b + g * a.v.stride_h +
                       kv0 * a.v.stride_n;
-    for (int64_t i0 = 0; i0 < cta_lim; i0 += kTile) {
+    for (int64_t i0 = cta_lo; i0 < cta_hi; i0 += kTile) {
       __syncthreads();
       stage<DMAX>(ks, kb, a.k.stride_n, i0, kmap.L, a.d);
       stage<DMAX>(vs, vb, a.v.stride_n, i0, kmap.L, a.d);
@@ -113,7 +140,7 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
 #pragma unroll
         for (int c = 0; c < DMAX / 4; ++c) part = fmaf(q.v[c], ks[kk][col_of(c, sub)], part);
         float sv = row_sum4(part) * a.scale;
-        sc[kk] = (i0 + kk < row_lim) ? sv : -INFINITY;
+        sc[kk] = (i0 + kk >= row_lo && i0 + kk < row_hi) ? sv : -INFINITY;
         tmax = fmaxf(tmax, sc[kk]);
       }
       if (tmax == -INFINITY) continue;  // nothing visible in this tile for this row
@@ -164,6 +191,10 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
   const bool live = j < L;
   const int64_t qrow = (ring ? (int64_t)r * L : 0) + j;
   const int64_t tq = live ? lay.pos(r, j) : 0;
+  const Segs sg{a.cu_seqlens, a.num_segments, a.seq_lens, a.N, a.seg_div > 1 ? a.seg_div : 1};
+  int64_t qf = 0, ql = -1;
+  if (live) sg.query_span(b, tq, a.causal, qf, ql);
+  __shared__ unsigned long long cta_range[2];
 
   Slice<DMAX> q, dO, dq;
 #pragma unroll
@@ -177,19 +208,19 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
     lse = a.lse_in[((int64_t)b * a.Hq + h) * a.lse_ld + qrow];
     D = a.delta[((int64_t)b * a.Hq + h) * a.lse_ld + qrow];
   }
-  const int64_t j_last = min((int64_t)(blockIdx.x + 1) * kRows, L) - 1;
-  const int64_t t_last = lay.pos(r, j_last);
   const int nsteps = ring ? a.P : 1;
   for (int step = 0; step < nsteps; ++step) {
     const int s = ring ? ((r - step) % a.P + a.P) % a.P : kv_rank;
-    const int64_t row_lim = !live ? 0 : (a.causal ? kmap.visible_count(s, tq) : kmap.L);
-    const int64_t cta_lim = a.causal ? kmap.visible_count(s, t_last) : kmap.L;
+    const int64_t row_lo = live ? kmap.visible_count(s, qf - 1) : 0;
+    const int64_t row_hi = live ? kmap.visible_count(s, ql) : 0;
+    int64_t cta_lo, cta_hi;
+    cta_key_range(cta_range, sub == 0 && row_hi > row_lo, row_lo, row_hi, cta_lo, cta_hi);
     const int64_t kv0 = ring ? (int64_t)s * L : 0;
     const float* kb = reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
                       kv0 * a.k.stride_n;
     const float* vb = reinterpret_cast<const float*>(a.v.ptr) + b * a.v.stride_b + g * a.v.stride_h +
                       kv0 * a.v.stride_n;
-    for (int64_t i0 = 0; i0 < cta_lim; i0 += kTile) {
+    for (int64_t i0 = cta_lo; i0 < cta_hi; i0 += kTile) {
       __syncthreads();
       stage<DMAX>(ks, kb, a.k.stride_n, i0, kmap.L, a.d);
       stage<DMAX>(vs, vb, a.v.stride_n, i0, kmap.L, a.d);
@@ -204,7 +235,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
         }
         const float sv = row_sum4(ps) * a.scale;
         const float dp = row_sum4(pd);
-        if (i0 + kk < row_lim) {
+        if (i0 + kk >= row_lo && i0 + kk < row_hi) {
           const float p = expf(sv - lse);
           const float ds = p * (dp - D) * a.scale;
 #pragma unroll
@@ -244,6 +275,10 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int
   const int64_t tk = live ? kmap.pos(s, i) : 0;
   const int64_t i_first = (int64_t)blockIdx.x * kRows;
   const int64_t t_first = kmap.pos(s, i_first);
+  // global positions [kf, kl] of the queries that see this key
+  const Segs sg{a.cu_seqlens, a.num_segments, a.seq_lens, a.N, a.seg_div > 1 ? a.seg_div : 1};
+  int64_t kf = 0, kl = -1;
+  if (live) sg.key_span(b, tk, a.causal, kf, kl);
 
   Slice<DMAX> k, v, dk, dv;
 #pragma unroll
@@ -290,7 +325,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int
           }
           const float sv = row_sum4(ps) * a.scale;
           const float dp = row_sum4(pd);
-          const bool vis = live && tpos[qq] >= 0 && (!a.causal || tk <= tpos[qq]);
+          const bool vis = live && tpos[qq] >= kf && tpos[qq] <= kl;
           if (vis) {
             const float p = expf(sv - lses[qq]);
             const float dsv = p * (dp - ds_[qq]) * a.scale;

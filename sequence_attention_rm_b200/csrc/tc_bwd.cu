@@ -63,6 +63,7 @@ struct BwdParams {
   const int* cu_seqlens;  // packing boundaries (device) or null
   int num_segments;
   const int* seq_lens;    // right-padding lengths (device) or null
+  int seg_div;            // batch entries per seq_lens entry
   unsigned int* status;
   long long wait_limit;
 };
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   W.P = p.P;
   W.causal = p.causal;
   const int64_t i0 = (int64_t)xt * BK;  // first key (local index in shard s)
-  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N, p.seg_div};
   {  // queries that may see a key of the CTA (the bounds are monotone in the key)
     int64_t f, l;
     sg.key_span(b, kpos(W.s, i0), p.causal, W.span_first, l);
@@ -716,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = h / (p.Hq / p.Hkv);
   const int64_t last_row = LayoutMap::min64(row0 + BM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
-  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N, p.seg_div};
   // global span of the keys any row of the CTA may see (the bounds are
   // monotone in the row, so its first and last rows give them)
   int64_t span_first, span_last;
@@ -1025,6 +1026,7 @@ rm_status tc_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream
   p.cu_seqlens = a.cu_seqlens;
   p.num_segments = a.num_segments;
   p.seq_lens = a.seq_lens;
+  p.seg_div = a.seg_div > 1 ? a.seg_div : 1;
   const int view = operand_view(a, ring);
   p.status = a.status;
   p.wait_limit = tc_wait_limit();

@@ -84,6 +84,7 @@ struct FwdParams {
   const int* cu_seqlens;  // packing boundaries (device) or null
   int num_segments;
   const int* seq_lens;    // right-padding lengths (device) or null
+  int seg_div;            // batch entries per seq_lens entry
   void* o;
   int64_t o_sb, o_sn, o_sh;
   int o_f32;
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   const int64_t last_row = min((p.head_pairs ? rowA : rowB) + kBM - 1, L - 1);
   const int64_t t_last = lay.pos(r, last_row);
-  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N};
+  const Segs sg{p.cu_seqlens, p.num_segments, p.seq_lens, p.N, p.seg_div};
   // global span of the keys any row of the CTA may see (bounds are monotone
   // in the row, so its first and last rows give them)
   int64_t span_first, span_last;
@@ -703,6 +704,7 @@ static rm_status launch_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   p.cu_seqlens = a.cu_seqlens;
   p.num_segments = a.num_segments;
   p.seq_lens = a.seq_lens;
+  p.seg_div = a.seg_div > 1 ? a.seg_div : 1;
   p.o = a.o.ptr;
   p.o_sb = a.o.stride_b;
   p.o_sn = a.o.stride_n;

@@ -315,12 +315,13 @@ def usp_workspace_size(dsc: RmAttnDesc, ulysses: int, backward: bool) -> int:
 
 
 def usp_attn_fwd(q, k, v, *, P: int, ulysses: int, layout: str, causal: bool,
-                 scale: float | None = None, mode: str = "fused", order: str = "rank", out=None,
-                 lse=None, ws=None, stream=None):
+                 scale: float | None = None, mode: str = "fused", order: str = "rank",
+                 cu_seqlens=None, seq_lens=None, out=None, lse=None, ws=None, stream=None):
     """USP forward: Ulysses degree `ulysses` x ring degree P; dense q/k/v
     [B, N, H, d] in `order` for the P ring ranks -> (O, LSE [B, Hq, N])."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, mode, order,
+               cu_seqlens, seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
     wp, wn = _workspace(usp_workspace_size(dsc, ulysses, False), q.device, ws)
@@ -330,11 +331,12 @@ def usp_attn_fwd(q, k, v, *, P: int, ulysses: int, layout: str, causal: bool,
 
 
 def usp_attn_bwd(q, k, v, o, lse, dout, *, P: int, ulysses: int, layout: str, causal: bool,
-                 scale: float | None = None, order: str = "rank", dq=None, dk=None, dv=None,
-                 ws=None, stream=None):
+                 scale: float | None = None, order: str = "rank", cu_seqlens=None,
+                 seq_lens=None, dq=None, dk=None, dv=None, ws=None, stream=None):
     """USP backward -> (dq, dk, dv) in the input dtype and order."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale, order=order,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
@@ -353,11 +355,13 @@ def mesh2d_workspace_size(dsc: RmAttnDesc, grid_q: int, grid_k: int, backward: b
 
 
 def mesh2d_attn_fwd(q, k, v, *, grid_q: int, grid_k: int, causal: bool,
-                    scale: float | None = None, out=None, lse=None, ws=None, stream=None):
+                    scale: float | None = None, cu_seqlens=None, seq_lens=None, out=None,
+                    lse=None, ws=None, stream=None):
     """Mesh2D forward over a grid_q x grid_k grid of (query chunk, key chunk)
     tiles; q/k/v [B, N, H, d] in token order -> (O, LSE [B, Hq, N])."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
     wp, wn = _workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, False), q.device, ws)
@@ -367,10 +371,12 @@ def mesh2d_attn_fwd(q, k, v, *, grid_q: int, grid_k: int, causal: bool,
 
 
 def mesh2d_attn_bwd(q, k, v, o, lse, dout, *, grid_q: int, grid_k: int, causal: bool,
-                    scale: float | None = None, dq=None, dk=None, dv=None, ws=None, stream=None):
+                    scale: float | None = None, cu_seqlens=None, seq_lens=None, dq=None,
+                    dk=None, dv=None, ws=None, stream=None):
     """Mesh2D backward -> (dq, dk, dv) in the input dtype."""
     B, N, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, grid_q, "contiguous", causal, scale,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv

@@ -69,13 +69,23 @@ def _desc(rm, **kw):
     (dict(cu_seqlens=16, num_segments=2, seq_lens=16), 1),  # exclusive
     (dict(cu_seqlens=16, num_segments=2, B=2), 1),          # packing needs B == 1
     (dict(cu_seqlens=16, num_segments=0), 1),
-    (dict(seq_lens=16, dtype=0), 2),                        # fp32: no segments
 ])
 def test_desc_validation(rm, bad, status):
     n = ctypes.c_size_t(0)
     d = _desc(rm, **bad)
     assert rm.raw().rm_ring_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == status
     assert rm.raw().rm_last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(seq_lens=16, dtype=0), dict(cu_seqlens=16, num_segments=3, dtype=0),
+                                dict(seq_lens=16), dict(cu_seqlens=16, num_segments=3)])
+def test_desc_accepts_segments(rm, kw):
+    """Packed and right-padded batches in bf16 (tensor-core kernels) and fp32
+    (SIMT kernels)."""
+    n = ctypes.c_size_t(0)
+    d = _desc(rm, **kw)
+    for backward in (0, 1):
+        assert rm.raw().rm_ring_workspace_size(ctypes.byref(d), backward, ctypes.byref(n)) == 0
 
 
 def test_global_order_accepted(rm):
@@ -155,11 +165,21 @@ def test_usp_auto_select_hand_table(rm):
 
 @pytest.mark.parametrize("kw,u", [(dict(), 3), (dict(), 16), (dict(N=16386, P=2), 4),
                                   (dict(Hq=12, Hkv=6), 4),
-                                  (dict(seq_lens=16), 2)])  # no segments under USP
+                                  (dict(cu_seqlens=16, num_segments=2, B=2), 2)])  # packing: B == 1
 def test_usp_validation(rm, kw, u):
     n = ctypes.c_size_t(0)
     d = _desc(rm, **kw)
     assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), u, 0, ctypes.byref(n)) != 0
+
+
+@pytest.mark.parametrize("kw", [dict(seq_lens=16), dict(cu_seqlens=16, num_segments=3)])
+def test_usp_accepts_segments(rm, kw):
+    """Packed (B == 1) and right-padded batches under USP: the inner ring sees
+    B x u batch entries that share the caller's segment description."""
+    n = ctypes.c_size_t(0)
+    d = _desc(rm, **kw)
+    for backward in (0, 1):
+        assert rm.raw().rm_usp_workspace_size(ctypes.byref(d), 2, backward, ctypes.byref(n)) == 0
 
 
 def test_usp_workspace_sizes(rm):
@@ -179,8 +199,8 @@ def test_mesh2d_validation(rm, gq, gk, status):
     d = _desc(rm)  # N = 16384
     assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), gq, gk, 0, ctypes.byref(n)) == status
     assert rm.raw().rm_last_error()
-    d = _desc(rm, seq_lens=16)
-    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 2, 2, 0, ctypes.byref(n)) == 2
+    d = _desc(rm, seq_lens=16)  # right-padded (and packed) batches are accepted
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 2, 2, 0, ctypes.byref(n)) == 0
 
 
 def test_mesh2d_workspace_sizes(rm):

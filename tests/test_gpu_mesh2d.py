@@ -80,13 +80,15 @@ def test_mesh2d_strided_operands(rm):
     assert_max_abs(np64(l), l_ref, BF16_LSE_TOL, "LSE")
 
 
-def test_mesh2d_rejects_segments_and_bad_grids(rm):
+def test_mesh2d_rejects_bad_grids(rm):
     q = torch.zeros(1, 64, 2, 64, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(rm.RmError):
         rm.mesh2d_attn_fwd(q, q, q, grid_q=3, grid_k=1, causal=True)
     with pytest.raises(rm.RmError):
         rm.mesh2d_attn_fwd(q, q, q, grid_q=2, grid_k=32, causal=True)
-    lens = torch.tensor([10], dtype=torch.int32, device="cuda")
-    dsc = rm.desc(torch.bfloat16, 1, 2, 2, 64, 64, 2, "contiguous", True, seq_lens=lens)
+    # packed batches need B == 1, as for the ring
+    cu = torch.tensor([0, 10, 64], dtype=torch.int32, device="cuda")
+    dsc = rm.desc(torch.bfloat16, 1, 2, 2, 64, 64, 2, "contiguous", True, cu_seqlens=cu)
+    dsc.B = 2
     n = ctypes.c_size_t(0)
-    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(dsc), 2, 2, 0, ctypes.byref(n)) == 2
+    assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(dsc), 2, 2, 0, ctypes.byref(n)) == 1
