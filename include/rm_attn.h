@@ -105,8 +105,9 @@ typedef enum { RM_ORDER_RANK_MAJOR = 0, RM_ORDER_GLOBAL = 1 } rm_order;
 
 /* One attention problem: B sequences of N tokens split over P virtual ranks
  * (L = N / P tokens each) laid out by `layout`; N < 2^31 (token positions
- * are 32-bit on the device).  d is the true head dimension.  bf16 supports d in {24, 32, 64, 128} (24 is zero-padded to 32
- * on chip); fp32 supports d % 4 == 0, d <= 128. */
+ * are 32-bit on the device).  d is the true head dimension.  bf16 supports
+ * d in {24, 32, 64, 128} (24 is zero-padded to 32 on chip); fp32 supports
+ * d % 4 == 0, d <= 128. */
 typedef struct {
   rm_dtype dtype;
   int B;
@@ -131,10 +132,12 @@ typedef struct {
    *               from cu[num_segments] on are padding; needs B == 1;
    *   seq_lens:   device int32[B], valid tokens of each batch entry (right
    *               padding).
-   * NULL / 0: dense.  Supported on the bf16 tensor-core path (fwd: d in
-   * {24, 32, 64, 128}; bwd: d = 128); fp32 and the <= 16-token path return
-   * RM_ERR_UNSUPPORTED.  The values are read on the device: malformed
-   * boundaries give wrong results but no out-of-range access. */
+   * NULL / 0: dense.  Taken by every entry point with a descriptor (block,
+   * ring, USP, Mesh2D), bf16 and fp32; sequences of at most 16 tokens with
+   * segments run on the general kernels instead of the short-sequence ones.
+   * USP applies the caller's description to every head group (packing still
+   * needs the caller's B == 1).  The values are read on the device:
+   * malformed boundaries give wrong results but no out-of-range access. */
   const int32_t* cu_seqlens;
   int num_segments;
   const int32_t* seq_lens;
@@ -303,8 +306,9 @@ rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
  * without a visible pair under the causal rule are skipped.
  *
  * desc: dtype, B, Hq, Hkv, d, N, causal, scale as for the ring; P, layout,
- * mode and order are ignored (operands in global token order); no segments
- * (RM_ERR_UNSUPPORTED).  grid_q, grid_k >= 1 must divide N; grid_k <= 16
+ * mode and order are ignored (operands in global token order); segments
+ * (cu_seqlens / seq_lens) apply by global position.  grid_q, grid_k >= 1
+ * must divide N; grid_k <= 16
  * (RM_ERR_UNSUPPORTED above).  The bf16 backward needs d = 128.
  * q/o/dout/dq [B, N, Hq, d], k/v/dk/dv [B, N, Hkv, d] strided as rm_tensor;
  * lse fp32 [B, Hq, N].  Workspace (caller-owned, 256-byte aligned):
