@@ -218,9 +218,12 @@ rm_status rm_ring_attn_fwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
 
 /* Ring backward: delta from the final (o, dout), then every (query shard,
  * KV shard) pair's contribution accumulated in fp32, KV shards visiting the
- * ranks in reverse ring order; dq/dk/dv written in desc->dtype, rank-major.
- * o, lse: the outputs of rm_ring_attn_fwd.  ws: rm_ring_workspace_size(desc, 1)
- * bytes, 256-byte aligned. */
+ * ranks in reverse ring order; dq/dk/dv written in desc->dtype, in
+ * desc->order.  o, lse: the outputs of rm_ring_attn_fwd.
+ * ws: rm_ring_workspace_size(desc, 1) bytes, 256-byte aligned (delta; for
+ * bf16 at head dims other than 128, which run on the CUDA-core kernels, also
+ * fp32 dq/dk/dv that are then rounded to bf16).  Global token order in the
+ * backward needs d = 128 (RM_ERR_UNSUPPORTED otherwise). */
 rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k,
                            rm_tensor v, rm_tensor o, const float* lse,
                            rm_tensor dout, rm_tensor dq, rm_tensor dk,
@@ -309,7 +312,7 @@ rm_status rm_usp_attn_bwd(const rm_attn_desc* desc, int ulysses, rm_tensor q, rm
  * mode and order are ignored (operands in global token order); segments
  * (cu_seqlens / seq_lens) apply by global position.  grid_q, grid_k >= 1
  * must divide N; grid_k <= 16
- * (RM_ERR_UNSUPPORTED above).  The bf16 backward needs d = 128.
+ * (RM_ERR_UNSUPPORTED above).
  * q/o/dout/dq [B, N, Hq, d], k/v/dk/dv [B, N, Hkv, d] strided as rm_tensor;
  * lse fp32 [B, Hq, N].  Workspace (caller-owned, 256-byte aligned):
  * forward grid_k fp32 partial O [B, N, Hq, d] and LSE [B, Hq, N] slots;

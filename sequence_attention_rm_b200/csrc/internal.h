@@ -86,8 +86,10 @@ __host__ __device__ inline int kv_shards(const AttnArgs& a) { return a.Pk > 0 ? 
 // Forward.  q_rank < 0: all ranks (ring, rank-major operands, fused merge);
 // else one (q_rank, kv_rank) pair with shard-local operands.
 cudaError_t launch_simt_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
-// Backward, same rank convention; accumulates dq (+=) and dk/dv (+=).
-cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream);
+// Backward, same rank convention; dq / dk / dv are fp32 (+= when
+// a.accumulate); operands fp32, or bf16 (in_bf16) widened as they are read.
+cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, int in_bf16,
+                            cudaStream_t stream);
 
 // Short sequences (L <= 16, d <= 64): one warp per (sequence, head), any dtype.
 bool small_seq_supported(int64_t L, int d);

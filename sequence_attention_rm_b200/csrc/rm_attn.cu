@@ -99,6 +99,9 @@ rm_status check_order(const rm_attn_desc* d, int backward) {
   if (d->order != RM_ORDER_GLOBAL || d->layout == RM_LAYOUT_CONTIGUOUS || d->P == 1) return RM_OK;
   if (d->dtype != RM_BF16)
     return fail(RM_ERR_UNSUPPORTED, "global token order needs bf16 (the tensor-core path)");
+  if (backward && d->d != 128)
+    return fail(RM_ERR_UNSUPPORTED,
+                "global token order in the backward needs head dim 128 (the tensor-core path)");
   if (!backward && d->mode != RM_RING_FUSED)
     return fail(RM_ERR_UNSUPPORTED, "global token order needs the fused ring mode");
   if (d->layout == RM_LAYOUT_ZIGZAG && (d->N / (2 * (int64_t)d->P)) % 128)
@@ -156,15 +159,27 @@ FwdWs fwd_ws(const rm_attn_desc* d) {
   w.total = w.lse_parts + align_up(rows * 4 * (size_t)d->P);
   return w;
 }
+// The bf16 backward at head dims other than 128 runs on the SIMT kernels
+// (bf16 operands read as fp32) into fp32 dQ / dK / dV, then rounds them.
+bool bf16_simt_bwd(const rm_attn_desc* d) { return d->dtype == RM_BF16 && d->d != 128; }
+
 struct BwdWs {
-  size_t delta, total;
+  size_t delta, dq, dk, dv, total;  // dq / dk / dv: fp32 [B, N, H, d], bf16 SIMT backward only
 };
 BwdWs bwd_ws(const rm_attn_desc* d) {
   BwdWs w;
-  const size_t rows_q = (size_t)d->B * d->N * d->Hq;
+  memset(&w, 0, sizeof(w));
+  const size_t rows_q = (size_t)d->B * d->N * d->Hq, rows_kv = (size_t)d->B * d->N * d->Hkv;
   w.delta = 0;
-  // both backward paths write dQ / dK / dV themselves: delta is all they keep
+  // the tensor-core and fp32 backward paths write dQ / dK / dV themselves:
+  // delta is all they keep
   w.total = align_up(rows_q * 4);
+  if (bf16_simt_bwd(d)) {
+    w.dq = w.total;
+    w.dk = w.dq + align_up(rows_q * d->d * 4);
+    w.dv = w.dk + align_up(rows_kv * d->d * 4);
+    w.total = w.dv + align_up(rows_kv * d->d * 4);
+  }
   return w;
 }
 
@@ -446,12 +461,10 @@ rm_status rm_attn_block_bwd(const rm_attn_desc* desc, int q_rank, int kv_rank, r
   a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse_in = lse_final; a.delta = delta;
   a.dq = dq_acc; a.dk = dk_acc; a.dv = dv_acc;
   a.accumulate = 1;
-  if (desc->dtype == RM_F32) {
-    RM_CUDA(launch_simt_bwd(a, q_rank, kv_rank, st), "simt bwd launch");
+  if (desc->dtype == RM_F32 || bf16_simt_bwd(desc)) {
+    RM_CUDA(launch_simt_bwd(a, q_rank, kv_rank, desc->dtype == RM_BF16, st), "simt bwd launch");
     return RM_OK;
   }
-  if (desc->d != 128)
-    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", desc->d);
   return tc_bwd(a, q_rank, kv_rank, st);
 }
 
@@ -548,8 +561,6 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
   RM_TRY(check_tensor("dk", dk, es, rows, desc->Hkv, desc->d));
   RM_TRY(check_tensor("dv", dv, es, rows, desc->Hkv, desc->d));
   if (!lse) return fail(RM_ERR_INVALID_ARG, "lse NULL");
-  if (desc->dtype == RM_BF16 && desc->d != 128)
-    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", desc->d);
   const BwdWs w = bwd_ws(desc);
   if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
     return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
@@ -564,7 +575,25 @@ rm_status rm_ring_attn_bwd(const rm_attn_desc* desc, rm_tensor q, rm_tensor k, r
                                   st),
             "bwd preprocess launch");
     a.dq = dq; a.dk = dk; a.dv = dv;
-    RM_CUDA(launch_simt_bwd(a, -1, -1, st), "simt ring bwd launch");
+    RM_CUDA(launch_simt_bwd(a, -1, -1, 0, st), "simt ring bwd launch");
+    return RM_OK;
+  }
+  if (bf16_simt_bwd(desc)) {
+    // SIMT kernels on the bf16 operands into fp32 dQ / dK / dV, rounded (RNE)
+    // into the caller's tensors
+    RM_CUDA(launch_bwd_preprocess(1, desc->B, desc->N, desc->Hq, desc->d, o, dout, delta, nullptr,
+                                  st),
+            "bwd preprocess launch");
+    char* base = (char*)ws;
+    a.dq = dense_bnhd(base + w.dq, desc->N, desc->Hq, desc->d);
+    a.dk = dense_bnhd(base + w.dk, desc->N, desc->Hkv, desc->d);
+    a.dv = dense_bnhd(base + w.dv, desc->N, desc->Hkv, desc->d);
+    RM_CUDA(launch_simt_bwd(a, -1, -1, 1, st), "simt ring bwd launch");
+    RM_CUDA(launch_convert_f32(1, desc->B, desc->N, desc->Hq, desc->d, a.dq, dq, st), "dQ convert");
+    RM_CUDA(launch_convert_f32(1, desc->B, desc->N, desc->Hkv, desc->d, a.dk, dk, st),
+            "dK convert");
+    RM_CUDA(launch_convert_f32(1, desc->B, desc->N, desc->Hkv, desc->d, a.dv, dv, st),
+            "dV convert");
     return RM_OK;
   }
   // delta from the final O, then the dK/dV and dQ kernels write their outputs
@@ -876,8 +905,6 @@ rm_status rm_mesh2d_attn_bwd(const rm_attn_desc* desc, int grid_q, int grid_k, r
   RM_TRY(check_tensor("dk", dk, es, rows, d2.Hkv, d2.d));
   RM_TRY(check_tensor("dv", dv, es, rows, d2.Hkv, d2.d));
   if (!lse) return fail(RM_ERR_INVALID_ARG, "lse NULL");
-  if (d2.dtype == RM_BF16 && d2.d != 128)
-    return fail(RM_ERR_UNSUPPORTED, "the bf16 backward supports head dim 128 (got %d)", d2.d);
   const MeshWs w = mesh2d_ws(&d2, grid_k, 1);
   if (!ws || ws_bytes < w.total || ((uintptr_t)ws & 255))
     return fail(RM_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", w.total);
@@ -909,8 +936,8 @@ rm_status rm_mesh2d_attn_bwd(const rm_attn_desc* desc, int grid_q, int grid_k, r
       a.dk = offset_rows(dk_acc, j * Lk, 4);
       a.dv = offset_rows(dv_acc, j * Lk, 4);
       a.accumulate = 1;
-      if (d2.dtype == RM_F32) {
-        RM_CUDA(launch_simt_bwd(a, i, j, st), "simt Mesh2D tile bwd launch");
+      if (d2.dtype == RM_F32 || bf16_simt_bwd(&d2)) {
+        RM_CUDA(launch_simt_bwd(a, i, j, d2.dtype == RM_BF16, st), "simt Mesh2D tile bwd launch");
       } else {
         RM_TRY(tc_bwd(a, i, j, st));
       }

@@ -2,7 +2,9 @@
 // bf16).  TF32 tensor cores could not hold 1e-5 parity, so fp32 problems are
 // computed with fp32 FMA: each query (or key) row is owned by 4 lanes, each
 // holding d/4 of its columns; K/V (or Q/dO) tiles of 32 rows are staged in
-// shared memory and read as broadcasts.
+// shared memory and read as broadcasts.  The backward kernels also take bf16
+// operands (widened to fp32 as they are read): the bf16 backward at head dims
+// other than 128, which the tensor-core backward does not cover.
 //
 // Forward: online softmax over the KV tiles of every KV shard the row sees
 // (Ring Attention & Friends, "Tiling with the Softmax Rescaling Trick"), the
@@ -30,12 +32,15 @@ struct Slice {
 // column of slot c for lane `sub` of the row's 4 lanes
 __device__ __forceinline__ int col_of(int c, int sub) { return c * 4 + sub; }
 
-template <int DMAX>
-__device__ __forceinline__ void load_slice(Slice<DMAX>& s, const float* row, int d, int sub) {
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <int DMAX, typename InT>
+__device__ __forceinline__ void load_slice(Slice<DMAX>& s, const InT* row, int d, int sub) {
 #pragma unroll
   for (int c = 0; c < DMAX / 4; ++c) {
     int col = col_of(c, sub);
-    s.v[c] = col < d ? row[col] : 0.f;
+    s.v[c] = col < d ? to_f32(row[col]) : 0.f;
   }
 }
 
@@ -47,13 +52,13 @@ __device__ __forceinline__ float row_sum4(float x) {
 
 // Stage rows [row0, row0 + kTile) of a [rows, d] operand (row stride `ld`
 // elements from `base`) into smem [kTile][DMAX]; rows >= nrows are zeroed.
-template <int DMAX>
-__device__ __forceinline__ void stage(float (*dst)[DMAX], const float* base, int64_t ld,
+template <int DMAX, typename InT>
+__device__ __forceinline__ void stage(float (*dst)[DMAX], const InT* base, int64_t ld,
                                       int64_t row0, int64_t nrows, int d) {
   for (int i = threadIdx.x; i < kTile * DMAX; i += blockDim.x) {
     int rr = i / DMAX, col = i % DMAX;
     int64_t row = row0 + rr;
-    dst[rr][col] = (row < nrows && col < d) ? base[row * ld + col] : 0.f;
+    dst[rr][col] = (row < nrows && col < d) ? to_f32(base[row * ld + col]) : 0.f;
   }
 }
 
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(AttnArgs a, int q_ra
 
 // ---------------------------------------------------------------------------
 // dQ pass: one CTA owns 32 query rows of (b, h, rank r).
-template <int DMAX>
+template <int DMAX, typename InT>
 __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q_rank, int kv_rank) {
   __shared__ float ks[kTile][DMAX];
   __shared__ float vs[kTile][DMAX];
@@ -201,9 +206,9 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
   for (int c = 0; c < DMAX / 4; ++c) { q.v[c] = 0.f; dO.v[c] = 0.f; dq.v[c] = 0.f; }
   float lse = 0.f, D = 0.f;
   if (live) {
-    load_slice<DMAX>(q, reinterpret_cast<const float*>(a.q.ptr) + b * a.q.stride_b +
+    load_slice<DMAX>(q, reinterpret_cast<const InT*>(a.q.ptr) + b * a.q.stride_b +
                             qrow * a.q.stride_n + h * a.q.stride_h, a.d, sub);
-    load_slice<DMAX>(dO, reinterpret_cast<const float*>(a.dout.ptr) + b * a.dout.stride_b +
+    load_slice<DMAX>(dO, reinterpret_cast<const InT*>(a.dout.ptr) + b * a.dout.stride_b +
                              qrow * a.dout.stride_n + h * a.dout.stride_h, a.d, sub);
     lse = a.lse_in[((int64_t)b * a.Hq + h) * a.lse_ld + qrow];
     D = a.delta[((int64_t)b * a.Hq + h) * a.lse_ld + qrow];
@@ -216,9 +221,9 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
     int64_t cta_lo, cta_hi;
     cta_key_range(cta_range, sub == 0 && row_hi > row_lo, row_lo, row_hi, cta_lo, cta_hi);
     const int64_t kv0 = ring ? (int64_t)s * L : 0;
-    const float* kb = reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
+    const InT* kb = reinterpret_cast<const InT*>(a.k.ptr) + b * a.k.stride_b + g * a.k.stride_h +
                       kv0 * a.k.stride_n;
-    const float* vb = reinterpret_cast<const float*>(a.v.ptr) + b * a.v.stride_b + g * a.v.stride_h +
+    const InT* vb = reinterpret_cast<const InT*>(a.v.ptr) + b * a.v.stride_b + g * a.v.stride_h +
                       kv0 * a.v.stride_n;
     for (int64_t i0 = cta_lo; i0 < cta_hi; i0 += kTile) {
       __syncthreads();
@@ -254,7 +259,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq_kernel(AttnArgs a, int q
 
 // dK/dV pass: one CTA owns 32 key rows of (b, kv head g, shard s); it walks
 // the query heads of the group and the query ranks that use the shard.
-template <int DMAX>
+template <int DMAX, typename InT>
 __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int q_rank, int kv_rank) {
   __shared__ float qs[kTile][DMAX];
   __shared__ float dos[kTile][DMAX];
@@ -284,9 +289,9 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int
 #pragma unroll
   for (int c = 0; c < DMAX / 4; ++c) { k.v[c] = 0.f; v.v[c] = 0.f; dk.v[c] = 0.f; dv.v[c] = 0.f; }
   if (live) {
-    load_slice<DMAX>(k, reinterpret_cast<const float*>(a.k.ptr) + b * a.k.stride_b +
+    load_slice<DMAX>(k, reinterpret_cast<const InT*>(a.k.ptr) + b * a.k.stride_b +
                             krow * a.k.stride_n + g * a.k.stride_h, a.d, sub);
-    load_slice<DMAX>(v, reinterpret_cast<const float*>(a.v.ptr) + b * a.v.stride_b +
+    load_slice<DMAX>(v, reinterpret_cast<const InT*>(a.v.ptr) + b * a.v.stride_b +
                             krow * a.v.stride_n + g * a.v.stride_h, a.d, sub);
   }
   const int nranks = ring ? a.P : 1;
@@ -296,9 +301,9 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv_kernel(AttnArgs a, int
       // reverse ring: shard s visits ranks s, s+1, ...
       const int r = ring ? (s + step) % a.P : q_rank;
       const int64_t q0 = ring ? (int64_t)r * L : 0;
-      const float* qb = reinterpret_cast<const float*>(a.q.ptr) + b * a.q.stride_b + h * a.q.stride_h +
+      const InT* qb = reinterpret_cast<const InT*>(a.q.ptr) + b * a.q.stride_b + h * a.q.stride_h +
                         q0 * a.q.stride_n;
-      const float* dob = reinterpret_cast<const float*>(a.dout.ptr) + b * a.dout.stride_b +
+      const InT* dob = reinterpret_cast<const InT*>(a.dout.ptr) + b * a.dout.stride_b +
                          h * a.dout.stride_h + q0 * a.dout.stride_n;
       const float* lse_b = a.lse_in + ((int64_t)b * a.Hq + h) * a.lse_ld + q0;
       const float* del_b = a.delta + ((int64_t)b * a.Hq + h) * a.lse_ld + q0;
@@ -368,24 +373,34 @@ cudaError_t launch_simt_fwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStre
   return cudaGetLastError();
 }
 
-cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream) {
+namespace {
+template <typename InT>
+cudaError_t launch_simt_bwd_t(const AttnArgs& a, int q_rank, int kv_rank, cudaStream_t stream) {
   const int64_t L = a.N / a.P;
-  if (L == 0 || a.B == 0 || a.Hq == 0) return cudaSuccess;
   const unsigned z = (unsigned)(q_rank < 0 ? a.B * a.P : a.B);
   dim3 gq((unsigned)ceil_div(L, kRows), (unsigned)a.Hq, z);
   dim3 gk((unsigned)ceil_div(q_rank < 0 ? L : a.N / kv_shards(a), kRows), (unsigned)a.Hkv, z);
-  ProfScope ps("simt_bwd", stream);
   if (a.d <= 32) {
-    simt_bwd_dq_kernel<32><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
-    simt_bwd_dkdv_kernel<32><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dq_kernel<32, InT><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dkdv_kernel<32, InT><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
   } else if (a.d <= 64) {
-    simt_bwd_dq_kernel<64><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
-    simt_bwd_dkdv_kernel<64><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dq_kernel<64, InT><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dkdv_kernel<64, InT><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
   } else {
-    simt_bwd_dq_kernel<128><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
-    simt_bwd_dkdv_kernel<128><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dq_kernel<128, InT><<<gq, kThreads, 0, stream>>>(a, q_rank, kv_rank);
+    simt_bwd_dkdv_kernel<128, InT><<<gk, kThreads, 0, stream>>>(a, q_rank, kv_rank);
   }
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_simt_bwd(const AttnArgs& a, int q_rank, int kv_rank, int in_bf16,
+                            cudaStream_t stream) {
+  const int64_t L = a.N / a.P;
+  if (L == 0 || a.B == 0 || a.Hq == 0) return cudaSuccess;
+  ProfScope ps("simt_bwd", stream);
+  return in_bf16 ? launch_simt_bwd_t<__nv_bfloat16>(a, q_rank, kv_rank, stream)
+                 : launch_simt_bwd_t<float>(a, q_rank, kv_rank, stream);
 }
 
 }  // namespace rm

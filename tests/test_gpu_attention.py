@@ -193,13 +193,55 @@ def test_block_backward_bf16_every_pair(rm):
         assert_grad_close(np64(g), ref, what=name)
 
 
-def test_bf16_backward_other_head_dims_are_rejected(rm):
-    q, k, v, do = _inputs(torch.bfloat16, 1, 2, 2, 256, 64, 5)
-    qg, kg, vg, dog = q.cuda(), k.cuda(), v.cuda(), do.cuda()
-    o, l = rm.ring_attn_fwd(qg, kg, vg, P=2, layout="contiguous", causal=True)
-    with pytest.raises(rm.RmError) as e:
-        rm.ring_attn_bwd(qg, kg, vg, o, l, dog, P=2, layout="contiguous", causal=True)
-    assert e.value.status == rm.RM_ERR_UNSUPPORTED
+@pytest.mark.parametrize("d", [64, 32, 24])
+@pytest.mark.parametrize("layout,P", [("zigzag", 2), ("striped", 4), ("contiguous", 2)])
+def test_bf16_backward_other_head_dims(rm, d, layout, P):
+    """bf16 at head dims other than 128: the backward runs on the SIMT kernels
+    (bf16 operands read as fp32, fp32 sums, RNE outputs) and matches the
+    oracle like the tensor-core backward does."""
+    N = 384
+    q, k, v, do = _inputs(torch.bfloat16, 2, 4, 2, N, d, 5 + d)
+    o_ref, l_ref = oatt.attention_forward(np64(q), np64(k), np64(v), causal=True)
+    g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=True)
+    perm = lambda x: rm.layout_permute(x.cuda(), layout, P)
+    unperm = lambda x: rm.layout_permute(x, layout, P, inverse=True)
+    qr, kr, vr, dor = perm(q), perm(k), perm(v), perm(do)
+    o, l = rm.ring_attn_fwd(qr, kr, vr, P=P, layout=layout, causal=True)
+    assert_max_abs(np64(unperm(o)), o_ref, BF16_O_TOL, "O")
+    grads = rm.ring_attn_bwd(qr, kr, vr, o, l, dor, P=P, layout=layout, causal=True)
+    for name, g, ref in zip(("dq", "dk", "dv"), grads, g_ref):
+        assert g.dtype == torch.bfloat16
+        assert_grad_close(np64(unperm(g)), ref, what=name)
+    # global token order in the backward needs the tensor-core path (d = 128)
+    if layout != "contiguous":
+        with pytest.raises(rm.RmError) as e:
+            rm.ring_attn_bwd(q.cuda(), k.cuda(), v.cuda(), o, l, do.cuda(), P=P, layout=layout,
+                             causal=True, order="global")
+        assert e.value.status == rm.RM_ERR_UNSUPPORTED
+
+
+def test_bf16_block_backward_head_dim_64(rm):
+    """The block API at d = 64 accumulates one shard pair's gradients in fp32."""
+    N, P, d = 256, 2, 64
+    q, k, v, do = _inputs(torch.bfloat16, 1, 4, 2, N, d, 17)
+    L = N // P
+    f64 = lambda t: np64(t)
+    qs, ks, vs, dos = q[:, L:], k[:, :L], v[:, :L], do[:, L:]
+    o_ref, l_ref = oatt.attention_forward(f64(q), f64(k), f64(v), causal=True)
+    delta = oatt.delta_from_output(f64(do), o_ref)
+    ref = oatt.attention_backward_block(f64(qs), f64(ks), f64(vs), f64(dos), l_ref[:, :, L:],
+                                        delta[:, :, L:], causal=True,
+                                        q_pos=np.arange(L, N), k_pos=np.arange(0, L))
+    dq = torch.zeros(1, L, 4, d, device="cuda")
+    dk = torch.zeros(1, L, 2, d, device="cuda")
+    dv = torch.zeros(1, L, 2, d, device="cuda")
+    lse = torch.from_numpy(np.ascontiguousarray(l_ref[:, :, L:])).float().cuda()
+    dlt = torch.from_numpy(np.ascontiguousarray(delta[:, :, L:])).float().cuda()
+    rm.attn_block_bwd(qs.cuda().contiguous(), ks.cuda().contiguous(), vs.cuda().contiguous(),
+                      dos.cuda().contiguous(), lse, dlt, dq, dk, dv, N=N, P=P,
+                      layout="contiguous", causal=True, q_rank=1, kv_rank=0)
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        assert_grad_close(np64(g), r, what=name)
 
 
 def _global_ok(case):

@@ -38,7 +38,7 @@ CASES = [
     (torch.bfloat16, 1, 4, 4, 768, 128, 4, 2, False),
     (torch.bfloat16, 1, 4, 2, 600, 128, 2, 3, True),     # ragged chunks 300 / 200
     (torch.bfloat16, 1, 4, 2, 1200, 128, 3, 8, True),    # chunks 400 / 150
-    (torch.bfloat16, 1, 8, 2, 640, 64, 5, 2, True),      # forward only (d = 64)
+    (torch.bfloat16, 1, 8, 2, 640, 64, 5, 2, True),      # d = 64: backward on the SIMT kernels
     (torch.float32, 1, 4, 2, 384, 64, 2, 3, True),
     (torch.float32, 2, 2, 2, 96, 32, 3, 4, False),
 ]
@@ -54,8 +54,6 @@ def test_mesh2d_matches_oracle(rm, case):
     tol_o, tol_l = (F32_TOL, F32_TOL) if dtype == torch.float32 else (BF16_O_TOL, BF16_LSE_TOL)
     assert_max_abs(np64(o), o_ref, tol_o, "O")
     assert_max_abs(np64(l), l_ref, tol_l, "LSE")
-    if dtype == torch.bfloat16 and d != 128:
-        return
     g_ref = omesh.mesh2d_backward(np64(q), np64(k), np64(v), o_ref, l_ref, np64(do), gq, gk,
                                   causal)
     grads = rm.mesh2d_attn_bwd(qg, kg, vg, o, l, dog, grid_q=gq, grid_k=gk, causal=causal)
