@@ -280,9 +280,10 @@ def fused_kv(k, v):
 # key) pair: the contractions the kernel performs for its outputs.
 FLOPS_PER_PAIR = {"tc_fwd_kernel": 4, "tc_bwd_dkdv_kernel": 8, "tc_bwd_dq_kernel": 6}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of each kernel on
-# the headline workload, from the committed ncu capture of the current
-# kernels (profiles/); None until captured.
-TRAFFIC = {}
+# the headline workload (one-pass ncu capture of the current kernels at full
+# size, profiles/launch_list_long_zigzag_256k.md).
+TRAFFIC = {"tc_fwd_kernel": 8_362_033_920, "tc_bwd_dkdv_kernel": 18_578_496_512,
+           "tc_bwd_dq_kernel": 15_350_899_456}
 
 
 def kernel_table(records, steps, step_ms, w):
