@@ -180,6 +180,15 @@ rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
                                  rm_tensor o, rm_tensor dout, float* delta,
                                  void* stream);
 
+/* fp32 [B, N, H, d] -> out_dtype [B, N, H, d] (bf16: round to nearest even;
+ * fp32: a copy), both strided as rm_tensor (d contiguous): the last step of a
+ * backward that accumulated its gradients in fp32 (the block API's
+ * accumulators; the distributed ring, whose dK / dV accumulators travel
+ * between ranks in fp32).  d % 4 == 0, pointers and strides aligned to 4
+ * elements; in and out must not overlap. */
+rm_status rm_convert_f32(rm_dtype out_dtype, int B, int64_t N, int H, int d, rm_tensor in,
+                         rm_tensor out, void* stream);
+
 /* ---- LSE merge ---------------------------------------------------------- */
 
 /* Merge n_parts partial results [ringmaster, "Layout": ring/merge.py, the

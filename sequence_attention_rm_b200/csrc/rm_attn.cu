@@ -313,6 +313,19 @@ rm_status rm_seq_head_repack(rm_dtype dtype, int P, int64_t N_local, int H, int 
   return RM_OK;
 }
 
+rm_status rm_convert_f32(rm_dtype out_dtype, int B, int64_t N, int H, int d, rm_tensor in,
+                         rm_tensor out, void* stream) {
+  if (out_dtype != RM_F32 && out_dtype != RM_BF16) return fail(RM_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || N < 0 || H < 1 || d < 4 || d % 4) return fail(RM_ERR_INVALID_ARG, "bad sizes");
+  const int64_t rows = (int64_t)B * N;
+  if (rows == 0) return RM_OK;
+  RM_TRY(check_tensor("in", in, 4, rows, H, d, 16));
+  RM_TRY(check_tensor("out", out, esize_of(out_dtype), rows, H, d, out_dtype == RM_BF16 ? 8 : 16));
+  RM_CUDA(launch_convert_f32(out_dtype == RM_BF16, B, N, H, d, in, out, (cudaStream_t)stream),
+          "convert launch");
+  return RM_OK;
+}
+
 rm_status rm_lse_merge(rm_dtype out_dtype, int B, int H, int64_t Nq, int d, int n_parts,
                        const rm_tensor* o_parts, const float* const* lse_parts, rm_tensor o_out,
                        float* lse_out, void* stream) {

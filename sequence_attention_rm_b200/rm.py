@@ -32,6 +32,7 @@ EXPORTED = (
     "rm_debug_expire_wait", "rm_debug_exp2_poly", "rm_ring_attn_bwd_noalloc", "rm_profile_enable", "rm_profile_count",
     "rm_profile_get", "rm_usp_auto_select", "rm_usp_workspace_size", "rm_usp_attn_fwd",
     "rm_usp_attn_bwd", "rm_mesh2d_workspace_size", "rm_mesh2d_attn_fwd", "rm_mesh2d_attn_bwd",
+    "rm_convert_f32",
 )
 
 
@@ -66,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "rm_attn_block_fwd": [D, i, i, T, T, T, T, i, vp, vp],
         "rm_attn_block_bwd": [D, i, i, T, T, T, T, vp, vp, T, T, T, vp],
         "rm_attn_bwd_preprocess": [i, i, i64, i, i, T, T, vp, vp],
+        "rm_convert_f32": [i, i, i64, i, i, T, T, vp],
         "rm_lse_merge": [i, i, i, i64, i, i, ctypes.POINTER(RmTensor), ctypes.POINTER(vp), T, vp, vp],
         "rm_ring_workspace_size": [D, i, ctypes.POINTER(sz)],
         "rm_ring_attn_fwd": [D, T, T, T, T, vp, vp, sz, vp],
@@ -226,6 +228,18 @@ def attn_block_bwd(q, k, v, dout, lse_final, delta, dq_acc, dk_acc, dv_acc, *, N
     _check(_lib.rm_attn_block_bwd(ctypes.byref(dsc), q_rank, kv_rank, _bnhd(q), _bnhd(k), _bnhd(v),
                                   _bnhd(dout), _ptr(lse_final), _ptr(delta), _bnhd(dq_acc),
                                   _bnhd(dk_acc), _bnhd(dv_acc), _stream(stream)))
+
+
+def convert_f32(x: torch.Tensor, dtype: torch.dtype, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """fp32 [B, N, H, d] -> dtype (bf16: round to nearest even)."""
+    if x.dtype != torch.float32:
+        raise TypeError("convert_f32 takes an fp32 tensor")
+    B, N, H, d = x.shape
+    out = torch.empty(x.shape, dtype=dtype, device=x.device) if out is None else out
+    _check(_lib.rm_convert_f32(_dtype_code(dtype), B, N, H, d, _bnhd(x), _bnhd(out),
+                               _stream(stream)))
+    return out
 
 
 def attn_bwd_preprocess(o, dout, delta=None, stream=None):
