@@ -55,9 +55,10 @@ class KernelBlocks:
         from . import rm
         self.rm = rm
 
-    def block_fwd(self, q, k, v, *, N, P, layout, causal, q_rank, kv_rank, scale):
+    def block_fwd(self, q, k, v, *, N, P, layout, causal, q_rank, kv_rank, scale, segs):
         return self.rm.attn_block_fwd(q, k, v, N=N, P=P, layout=layout, causal=causal,
-                                      q_rank=q_rank, kv_rank=kv_rank, scale=scale, o_f32=True)
+                                      q_rank=q_rank, kv_rank=kv_rank, scale=scale, o_f32=True,
+                                      **segs)
 
     def merge_into(self, o_acc, lse_acc, o_new, lse_new):
         self.rm.lse_merge([o_acc, o_new], [lse_acc, lse_new], torch.float32, out=o_acc,
@@ -72,9 +73,9 @@ class KernelBlocks:
         return self.rm.attn_bwd_preprocess(o, dout)
 
     def block_bwd(self, q, k, v, dout, lse, delta, dq, dk, dv, *, N, P, layout, causal, q_rank,
-                  kv_rank, scale):
+                  kv_rank, scale, segs):
         self.rm.attn_block_bwd(q, k, v, dout, lse, delta, dq, dk, dv, N=N, P=P, layout=layout,
-                               causal=causal, q_rank=q_rank, kv_rank=kv_rank, scale=scale)
+                               causal=causal, q_rank=q_rank, kv_rank=kv_rank, scale=scale, **segs)
 
     def cast(self, acc, dtype):
         if dtype == torch.float32:
@@ -109,8 +110,15 @@ def _wait(reqs):
         r.wait()
 
 
-def ring_forward(q, k, v, *, layout: str, causal: bool, scale=None, group=None, blocks=None):
-    """This rank's (O [B, L, Hq, d] in q's dtype, LSE fp32 [B, Hq, L])."""
+def ring_forward(q, k, v, *, layout: str, causal: bool, scale=None, group=None, blocks=None,
+                 cu_seqlens=None, seq_lens=None):
+    """This rank's (O [B, L, Hq, d] in q's dtype, LSE fp32 [B, Hq, L]).
+
+    cu_seqlens (packing boundaries in global positions, B = 1) or seq_lens
+    (right-padding lengths per batch entry), int32, on the operands' device,
+    the same on every rank: as in the single-GPU ring, a key is visible only
+    inside its query's segment."""
+    segs = {"cu_seqlens": cu_seqlens, "seq_lens": seq_lens}
     blocks = KernelBlocks() if blocks is None else blocks
     P = dist.get_world_size(group)
     r = dist.get_rank(group)
@@ -128,19 +136,22 @@ def ring_forward(q, k, v, *, layout: str, causal: bool, scale=None, group=None, 
         reqs = _exchange(cur, bufs[step % 2], dst, src, group) if step + 1 < P else []
         if not pair_is_empty(layout, N, P, r, s, causal):
             o_s, lse_s = blocks.block_fwd(q, cur[0], cur[1], N=N, P=P, layout=layout,
-                                          causal=causal, q_rank=r, kv_rank=s, scale=scale)
+                                          causal=causal, q_rank=r, kv_rank=s, scale=scale,
+                                          segs=segs)
             if o_acc is None:
                 o_acc, lse_acc = o_s, lse_s
             else:
                 blocks.merge_into(o_acc, lse_acc, o_s, lse_s)
         _wait(reqs)
-    # the pair (r, r) always holds the diagonal, so o_acc is set
+    # the pair (r, r) is never skipped, so o_acc is set
     return blocks.finish(o_acc, lse_acc, q.dtype), lse_acc
 
 
 def ring_backward(q, k, v, o, lse, dout, *, layout: str, causal: bool, scale=None, group=None,
-                  blocks=None):
-    """This rank's (dQ, dK, dV) in the operands' dtypes, from the final O and LSE."""
+                  blocks=None, cu_seqlens=None, seq_lens=None):
+    """This rank's (dQ, dK, dV) in the operands' dtypes, from the final O and
+    LSE (segments as in ring_forward)."""
+    segs = {"cu_seqlens": cu_seqlens, "seq_lens": seq_lens}
     blocks = KernelBlocks() if blocks is None else blocks
     P = dist.get_world_size(group)
     r = dist.get_rank(group)
@@ -162,7 +173,8 @@ def ring_backward(q, k, v, o, lse, dout, *, layout: str, causal: bool, scale=Non
         kv_reqs = _exchange(kv, bufs[step % 2], dst, src, group) if step + 1 < P else []
         if not pair_is_empty(layout, N, P, r, s, causal):
             blocks.block_bwd(q, kv[0], kv[1], dout, lse, delta, dq, acc[0], acc[1], N=N, P=P,
-                             layout=layout, causal=causal, q_rank=r, kv_rank=s, scale=scale)
+                             layout=layout, causal=causal, q_rank=r, kv_rank=s, scale=scale,
+                             segs=segs)
         if P > 1:
             # after the last step shard s sits on rank s - 1: this transfer
             # returns every shard's dK / dV to its owner.  (The transfers are

@@ -207,10 +207,11 @@ def lse_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor]
 
 def attn_block_fwd(q, k, v, *, N: int, P: int, layout: str, causal: bool, q_rank: int,
                    kv_rank: int, scale: float | None = None, o_f32: bool = False, out=None,
-                   lse=None, stream=None):
+                   lse=None, stream=None, cu_seqlens=None, seq_lens=None):
     """One Q shard [B, L, Hq, d] against one KV shard [B, L, Hkv, d] -> (O, LSE)."""
     B, L, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     odt = torch.float32 if (o_f32 or q.dtype == torch.float32) else q.dtype
     out = torch.empty((B, L, Hq, d), dtype=odt, device=q.device) if out is None else out
     lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -221,10 +222,11 @@ def attn_block_fwd(q, k, v, *, N: int, P: int, layout: str, causal: bool, q_rank
 
 def attn_block_bwd(q, k, v, dout, lse_final, delta, dq_acc, dk_acc, dv_acc, *, N: int, P: int,
                    layout: str, causal: bool, q_rank: int, kv_rank: int,
-                   scale: float | None = None, stream=None):
+                   scale: float | None = None, stream=None, cu_seqlens=None, seq_lens=None):
     """Accumulate one shard pair's gradients into fp32 dq_acc / dk_acc / dv_acc."""
     B, L, Hq, d = q.shape
-    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale)
+    dsc = desc(q.dtype, B, Hq, k.shape[2], d, N, P, layout, causal, scale,
+               cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     _check(_lib.rm_attn_block_bwd(ctypes.byref(dsc), q_rank, kv_rank, _bnhd(q), _bnhd(k), _bnhd(v),
                                   _bnhd(dout), _ptr(lse_final), _ptr(delta), _bnhd(dq_acc),
                                   _bnhd(dk_acc), _bnhd(dv_acc), _stream(stream)))

@@ -111,37 +111,50 @@ def _run_ranks(world, fn):
 
 
 CASES = [
-    # dtype, B, Hq, Hkv, N, d, P, layout, causal
-    (torch.bfloat16, 1, 4, 2, 2048, 128, 4, "zigzag", True),
-    (torch.bfloat16, 1, 4, 2, 2048, 128, 2, "zigzag", True),
-    (torch.bfloat16, 2, 2, 1, 1536, 128, 3, "striped", True),
-    (torch.bfloat16, 1, 2, 2, 1024, 128, 4, "contiguous", True),
-    (torch.bfloat16, 1, 4, 2, 768, 64, 2, "contiguous", False),
-    (torch.float32, 1, 2, 1, 512, 64, 4, "zigzag", True),
+    # dtype, B, Hq, Hkv, N, d, P, layout, causal, segments
+    (torch.bfloat16, 1, 4, 2, 2048, 128, 4, "zigzag", True, None),
+    (torch.bfloat16, 1, 4, 2, 2048, 128, 2, "zigzag", True, None),
+    (torch.bfloat16, 2, 2, 1, 1536, 128, 3, "striped", True, None),
+    (torch.bfloat16, 1, 2, 2, 1024, 128, 4, "contiguous", True, None),
+    (torch.bfloat16, 1, 4, 2, 768, 64, 2, "contiguous", False, None),
+    (torch.float32, 1, 2, 1, 512, 64, 4, "zigzag", True, None),
+    # packed: boundaries inside shards and across them; right padding with a
+    # one-token entry
+    (torch.bfloat16, 1, 4, 2, 2048, 128, 4, "zigzag", True, ("packed", [0, 1, 700, 1300, 2040, 2048])),
+    (torch.float32, 3, 2, 1, 512, 64, 2, "striped", True, ("padded", [1, 512, 300])),
 ]
 
 
-@pytest.mark.parametrize("dtype,B,Hq,Hkv,N,d,P,layout,causal", CASES)
-def test_ring_dist_schedule_on_the_kernels(dtype, B, Hq, Hkv, N, d, P, layout, causal):
+@pytest.mark.parametrize("dtype,B,Hq,Hkv,N,d,P,layout,causal,segments", CASES)
+def test_ring_dist_schedule_on_the_kernels(dtype, B, Hq, Hkv, N, d, P, layout, causal, segments):
     seed = 7000 + N + P
     q = synthetic.tensor(seed, (B, N, Hq, d), dtype)
     k = synthetic.tensor(seed + 1, (B, N, Hkv, d), dtype)
     v = synthetic.tensor(seed + 2, (B, N, Hkv, d), dtype)
     do = synthetic.tensor(seed + 3, (B, N, Hq, d), dtype)
     pos = [olay.rank_positions(layout, N, P, r) for r in range(P)]
+    segs, seg = {}, None
+    if segments is not None:
+        kind, vals = segments
+        t32 = torch.tensor(vals, dtype=torch.int32, device="cuda")
+        if kind == "packed":
+            segs, seg = {"cu_seqlens": t32}, oatt.segments_from_boundaries(np.array(vals), N)
+        else:
+            segs, seg = {"seq_lens": t32}, oatt.segments_from_lengths(np.array(vals), N)
     shard = lambda x, r: x[:, torch.from_numpy(pos[r])].contiguous().cuda()
 
     def rank(r):
         qr, kr, vr, dor = shard(q, r), shard(k, r), shard(v, r), shard(do, r)
         kept = [x.clone() for x in (qr, kr, vr, dor)]
-        o, lse = ring_dist.ring_forward(qr, kr, vr, layout=layout, causal=causal)
-        grads = ring_dist.ring_backward(qr, kr, vr, o, lse, dor, layout=layout, causal=causal)
+        o, lse = ring_dist.ring_forward(qr, kr, vr, layout=layout, causal=causal, **segs)
+        grads = ring_dist.ring_backward(qr, kr, vr, o, lse, dor, layout=layout, causal=causal,
+                                        **segs)
         assert all(torch.equal(a, b) for a, b in zip((qr, kr, vr, dor), kept)), "inputs written"
         return o, lse, grads
 
     out = _run_ranks(P, rank)
-    o_ref, l_ref = oatt.attention_forward(np64(q), np64(k), np64(v), causal=causal)
-    g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=causal)
+    o_ref, l_ref = oatt.attention_forward(np64(q), np64(k), np64(v), causal=causal, seg=seg)
+    g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=causal, seg=seg)
     o_tol, l_tol = (F32_TOL, F32_TOL) if dtype == torch.float32 else (BF16_O_TOL, BF16_LSE_TOL)
     g_tol = F32_TOL if dtype == torch.float32 else None
     for r, (o, lse, grads) in enumerate(out):

@@ -36,10 +36,18 @@ class OracleBlocks:
     def _pos(self, layout, N, P, r):
         return self.lay.rank_positions(layout, N, P, r)
 
-    def block_fwd(self, q, k, v, *, N, P, layout, causal, q_rank, kv_rank, scale):
+    def _seg(self, segs, N):
+        if segs["cu_seqlens"] is not None:
+            return self.att.segments_from_boundaries(segs["cu_seqlens"].numpy(), N)
+        if segs["seq_lens"] is not None:
+            return self.att.segments_from_lengths(segs["seq_lens"].numpy(), N)
+        return None
+
+    def block_fwd(self, q, k, v, *, N, P, layout, causal, q_rank, kv_rank, scale, segs):
         o, l = self.att.attention_forward(q.numpy(), k.numpy(), v.numpy(), scale, causal,
                                           q_pos=self._pos(layout, N, P, q_rank),
-                                          k_pos=self._pos(layout, N, P, kv_rank))
+                                          k_pos=self._pos(layout, N, P, kv_rank),
+                                          seg=self._seg(segs, N))
         return torch.from_numpy(o), torch.from_numpy(l)
 
     def merge_into(self, o_acc, lse_acc, o_new, lse_new):
@@ -54,11 +62,12 @@ class OracleBlocks:
         return torch.from_numpy(self.att.delta_from_output(dout.numpy(), o.numpy()))
 
     def block_bwd(self, q, k, v, dout, lse, delta, dq, dk, dv, *, N, P, layout, causal, q_rank,
-                  kv_rank, scale):
+                  kv_rank, scale, segs):
         g = self.att.attention_backward_block(q.numpy(), k.numpy(), v.numpy(), dout.numpy(),
                                               lse.numpy(), delta.numpy(), scale, causal,
                                               q_pos=self._pos(layout, N, P, q_rank),
-                                              k_pos=self._pos(layout, N, P, kv_rank))
+                                              k_pos=self._pos(layout, N, P, kv_rank),
+                                              seg=self._seg(segs, N))
         for acc, x in zip((dq, dk, dv), g):
             acc += torch.from_numpy(x)
 
@@ -66,7 +75,19 @@ class OracleBlocks:
         return acc.to(dtype)
 
 
-def _rank_main(rank, world, port, out_dir, layout, causal, hq, hkv):
+def _segments(kind, N, B):
+    """Seeded segment descriptions: packed boundaries (B = 1) or right-padding
+    lengths (one entry empty but one token, one full)."""
+    if kind == "packed":
+        cuts = sorted({0, N, 1, N // 3, N // 3 + 5, N - 2})
+        return {"cu_seqlens": torch.tensor(cuts, dtype=torch.int32), "seq_lens": None}
+    if kind == "padded":
+        lens = [1, N, N // 2 + 3][:B]
+        return {"cu_seqlens": None, "seq_lens": torch.tensor(lens, dtype=torch.int32)}
+    return {"cu_seqlens": None, "seq_lens": None}
+
+
+def _rank_main(rank, world, port, out_dir, layout, causal, hq, hkv, segkind="none"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -75,24 +96,31 @@ def _rank_main(rank, world, port, out_dir, layout, causal, hq, hkv):
     from sequence_attention_rm_b200 import ring_dist
     dist.init_process_group("gloo", rank=rank, world_size=world)
     N = 8 * world if layout != "zigzag" else 16 * world
+    B = 1 if segkind == "packed" else 2
     g = torch.Generator().manual_seed(1234)
-    q, k, v, do = (torch.randn(2, N, h, 8, generator=g, dtype=torch.float64)
+    q, k, v, do = (torch.randn(B, N, h, 8, generator=g, dtype=torch.float64)
                    for h in (hq, hkv, hkv, hq))
+    segs = _segments(segkind, N, B)
+    seg = OracleBlocks()._seg(segs, N)
     pos = layouts.rank_positions(layout, N, world, rank)
     shard = lambda x: x[:, torch.from_numpy(pos)].contiguous()
     blocks = OracleBlocks()
     mine = [shard(x) for x in (q, k, v, do)]
     kept = [x.clone() for x in mine]
     qr, kr, vr, dor = mine
-    o, lse = ring_dist.ring_forward(qr, kr, vr, layout=layout, causal=causal, blocks=blocks)
+    o, lse = ring_dist.ring_forward(qr, kr, vr, layout=layout, causal=causal, blocks=blocks,
+                                    **segs)
     grads = ring_dist.ring_backward(qr, kr, vr, o, lse, dor, layout=layout, causal=causal,
-                                    blocks=blocks)
-    o_ref, l_ref = attention.attention_forward(q.numpy(), k.numpy(), v.numpy(), causal=causal)
+                                    blocks=blocks, **segs)
+    o_ref, l_ref = attention.attention_forward(q.numpy(), k.numpy(), v.numpy(), causal=causal,
+                                               seg=seg)
     g_ref = attention.attention_backward(q.numpy(), k.numpy(), v.numpy(), do.numpy(),
-                                         causal=causal)
+                                         causal=causal, seg=seg)
     err = {
         "o": float(np.abs(o.numpy() - o_ref[:, pos]).max()),
-        "lse": float(np.abs(lse.numpy() - l_ref[:, :, pos]).max()),
+        "lse": float(np.nanmax(np.where(np.isneginf(l_ref[:, :, pos]) &
+                                        np.isneginf(lse.numpy()), 0.0,
+                                        np.abs(lse.numpy() - l_ref[:, :, pos])))),
     }
     for name, got, ref in zip(("dq", "dk", "dv"), grads, g_ref):
         err[name] = float(np.abs(got.numpy() - ref[:, pos]).max())
@@ -104,12 +132,15 @@ def _rank_main(rank, world, port, out_dir, layout, causal, hq, hkv):
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("world,layout,causal,hq,hkv", [
-    (2, "zigzag", True, 4, 2), (3, "striped", True, 2, 1), (4, "contiguous", True, 2, 2),
-    (2, "contiguous", False, 2, 1), (4, "zigzag", True, 2, 1), (3, "contiguous", True, 4, 2)])
-def test_ring_over_gloo_ranks_equals_unsharded(tmp_path, world, layout, causal, hq, hkv):
-    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), layout, causal, hq, hkv),
-             nprocs=world, join=True)
+@pytest.mark.parametrize("world,layout,causal,hq,hkv,segkind", [
+    (2, "zigzag", True, 4, 2, "none"), (3, "striped", True, 2, 1, "none"),
+    (4, "contiguous", True, 2, 2, "none"), (2, "contiguous", False, 2, 1, "none"),
+    (4, "zigzag", True, 2, 1, "none"), (3, "contiguous", True, 4, 2, "none"),
+    (3, "zigzag", True, 2, 1, "packed"), (2, "striped", False, 2, 2, "padded")])
+def test_ring_over_gloo_ranks_equals_unsharded(tmp_path, world, layout, causal, hq, hkv,
+                                                segkind):
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), layout, causal, hq, hkv,
+                               segkind), nprocs=world, join=True)
     for r in range(world):
         err = json.load(open(tmp_path / f"rank{r}.json"))
         for name, e in err.items():
