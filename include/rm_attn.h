@@ -180,12 +180,17 @@ rm_status rm_attn_bwd_preprocess(rm_dtype dtype, int B, int64_t N, int H, int d,
                                  rm_tensor o, rm_tensor dout, float* delta,
                                  void* stream);
 
-/* fp32 [B, N, H, d] -> out_dtype [B, N, H, d] (bf16: round to nearest even;
- * fp32: a copy), both strided as rm_tensor (d contiguous): the last step of a
- * backward that accumulated its gradients in fp32 (the block API's
- * accumulators; the distributed ring, whose dK / dV accumulators travel
- * between ranks in fp32).  d % 4 == 0, pointers and strides aligned to 4
- * elements; in and out must not overlap. */
+/* Backward finalize [ringmaster, "Status": the ring backward, whose dK / dV
+ * travel round the ring with their KV shard and come back to its owner]:
+ * fp32 [B, N, H, d] -> out_dtype [B, N, H, d] (bf16: round to nearest even;
+ * fp32: a copy), both strided as rm_tensor (d contiguous), for a backward that
+ * accumulated its gradients in fp32 (the block API's accumulators; the
+ * multi-rank ring, whose dK / dV accumulators cross ranks in fp32).
+ * The caller owns both buffers; in and out must not overlap.
+ * Errors: RM_ERR_INVALID_ARG for another out_dtype, B < 0, N < 0, H < 1,
+ * d < 4 or d % 4 != 0, a NULL pointer, or pointers / strides not aligned to
+ * 4 elements (16 bytes of fp32 input; 8 bytes of bf16 output).  B * N == 0
+ * launches nothing. */
 rm_status rm_convert_f32(rm_dtype out_dtype, int B, int64_t N, int H, int d, rm_tensor in,
                          rm_tensor out, void* stream);
 

@@ -145,6 +145,18 @@ def test_entry_points_reject_bad_arguments_before_launch(rm):
                                 nul) == 3
     # block forward: rank out of range
     assert lib.rm_attn_block_fwd(ctypes.byref(d), 2, 0, ok, kv, kv, ok, 0, p, nul) == 1
+    # fp32 -> out dtype conversion: dtype, sizes, NULL, alignment; empty is a no-op
+    src = T(p.value, 256 * 16 * 128, 16 * 128, 128)
+    dst = T(p.value + 2048, 256 * 16 * 128, 16 * 128, 128)
+    assert lib.rm_convert_f32(2, 1, 256, 16, 128, src, dst, nul) == 1  # no dtype 2
+    assert lib.rm_convert_f32(1, 1, 256, 16, 126, src, dst, nul) == 1  # d % 4
+    assert lib.rm_convert_f32(1, 1, 256, 0, 128, src, dst, nul) == 1  # H < 1
+    assert lib.rm_convert_f32(1, 1, 256, 16, 128, T(0, 0, 0, 0), dst, nul) == 1  # NULL
+    assert lib.rm_convert_f32(1, 1, 256, 16, 128, T(p.value + 4, 256 * 16 * 128, 16 * 128, 128),
+                              dst, nul) == 1  # fp32 input off a 16-byte boundary
+    assert lib.rm_convert_f32(1, 1, 256, 16, 128, src, T(p.value + 2, 256 * 16 * 128, 16 * 128,
+                                                         128), nul) == 1  # bf16 output off 8 bytes
+    assert lib.rm_convert_f32(1, 0, 256, 16, 128, T(0, 0, 0, 0), T(0, 0, 0, 0), nul) == 0
 
 
 def test_usp_auto_select_matches_the_rule(rm):
