@@ -2,8 +2,11 @@
 // backward preprocess (delta = rowsum(dO * O)) and the fp32 -> output-dtype
 // finalize.  A "row" is one (b, t, h) vector of d values; a group of
 // d/4 lanes (rounded up to a power of two) owns a row and moves it with
-// 16-byte fp32 vectors.  Rows are enumerated (b, h, t) with t fastest so that
-// the per-row LSE / delta scalars of neighbouring warps share sectors.
+// 16-byte fp32 vectors.  The preprocess and finalize enumerate rows (b, h, t)
+// with t fastest so that the per-row delta scalars of neighbouring warps
+// share sectors; the merge kernels state their own row order.
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -159,6 +162,87 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a, int lanes, 
     carry = x2 >= R2;
     if (carry) x2 -= R2;
     b += st_b + carry;
+  }
+}
+
+// Two parts, d = 128 (one 32-lane warp per row), the running-state merge of
+// the stepwise and multi-rank rings: a warp takes 32 consecutive t of one
+// (b, h).  Lane i reads the two LSE values of row t0 + i (one
+// coalesced load per part), computes the row's weights and new LSE once and
+// writes the LSE back (in place is safe: the lane that writes it read it);
+// the warp then streams the 32 rows U at a time, weights passed by shuffle,
+// all 2U loads of a pass issued before any is used.  The per-row kernel
+// repeats the exp / log chain in every lane between one row's loads and the
+// next (5.82 -> 5.95-5.99 TB/s with the same grid; rows in memory order or 8
+// rows per pass measured no better).  Same arithmetic as lse_merge_kernel, so
+// the same bits.
+constexpr int kMerge2Rows = 4;  // rows per pass
+
+template <typename OutT, int U>
+__global__ void __launch_bounds__(256) merge2_rows_kernel(MergeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int col = lane * 4;
+  const int64_t NC = (a.Nq + 31) / 32;  // 32-token chunks per (b, h)
+  const int64_t chunks = (int64_t)a.B * a.H * NC;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const float skip = __int_as_float(0x7fffffff);  // NaN: the part has weight 0
+  for (int64_t c = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); c < chunks;
+       c += nwarps) {
+    const int64_t bh = c / NC;
+    const int64_t t0 = (c - bh * NC) * 32;
+    const int h = (int)(bh % a.H), b = (int)(bh / a.H);
+    const int rows = (int)(a.Nq - t0 < 32 ? a.Nq - t0 : 32);
+    float c0 = skip, c1 = skip;
+    if (lane < rows) {
+      const int64_t lidx = bh * a.lse_ld + t0 + lane;
+      const float l0 = a.lse_ptr[0][lidx], l1 = a.lse_ptr[1][lidx];
+      const float m = fmaxf(l0, l1);
+      float lse = -INFINITY;
+      if (m != -INFINITY) {
+        const float w0 = expf(l0 - m);  // exp(-inf) = 0 for an empty partial
+        const float w1 = expf(l1 - m);
+        const float sum = 0.f + w0 + w1;
+        const float inv = 1.0f / sum;
+        lse = m + logf(sum);
+        if (w0 != 0.f) c0 = w0 * inv;
+        if (w1 != 0.f) c1 = w1 * inv;
+      }
+      a.lse_out[lidx] = lse;
+    }
+    const float* p0 = a.o_ptr[0] + b * a.o_sb[0] + t0 * a.o_sn[0] + h * a.o_sh[0] + col;
+    const float* p1 = a.o_ptr[1] + b * a.o_sb[1] + t0 * a.o_sn[1] + h * a.o_sh[1] + col;
+    OutT* po = reinterpret_cast<OutT*>(a.out) + b * a.out_sb + t0 * a.out_sn + h * a.out_sh + col;
+    for (int r0 = 0; r0 < rows; r0 += U) {
+      float4 x0[U], x1[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (r0 + u < rows) {
+          x0[u] = load4(p0 + (int64_t)(r0 + u) * a.o_sn[0]);
+          x1[u] = load4(p1 + (int64_t)(r0 + u) * a.o_sn[1]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float k0 = __shfl_sync(0xffffffffu, c0, (r0 + u) & 31);
+        const float k1 = __shfl_sync(0xffffffffu, c1, (r0 + u) & 31);
+        if (r0 + u < rows) {
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (k0 == k0) {
+            acc.x = fmaf(k0, x0[u].x, acc.x);
+            acc.y = fmaf(k0, x0[u].y, acc.y);
+            acc.z = fmaf(k0, x0[u].z, acc.z);
+            acc.w = fmaf(k0, x0[u].w, acc.w);
+          }
+          if (k1 == k1) {
+            acc.x = fmaf(k1, x1[u].x, acc.x);
+            acc.y = fmaf(k1, x1[u].y, acc.y);
+            acc.z = fmaf(k1, x1[u].z, acc.z);
+            acc.w = fmaf(k1, x1[u].w, acc.w);
+          }
+          store4(po + (int64_t)(r0 + u) * a.out_sn, acc);
+        }
+      }
+    }
   }
 }
 
@@ -339,6 +423,20 @@ cudaError_t launch_lse_merge(const MergeArgs& a, int out_bf16, cudaStream_t stre
   for (int i = 1; i < a.n_parts; ++i)
     same = same && a.o_sb[i] == a.o_sb[0] && a.o_sn[i] == a.o_sn[0] && a.o_sh[i] == a.o_sh[0];
   ProfScope ps("lse_merge", stream);
+  if (a.n_parts == 2 && a.d == 128) {
+    // one chunk per warp, blocks scheduled as SMs free up: on the 2-part
+    // in-place merge of [1, 131072, 16, 128] fp32 this ran at 6.35-6.38 TB/s
+    // against 5.93-5.98 for a single wave of resident blocks that loop over
+    // the chunks (whose SMs finish unevenly)
+    const int64_t chunks = (int64_t)a.B * a.H * ((a.Nq + 31) / 32);
+    const int grid = (int)((chunks + 7) / 8 < INT_MAX ? (chunks + 7) / 8 : INT_MAX);
+    if (out_bf16) {
+      merge2_rows_kernel<__nv_bfloat16, kMerge2Rows><<<grid, 256, 0, stream>>>(a);
+    } else {
+      merge2_rows_kernel<float, kMerge2Rows><<<grid, 256, 0, stream>>>(a);
+    }
+    return cudaGetLastError();
+  }
   if (same)
     return out_bf16 ? merge_order<__nv_bfloat16, true>(a, g, rows, stream)
                     : merge_order<float, true>(a, g, rows, stream);

@@ -86,7 +86,8 @@ def test_repack_workload_shapes(rm, L):
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("n,B,H,Nq,d", [(1, 1, 2, 5, 8), (2, 1, 3, 77, 64), (4, 2, 4, 130, 128),
-                                        (8, 1, 16, 300, 128), (3, 1, 2, 33, 24), (16, 1, 1, 9, 4)])
+                                        (8, 1, 16, 300, 128), (3, 1, 2, 33, 24), (16, 1, 1, 9, 4),
+                                        (2, 2, 3, 77, 128), (2, 1, 2, 31, 128)])
 def test_lse_merge(rm, out_dtype, n, B, H, Nq, d):
     o_parts = [synthetic.tensor(300 + i, (B, Nq, H, d)) for i in range(n)]
     lse_parts = [synthetic.tensor(400 + i, (B, H, Nq), scale=3.0) for i in range(n)]
@@ -153,11 +154,12 @@ def test_launch_profiler_records_each_launch(rm):
     assert rm.profile_records() == []  # disabled: nothing recorded
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_lse_merge_mixed_strides(rm, out_dtype):
+def test_lse_merge_mixed_strides(rm, out_dtype, d):
     """Partials whose strides differ (a head view of a wider tensor, a dense
     tensor) and an output view with its own strides."""
-    B, Nq, H, d = 2, 301, 3, 64
+    B, Nq, H = 2, 301, 3
     wide = synthetic.tensor(920, (B, Nq, H + 2, d)).cuda()
     o_parts = [wide[:, :, 1:1 + H], synthetic.tensor(921, (B, Nq, H, d)).cuda()]
     lse_parts = [synthetic.tensor(930 + i, (B, H, Nq), scale=3.0).cuda() for i in range(2)]
