@@ -259,12 +259,29 @@ def ring_workspace_size(dsc: RmAttnDesc, backward: bool) -> int:
     return n.value
 
 
-def _workspace(nbytes: int, device, ws: torch.Tensor | None):
-    if nbytes == 0:
-        return ctypes.c_void_p(0), 0
-    if ws is None or ws.numel() * ws.element_size() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+class _Workspace:
+    """The workspace of one call: the caller's tensor or one allocated here,
+    held until the call has queued its kernels.  A tensor allocated here is
+    only referenced through this object, so the allocator could hand its
+    memory to another allocation (another thread's, or one on another
+    stream) before the kernels that use it are queued if it were dropped
+    earlier; on a stream other than the current one it is also recorded on
+    that stream, so that its memory is not reused before that stream's work
+    is done."""
+
+    def __init__(self, nbytes: int, device, ws: torch.Tensor | None):
+        if nbytes == 0:
+            self.tensor, self.ptr, self.nbytes = None, ctypes.c_void_p(0), 0
+            return
+        if ws is None or ws.numel() * ws.element_size() < nbytes:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.tensor = ws
+        self.ptr, self.nbytes = ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+    def done(self, stream) -> None:
+        """Call after the library call returned (its kernels are queued)."""
+        if self.tensor is not None and stream is not None:
+            self.tensor.record_stream(stream)
 
 
 def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | None = None,
@@ -278,9 +295,10 @@ def ring_attn_fwd(q, k, v, *, P: int, layout: str, causal: bool, scale: float | 
                cu_seqlens, seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    wp, wn = _workspace(ring_workspace_size(dsc, False), q.device, ws)
+    w = _Workspace(ring_workspace_size(dsc, False), q.device, ws)
     _check(_lib.rm_ring_attn_fwd(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(out),
-                                 _ptr(lse), wp, wn, _stream(stream)))
+                                 _ptr(lse), w.ptr, w.nbytes, _stream(stream)))
+    w.done(stream)
     return out, lse
 
 
@@ -294,10 +312,11 @@ def ring_attn_bwd(q, k, v, o, lse, dout, *, P: int, layout: str, causal: bool,
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
-    wp, wn = _workspace(ring_workspace_size(dsc, True), q.device, ws)
+    w = _Workspace(ring_workspace_size(dsc, True), q.device, ws)
     _check(_lib.rm_ring_attn_bwd(ctypes.byref(dsc), _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
-                                 _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
+                                 _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), w.ptr, w.nbytes,
                                  _stream(stream)))
+    w.done(stream)
     return dq, dk, dv
 
 
@@ -340,9 +359,10 @@ def usp_attn_fwd(q, k, v, *, P: int, ulysses: int, layout: str, causal: bool,
                cu_seqlens, seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    wp, wn = _workspace(usp_workspace_size(dsc, ulysses, False), q.device, ws)
+    w = _Workspace(usp_workspace_size(dsc, ulysses, False), q.device, ws)
     _check(_lib.rm_usp_attn_fwd(ctypes.byref(dsc), ulysses, _bnhd(q), _bnhd(k), _bnhd(v),
-                                _bnhd(out), _ptr(lse), wp, wn, _stream(stream)))
+                                _bnhd(out), _ptr(lse), w.ptr, w.nbytes, _stream(stream)))
+    w.done(stream)
     return out, lse
 
 
@@ -356,10 +376,11 @@ def usp_attn_bwd(q, k, v, o, lse, dout, *, P: int, ulysses: int, layout: str, ca
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
-    wp, wn = _workspace(usp_workspace_size(dsc, ulysses, True), q.device, ws)
+    w = _Workspace(usp_workspace_size(dsc, ulysses, True), q.device, ws)
     _check(_lib.rm_usp_attn_bwd(ctypes.byref(dsc), ulysses, _bnhd(q), _bnhd(k), _bnhd(v), _bnhd(o),
-                                _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), wp, wn,
+                                _ptr(lse), _bnhd(dout), _bnhd(dq), _bnhd(dk), _bnhd(dv), w.ptr, w.nbytes,
                                 _stream(stream)))
+    w.done(stream)
     return dq, dk, dv
 
 
@@ -380,9 +401,10 @@ def mesh2d_attn_fwd(q, k, v, *, grid_q: int, grid_k: int, causal: bool,
                cu_seqlens=cu_seqlens, seq_lens=seq_lens)
     out = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    wp, wn = _workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, False), q.device, ws)
+    w = _Workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, False), q.device, ws)
     _check(_lib.rm_mesh2d_attn_fwd(ctypes.byref(dsc), grid_q, grid_k, _bnhd(q), _bnhd(k),
-                                   _bnhd(v), _bnhd(out), _ptr(lse), wp, wn, _stream(stream)))
+                                   _bnhd(v), _bnhd(out), _ptr(lse), w.ptr, w.nbytes, _stream(stream)))
+    w.done(stream)
     return out, lse
 
 
@@ -396,10 +418,11 @@ def mesh2d_attn_bwd(q, k, v, o, lse, dout, *, grid_q: int, grid_k: int, causal: 
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
-    wp, wn = _workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, True), q.device, ws)
+    w = _Workspace(mesh2d_workspace_size(dsc, grid_q, grid_k, True), q.device, ws)
     _check(_lib.rm_mesh2d_attn_bwd(ctypes.byref(dsc), grid_q, grid_k, _bnhd(q), _bnhd(k),
                                    _bnhd(v), _bnhd(o), _ptr(lse), _bnhd(dout), _bnhd(dq),
-                                   _bnhd(dk), _bnhd(dv), wp, wn, _stream(stream)))
+                                   _bnhd(dk), _bnhd(dv), w.ptr, w.nbytes, _stream(stream)))
+    w.done(stream)
     return dq, dk, dv
 
 
