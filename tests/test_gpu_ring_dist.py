@@ -2,18 +2,13 @@
 kernels, on one GPU.
 
 The ranks are threads of this process and the point-to-point transfers go
-through an in-process stand-in for torch.distributed's P2P calls: a send
-queues a device copy of its tensor, a receive copies it into its buffer when
-waited on.  Every transfer is a host hand-off of stream-ordered copies, so no
-kernel ever waits for another rank's kernel.  What this checks is the kernel
+through an in-process stand-in for torch.distributed's P2P calls
+(``tests/_thread_ranks.py``: host hand-offs of stream-ordered copies, so no
+kernel ever waits for another rank's kernel).  What this checks is the kernel
 side of the schedule (the fp32 partials merged in place, the travelling fp32
 dK / dV accumulators, the final casts); the transfers themselves are checked
 over real gloo ranks on the CPU.  Results are compared with the unsharded
 fp64 oracle."""
-
-import queue
-import threading
-import types
 
 import numpy as np
 import pytest
@@ -24,90 +19,9 @@ from oracle import layouts as olay
 from sequence_attention_rm_b200 import ring_dist, synthetic
 from tests._helpers import (BF16_LSE_TOL, BF16_O_TOL, F32_TOL, assert_grad_close, assert_max_abs,
                             gpu, np64)
+from tests._thread_ranks import run_ranks
 
 pytestmark = gpu
-
-
-class _Req:
-    def __init__(self, fn=None):
-        self.fn = fn
-
-    def wait(self):
-        if self.fn is not None:
-            self.fn()
-
-
-class ThreadRanks:
-    """torch.distributed's point-to-point surface for P threads of one
-    process.  As in the real backends, the n-th receive a rank posts from a
-    peer matches the n-th send that peer posted to it, whatever order the
-    requests are waited on."""
-
-    def __init__(self, world):
-        self.world = world
-        self.local = threading.local()
-        self.lock = threading.Lock()
-        self.slots = {}
-        self.posted = {}
-        self.isend, self.irecv = "isend", "irecv"
-
-    def P2POp(self, op, tensor, peer, group=None):
-        return types.SimpleNamespace(op=op, tensor=tensor, peer=peer)
-
-    def get_world_size(self, group=None):
-        return self.world
-
-    def get_rank(self, group=None):
-        return self.local.rank
-
-    def get_global_rank(self, group, r):
-        return r
-
-    def _slot(self, key):
-        """The queue of the next message on a (src, dst, direction) counter."""
-        with self.lock:
-            n = self.posted.get(key, 0)
-            self.posted[key] = n + 1
-            return self.slots.setdefault(key[:2] + (n,), queue.Queue(maxsize=1))
-
-    def batch_isend_irecv(self, ops):
-        me = self.local.rank
-        reqs = []
-        for op in ops:
-            if op.op == self.isend:
-                self._slot((me, op.peer, "send")).put(op.tensor.clone())
-                reqs.append(_Req())
-            else:
-                slot, buf = self._slot((op.peer, me, "recv")), op.tensor
-                reqs.append(_Req(lambda slot=slot, buf=buf: buf.copy_(slot.get(timeout=120))))
-        return reqs
-
-
-def _run_ranks(world, fn):
-    fake = ThreadRanks(world)
-    results, errors = [None] * world, []
-
-    def body(r):
-        fake.local.rank = r
-        try:
-            results[r] = fn(r)
-        except BaseException as e:  # reported by the main thread
-            errors.append(e)
-
-    real = ring_dist.dist
-    ring_dist.dist = fake
-    try:
-        threads = [threading.Thread(target=body, args=(r,)) for r in range(world)]
-        for t in threads:
-            t.start()
-        for t in threads:
-            t.join(timeout=300)
-        torch.cuda.synchronize()
-    finally:
-        ring_dist.dist = real
-    if errors:
-        raise errors[0]
-    return results
 
 
 CASES = [
@@ -152,7 +66,7 @@ def test_ring_dist_schedule_on_the_kernels(dtype, B, Hq, Hkv, N, d, P, layout, c
         assert all(torch.equal(a, b) for a, b in zip((qr, kr, vr, dor), kept)), "inputs written"
         return o, lse, grads
 
-    out = _run_ranks(P, rank)
+    out = run_ranks(ring_dist, P, rank)
     o_ref, l_ref = oatt.attention_forward(np64(q), np64(k), np64(v), causal=causal, seg=seg)
     g_ref = oatt.attention_backward(np64(q), np64(k), np64(v), np64(do), causal=causal, seg=seg)
     o_tol, l_tol = (F32_TOL, F32_TOL) if dtype == torch.float32 else (BF16_O_TOL, BF16_LSE_TOL)
