@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "rm_attn.h")
@@ -223,3 +224,40 @@ def test_mesh2d_workspace_sizes(rm):
     assert n.value == 8 * o_slot + 8 * lse_slot
     assert rm.raw().rm_mesh2d_workspace_size(ctypes.byref(d), 4, 8, 1, ctypes.byref(n)) == 0
     assert n.value == lse_slot + o_slot + 2 * (16384 * 8 * 128 * 4)
+
+
+def test_call_workspace_is_held_and_recorded(rm):
+    """A workspace the binding allocates is referenced by the call's holder
+    (so it outlives the library call that queues kernels on it), a caller's
+    large-enough tensor is used as given, and the tensor is recorded on a
+    stream the caller names (not on the current one)."""
+    w = rm._Workspace(0, "cpu", None)
+    assert w.tensor is None and w.nbytes == 0 and not w.ptr.value
+    w = rm._Workspace(64, "cpu", None)
+    assert w.tensor is not None and w.nbytes == 64 and w.ptr.value == w.tensor.data_ptr()
+
+    class Caller:
+        def __init__(self, n):
+            self.buf, self.streams = torch.empty(n, dtype=torch.uint8), []
+
+        def numel(self):
+            return self.buf.numel()
+
+        def element_size(self):
+            return 1
+
+        def data_ptr(self):
+            return self.buf.data_ptr()
+
+        def record_stream(self, s):
+            self.streams.append(s)
+
+    mine = Caller(128)
+    w = rm._Workspace(100, "cpu", mine)
+    assert w.tensor is mine and w.nbytes == 128
+    w.done(None)
+    assert mine.streams == []
+    w.done("side stream")
+    assert mine.streams == ["side stream"]
+    small = Caller(8)
+    assert rm._Workspace(100, "cpu", small).tensor is not small  # too small: one of its own
