@@ -155,3 +155,46 @@ def test_empty_pairs_are_the_contiguous_future_shards():
     assert not pair_is_empty("contiguous", 64, 4, 1, 2, False)
     for layout in ("zigzag", "striped"):
         assert not any(pair_is_empty(layout, 64, 4, r, s, True) for r in range(4) for s in range(4))
+
+
+def _absent_rank_main(rank, world, port, out_dir, which):
+    """Every rank but the last joins the exchange; the last never does (it
+    sleeps past the process group's timeout, then exits)."""
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from sequence_attention_rm_b200 import ring_dist, ulysses_dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=3))
+    if rank == world - 1:
+        time.sleep(10)
+        return
+    x = torch.randn(1, 8, 2, 8, dtype=torch.float64)
+    t0 = time.time()
+    try:
+        if which == "ring":
+            ring_dist.ring_forward(x, x, x, layout="contiguous", causal=True, blocks=OracleBlocks())
+        else:
+            from tests.test_ulysses_dist_gloo import OracleOps
+            ulysses_dist.ulysses_forward(x, x, x, layout="contiguous", causal=True, ops=OracleOps())
+        outcome = "returned"
+    except Exception as e:  # the expected path: the exchange times out
+        outcome = f"raised: {type(e).__name__}: {str(e)[:200]}"
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"outcome": outcome, "seconds": time.time() - t0}, f)
+
+
+@pytest.mark.timeout(120)
+@pytest.mark.parametrize("which", ["ring", "ulysses"])
+def test_a_rank_that_never_joins_ends_the_others_with_an_error(tmp_path, which):
+    """Failure made on the host: one rank never reaches the exchange; the
+    others' transfers end with an error after the process group's timeout
+    (3 s) instead of waiting for good."""
+    mp.spawn(_absent_rank_main, args=(2, _free_port(), str(tmp_path), which), nprocs=2,
+             join=True)
+    res = json.load(open(tmp_path / "rank0.json"))
+    assert res["outcome"].startswith("raised"), res
+    assert res["seconds"] < 30, res
