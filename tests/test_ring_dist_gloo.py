@@ -1,4 +1,4 @@
-"""The multi-rank ring (``ring_dist``) on CPU: 2 to 4 gloo ranks, with the
+"""The multi-rank ring (``ring_dist``) on CPU: 1 to 4 gloo ranks, with the
 shard-pair arithmetic supplied by the fp64 oracle instead of the CUDA
 kernels, so that what is checked is the communication schedule (Mosaic, "How
 Ring Attention Works": each device keeps its query chunk and passes KV
@@ -136,7 +136,8 @@ def _rank_main(rank, world, port, out_dir, layout, causal, hq, hkv, segkind="non
     (2, "zigzag", True, 4, 2, "none"), (3, "striped", True, 2, 1, "none"),
     (4, "contiguous", True, 2, 2, "none"), (2, "contiguous", False, 2, 1, "none"),
     (4, "zigzag", True, 2, 1, "none"), (3, "contiguous", True, 4, 2, "none"),
-    (3, "zigzag", True, 2, 1, "packed"), (2, "striped", False, 2, 2, "padded")])
+    (3, "zigzag", True, 2, 1, "packed"), (2, "striped", False, 2, 2, "padded"),
+    (1, "zigzag", True, 2, 1, "none")])
 def test_ring_over_gloo_ranks_equals_unsharded(tmp_path, world, layout, causal, hq, hkv,
                                                 segkind):
     mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), layout, causal, hq, hkv,

@@ -1,4 +1,4 @@
-"""Ulysses attention over real ranks (``ulysses_dist``) on CPU: 2 and 4 gloo
+"""Ulysses attention over real ranks (``ulysses_dist``) on CPU: 1, 2 and 4 gloo
 ranks exchange with all_to_all_single, with the pack / unpack and the
 attention supplied by the fp64 oracle (``oracle/repack.py`` index loops and
 the rank-major ``oracle/ring.py``), so that what is checked is the exchange:
@@ -113,7 +113,7 @@ def _rank_main(rank, world, port, out_dir, layout, causal, B, hq, hkv, segkind):
 @pytest.mark.parametrize("world,layout,causal,B,hq,hkv,segkind", [
     (2, "zigzag", True, 1, 4, 2, "none"), (4, "striped", True, 2, 4, 4, "none"),
     (2, "contiguous", False, 1, 2, 2, "packed"), (4, "contiguous", True, 1, 8, 4, "none"),
-    (2, "zigzag", True, 3, 2, 2, "padded")])
+    (2, "zigzag", True, 3, 2, 2, "padded"), (1, "striped", True, 1, 2, 1, "none")])
 def test_ulysses_over_gloo_ranks_equals_unsharded(tmp_path, world, layout, causal, B, hq, hkv,
                                                    segkind):
     mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), layout, causal, B, hq, hkv,
