@@ -37,14 +37,19 @@ class ThreadRanks:
     def P2POp(self, op, tensor, peer, group=None):
         return types.SimpleNamespace(op=op, tensor=tensor, peer=peer)
 
+    def new_group(self, ranks, backend=None):
+        """A group: its members' global ranks, in group-rank order."""
+        return types.SimpleNamespace(ranks=list(ranks))
+
     def get_world_size(self, group=None):
-        return self.world
+        return self.world if group is None else len(group.ranks)
 
     def get_rank(self, group=None):
-        return self.local.rank
+        me = self.local.rank
+        return me if group is None else group.ranks.index(me)
 
     def get_global_rank(self, group, r):
-        return r
+        return r if group is None else group.ranks[r]
 
     def _slot(self, src, dst, kind, role):
         """The queue of the next message from src to dst of this kind (the
@@ -69,16 +74,19 @@ class ThreadRanks:
 
     def all_to_all_single(self, output, input, group=None):
         me = self.local.rank
-        for dst, chunk in enumerate(input.chunk(self.world)):
+        members = list(range(self.world)) if group is None else group.ranks
+        for dst, chunk in zip(members, input.chunk(len(members))):
             self._slot(me, dst, "a2a", "send").put(chunk.clone())
-        for src, chunk in enumerate(output.chunk(self.world)):
+        for src, chunk in zip(members, output.chunk(len(members))):
             chunk.copy_(self._slot(src, me, "a2a", "recv").get(timeout=120))
 
 
-def run_ranks(module, world, fn):
-    """Run fn(rank) for every rank in its own thread with module.dist replaced
-    by a ThreadRanks; returns the results in rank order."""
-    fake = ThreadRanks(world)
+def run_ranks(module, world, fn, fake=None):
+    """Run fn(rank) for every rank in its own thread with module.dist (a
+    module or a list of modules) replaced by a ThreadRanks; returns the
+    results in rank order."""
+    fake = ThreadRanks(world) if fake is None else fake
+    modules = module if isinstance(module, (list, tuple)) else [module]
     results, errors = [None] * world, []
 
     def body(r):
@@ -88,8 +96,9 @@ def run_ranks(module, world, fn):
         except BaseException as e:  # reported by the caller's thread
             errors.append(e)
 
-    real = module.dist
-    module.dist = fake
+    real = [m.dist for m in modules]
+    for m in modules:
+        m.dist = fake
     try:
         threads = [threading.Thread(target=body, args=(r,)) for r in range(world)]
         for t in threads:
@@ -98,7 +107,8 @@ def run_ranks(module, world, fn):
             t.join(timeout=300)
         torch.cuda.synchronize()
     finally:
-        module.dist = real
+        for m, d in zip(modules, real):
+            m.dist = d
     if errors:
         raise errors[0]
     return results

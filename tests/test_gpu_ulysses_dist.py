@@ -78,3 +78,41 @@ def test_seq_to_head_round_trip_is_the_identity(P, L, H):
         assert torch.equal(back, shards[r])
         want = torch.cat([s[:, :, r * hp:(r + 1) * hp] for s in shards], dim=1)
         assert torch.equal(y, want)
+
+
+def test_real_nccl_group_of_one():
+    """ring_dist and ulysses_dist on a real NCCL process group of one rank
+    (this GPU): the all-to-all runs through NCCL itself and the results
+    equal the single-GPU ring's bit for bit (one rank: the same kernels on
+    the same operands)."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from sequence_attention_rm_b200 import ring_dist, rm
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        q, k, v, do = (synthetic.tensor(8300 + i, (1, 512, h, 128), torch.bfloat16).cuda()
+                       for i, h in enumerate((4, 2, 2, 4)))
+        o_ref, lse_ref = rm.ring_attn_fwd(q, k, v, P=1, layout="contiguous", causal=True)
+        g_ref = rm.ring_attn_bwd(q, k, v, o_ref, lse_ref, do, P=1, layout="contiguous",
+                                 causal=True)
+        o, ctx = ulysses_dist.ulysses_forward(q, k, v, layout="contiguous", causal=True)
+        grads = ulysses_dist.ulysses_backward(do, ctx)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(ctx["lse"], lse_ref)
+        assert all(torch.equal(a, b) for a, b in zip(grads, g_ref))
+        o2, lse2 = ring_dist.ring_forward(q, k, v, layout="contiguous", causal=True)
+        g2 = ring_dist.ring_backward(q, k, v, o2, lse2, do, layout="contiguous", causal=True)
+        torch.cuda.synchronize()
+        # the block path (fp32 partial, then the cast) against the fused ring
+        assert_max_abs(np64(o2), np64(o_ref), BF16_O_TOL, "ring_dist O")
+        for name, a, b in zip(("dQ", "dK", "dV"), g2, g_ref):
+            assert_grad_close(np64(a), np64(b), what=f"ring_dist {name}")
+    finally:
+        dist.destroy_process_group()
