@@ -314,7 +314,7 @@ def time_events(pairs):
 
 
 def tensor_peak(peaks, peak_src, timed_s, clocks):
-    """The bf16 peak a tensor-core kernel is judged against: the burst figure
+    """The bf16 peak a tensor-core kernel is measured against: the burst figure
     (a short region at full clocks), unless the timed region lasted seconds
     and its clock record shows the power-capped regime in which the
     sustained figure was measured (SM clock at most 85% of its maximum under
