@@ -9,7 +9,9 @@ the ranks.  This is the multi-rank form of the single-GPU rm_usp_attn_*:
 
 - the world of W = R * U ranks is R ring positions by U Ulysses positions;
   rank w is ring position w // U and Ulysses position w % U (``usp_groups``
-  builds the U-rank Ulysses groups and the R-rank ring groups);
+  builds the U-rank Ulysses groups and the R-rank ring groups), so a Ulysses
+  group is U consecutive ranks: inside one node when U divides the GPUs per
+  node, the ring crossing nodes, as the page's 2D mesh places them;
 - the sequence is cut into R ring shards by the layout (contiguous, zigzag
   or striped over R), and ring shard r into U contiguous pieces of its local
   order, piece u on rank (r, u);
